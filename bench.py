@@ -1,0 +1,450 @@
+#!/usr/bin/env python
+"""Benchmark: MoE layer forward+backward tokens/s on B200 (one replica per GPU).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload e128_bf16]
+                    [--impl ours|reference] [--router] [--no-cpu-baseline]
+
+One step is one pass of the whole hot path over one batch already resident in HBM:
+routing, dispatch, grouped GEMM forward (FC1 + SwiGLU, FC2), combine, combine
+backward, grouped GEMM backward (two dgrads, two wgrads), unpermute-reduce.  The
+default workload is T=16384 tokens, d=2048, E=128 experts, top-4, d_ff=1024, bf16,
+iid N(0,1) routing logits.  Under torchrun every rank runs its own replica on its own
+GPU (tokens are independent; there is no exchange on the data path): weak scaling.
+
+Prints one JSON line (rank 0).  `--impl reference` times the fp64 CPU oracle on a
+bounded token sample of the same workload instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "MoE layer fwd+bwd tokens/s at E=128 top-4; grouped-GEMM % of tensor peak"
+UNIT = "tokens/s"
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="e128_bf16")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--router", action="store_true", help="compute logits = x.Wr on the device")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--e2e-steps", type=int, default=30)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as fh:
+            d = json.load(fh)
+        return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
+                    bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+def workload_desc(w):
+    return (f"{w.name}: T={w.T}, d_model={w.d}, E={w.E}, top-{w.k}, SwiGLU d_ff={w.d_ff}, "
+            f"{w.dtype}, " + ("logits = x.Wr on device" if w.router else
+                              ("Zipf-skewed " if w.skew else "") + "iid N(0,1) routing logits"))
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.tmp = None
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu), "-lms", "100"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.tmp.flush()
+        with open(self.tmp.name) as fh:
+            rows = [r.strip().split(", ") for r in fh if r.strip()]
+        os.unlink(self.tmp.name)
+        sm, mx, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+                power.append(float(r[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "samples": len(sm),
+                "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------------------ oracle timing
+def oracle_sample_run(w, inp_cpu: dict, T_s: int):
+    """One oracle fwd+bwd over the first T_s tokens of the workload; returns seconds."""
+    import oracle
+    x = inp_cpu["x"][:T_s].double().numpy()
+    dy = inp_cpu["dy"][:T_s].double().numpy()
+    W13, W2 = inp_cpu["W13np"], inp_cpu["W2np"]
+    Wr = None if inp_cpu["Wr"] is None else inp_cpu["Wr"].double().numpy()
+    L = None if inp_cpu["logits"] is None else inp_cpu["logits"][:T_s].double().numpy()
+    t0 = time.perf_counter()
+    fwd = oracle.layer_fwd(x, W13, W2, logits=L, Wr=Wr if L is None else None, k=w.k)
+    oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr)
+    return time.perf_counter() - t0
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return max(n)
+    except Exception:  # noqa: BLE001
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def host_inputs(w, dev_inp: dict) -> dict:
+    """The bench's own inputs on the host (weights as float32 numpy for the oracle)."""
+    out = {k: (None if v is None else v.cpu()) for k, v in dev_inp.items()}
+    out["W13np"] = dev_inp["W13"].float().cpu().numpy()
+    out["W2np"] = dev_inp["W2"].float().cpu().numpy()
+    return out
+
+
+def cpu_baseline(w, inp_cpu, target_s: float) -> dict:
+    T_s = min(64, w.T)
+    t = oracle_sample_run(w, inp_cpu, T_s)
+    if t < target_s / 2 and T_s < w.T:
+        T_s = int(min(w.T, max(T_s + 1, T_s * target_s / max(t, 1e-3))))
+        t = oracle_sample_run(w, inp_cpu, T_s)
+    return {"value": T_s / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"fp64 NumPy oracle fwd+bwd on the first {T_s} of {w.T} tokens of the same "
+                      f"workload (all {w.E} experts' weights), one call, {t:.1f} s"}
+
+
+# ------------------------------------------------------------------------------ reference arm
+def run_reference(args, w, world, rank):
+    if rank != 0:
+        return
+    from routing_grouped_gemm_route_b200.inputs import make_inputs
+    inp = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    inp_cpu = host_inputs(w, inp)
+    del inp
+    T_s = min(128, w.T)
+    for _ in range(args.warmup):
+        oracle_sample_run(w, inp_cpu, T_s)
+    times = [oracle_sample_run(w, inp_cpu, T_s) for _ in range(args.steps)]
+    tot = sum(times)
+    value = T_s * args.steps / tot
+    sample = (f"fp64 NumPy oracle fwd+bwd on the first {T_s} of {w.T} tokens of the workload per "
+              f"step (all {w.E} experts' weights)")
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": workload_desc(w), "tokens_per_step": T_s},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------------------ our arm
+def main():
+    args = parse()
+    from routing_grouped_gemm_route_b200.inputs import WORKLOADS, make_inputs
+    w = WORKLOADS[args.workload]
+    if args.router:
+        w = w.replace(router=True)
+    world, rank, local = dist_setup()
+    if args.impl == "reference":
+        run_reference(args, w, world, rank)
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+        return
+
+    from routing_grouped_gemm_route_b200 import lib
+    lib.load()
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = make_inputs(w, device=dev, seed=w.seed + rank)
+    flags = lib.MOE_FLAG_ROUTER if w.router else 0
+    desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
+    act = lib.act_dtype(desc)
+    T, d, f, E, k = w.T, w.d, w.d_ff, w.E, w.k
+    R = T * k
+    es = 4 if act == torch.float32 else 2
+    ws = lib.alloc_workspace(desc)
+
+    def z(*shape, dt=act):
+        return torch.empty(*shape, dtype=dt, device=dev)
+    x, W13, W2, dy = inp["x"], inp["W13"], inp["W2"], inp["dy"]
+    Wr = inp["Wr"]
+    logits = inp["logits"] if not w.router else z(T, E, dt=torch.float32)
+    idx, gates = z(T, k, dt=torch.int32), z(T, k, dt=torch.float32)
+    counts, offsets = z(E, dt=torch.int32), z(E + 1, dt=torch.int32)
+    slot, row_token, row_gate = z(T, k, dt=torch.int32), z(R, dt=torch.int32), z(R, dt=torch.float32)
+    x_perm, H13, a, y_perm, y = z(R, d), z(R, 2 * f), z(R, f), z(R, d), z(T, d)
+    dy_perm, dH13, dx_perm, dx = z(R, d), z(R, 2 * f), z(R, d), z(T, d)
+    d_logits = z(T, E, dt=torch.float32)
+    dW13, dW2 = z(E, 2 * f, d), z(E, d, f)
+    dWr = z(d, E) if w.router else None
+
+    stages = ["route", "dispatch", "gemm_fwd", "combine", "combine_bwd", "gemm_bwd",
+              "dispatch_bwd"]
+    if w.router:
+        stages = ["router"] + stages + ["router_bwd"]
+    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 2, "combine": 1,
+                "combine_bwd": 1, "gemm_bwd": 4, "dispatch_bwd": 1, "router_bwd": 3}
+
+    def run_stage(name):
+        if name == "router":
+            lib.moe_router_logits(desc, x, Wr, logits)
+        elif name == "route":
+            lib.moe_route(desc, logits, idx, gates, counts, offsets, slot, row_token, row_gate, ws)
+        elif name == "dispatch":
+            lib.moe_dispatch(desc, x, slot, x_perm, ws)
+        elif name == "gemm_fwd":
+            lib.moe_grouped_gemm_fwd(desc, x_perm, W13, W2, offsets, H13, a, y_perm, ws)
+        elif name == "combine":
+            lib.moe_combine(desc, y_perm, gates, slot, y, ws)
+        elif name == "combine_bwd":
+            lib.moe_combine_bwd(desc, dy, y_perm, gates, idx, slot, dy_perm, d_logits, ws)
+        elif name == "gemm_bwd":
+            lib.moe_grouped_gemm_bwd(desc, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13,
+                                     dx_perm, dW13, dW2, ws)
+        elif name == "dispatch_bwd":
+            lib.moe_dispatch_bwd(desc, dx_perm, slot, dx, ws)
+        elif name == "router_bwd":
+            lib.moe_router_bwd(desc, x, Wr, d_logits, dx, dWr, ws)
+
+    K, W = args.steps, args.warmup
+    for _ in range(W):
+        for s in stages:
+            run_stage(s)
+    torch.cuda.synchronize()
+    if lib.moe_read_device_status(ws) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(K):
+        e = ev[i]
+        e[0].record()
+        for j, s in enumerate(stages):
+            run_stage(s)
+            e[j + 1].record()
+    stop.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(stop)
+    ms_total = max_over_ranks(ms_local, world)
+    if lib.moe_read_device_status(ws) != 0:
+        raise RuntimeError("device status set during the timed region")
+
+    stage_ms = {s: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K
+                for j, s in enumerate(stages)}
+    value = world * T * K / (ms_total / 1e3)
+    pk = peaks()
+
+    # algorithmic work per stage
+    gemm_flops = {"gemm_fwd": 6.0 * R * d * f, "gemm_bwd": 12.0 * R * d * f}
+    hbm_bytes = {
+        "route": T * E * 4 + T * k * 12 + R * 8 + 2 * 4 * ((T + 255) // 256) * E,
+        "dispatch": T * d * es + T * k * 4 + R * d * es,
+        "combine": R * d * es + T * k * 8 + T * d * es,
+        "combine_bwd": T * d * es + 2 * R * d * es + T * k * 12 + T * E * 4,
+        "dispatch_bwd": R * d * es + T * k * 4 + T * d * es,
+    }
+    stage_rep = {}
+    for s, ms in stage_ms.items():
+        r = {"ms": round(ms, 4)}
+        if s in gemm_flops:
+            tf = gemm_flops[s] / (ms * 1e-3) / 1e12
+            r.update({"TFLOP/s": round(tf, 1), "frac_of_sustained_bf16": round(tf / pk["bf16_sustained"], 3)})
+        elif s in hbm_bytes:
+            gbs = hbm_bytes[s] / (ms * 1e-3) / 1e9
+            r.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm"], 3)})
+        stage_rep[s] = r
+
+    gemm_ms = stage_ms["gemm_fwd"] + stage_ms["gemm_bwd"]
+    gemm_tflops = (gemm_flops["gemm_fwd"] + gemm_flops["gemm_bwd"]) / (gemm_ms * 1e-3) / 1e12
+    peak_tf = pk["bf16_sustained"]
+    if act == torch.float32:
+        peak_tf = pk["bf16_sustained"] * 1.1 / 2.25     # TF32 = bf16 x nominal ratio
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
+    if os.path.exists(tfile):
+        import hashlib
+        with open(tfile) as fh:
+            tr = json.load(fh)
+        src = open(os.path.join(ROOT, "routing_grouped_gemm_route_b200", "csrc",
+                                "gemm_sm100.cu"), "rb").read()
+        if tr.get("source_sha256") == hashlib.sha256(src).hexdigest() and \
+                tr.get("workload") == w.name:
+            traffic = tr.get("bytes_per_step")
+    roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak_tf,
+                "unit": "TFLOP/s", "frac": round(gemm_tflops / peak_tf, 4), "traffic": traffic,
+                "kernel": "grouped GEMM, 6 launches per step (FC1+SwiGLU, FC2, FC2 dgrad+SwiGLU "
+                          "bwd, FC2 wgrad, FC1 dgrad, FC1 wgrad), algorithmic 18*T*k*d*d_ff flops",
+                "peak_source": f"{pk['source']} sustained dense bf16 (MEASURED_PEAKS.json)"
+                if pk["source"] == "measured" else "fallback 1.4 PFLOP/s sustained"}
+
+    # ---------------------------------------------------------------- end to end (host buffers)
+    E2E = max(3, min(args.e2e_steps, K))
+    hx = torch.empty(T, d, dtype=act, pin_memory=True)
+    hx.copy_(x.cpu())
+    hdy = torch.empty(T, d, dtype=act, pin_memory=True)
+    hdy.copy_(dy.cpu())
+    hl = None
+    if not w.router:
+        hl = torch.empty(T, E, dtype=torch.float32, pin_memory=True)
+        hl.copy_(logits.cpu())
+    hy = torch.empty(T, d, dtype=act, pin_memory=True)
+    hdx = torch.empty(T, d, dtype=act, pin_memory=True)
+    layer = lib.Layer(desc, device=dev)
+    dx_in, dl_in, dy_in = z(T, d), (z(T, E, dt=torch.float32) if not w.router else None), z(T, d)
+    outs = dict(dx=dx, d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
+
+    def e2e_step():
+        dx_in.copy_(hx, non_blocking=True)
+        if dl_in is not None:
+            dl_in.copy_(hl, non_blocking=True)
+        dy_in.copy_(hdy, non_blocking=True)
+        layer.fwd(dx_in, W13, W2, logits=dl_in, Wr=Wr, y=y)
+        layer.bwd(dy_in, W13, W2, x=dx_in, Wr=Wr, out=outs)
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E2E):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = T * d * es * 2 + (0 if w.router else T * E * 4)
+    d2h = T * d * es * 2
+    e2e = {"value": world * T * E2E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": E2E,
+           "api": "moe_layer_fwd + moe_layer_bwd with pinned-host x, logits, dy in and y, dx out"}
+    if lib.moe_read_device_status(layer.ws) != 0:
+        raise RuntimeError("device status set during the end-to-end run")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        inp_cpu = host_inputs(w, inp)
+        cpu = cpu_baseline(w, inp_cpu, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": W, "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if act == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded N(0,1) activations/logits, N(0,0.02) weights)",
+            "config": {"workload": workload_desc(w), "T": T, "d_model": d, "E": E, "top_k": k,
+                       "d_ff": f, "router_on_device": w.router,
+                       "parallelism": f"replicas x{world} (data parallel, no data-path collective)",
+                       "l2": "no flush: each step's working set (~5 GB of weights, activations "
+                             "and grads) exceeds the 126 MB L2"},
+            "roofline": roofline,
+            "gemm_frac_of_peak": round(gemm_tflops / peak_tf, 4),
+            "stages": stage_rep,
+            "gpu_launches": K * sum(launches[s] for s in stages),
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,230 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) routed mixture-of-experts layer.
+ *
+ * The layer is the single-GPU MoE hot path of the Olmo-core 3 training stack as the
+ * write-ups describe it:
+ *   - routing metadata (expert indices, gates, per-expert counts and offsets) is
+ *     produced and kept on the device, with no host round trip
+ *     (deniz.in, "Ai2, Olmo-core 3'ü Apache 2.0 ile yayınladı", section
+ *      "Yeni stack nasıl çalışıyor"; unite.ai, "पैरालेलिज़्म, प्रिसीजन, और मेमोरी तकनीकें");
+ *   - each selected token row is written straight into its expert's contiguous input
+ *     buffer (same sections; donmalab.com, "擴展與最佳化手段");
+ *   - a device-scheduled grouped GEMM runs the imbalanced per-expert shapes that routing
+ *     produces, instead of padding every expert to a common capacity
+ *     (deniz.in, "Yeni stack nasıl çalışıyor");
+ *   - top-4 routing over 8..128 experts (deniz.in, "Ai2'nin raporladığı sayılar");
+ *   - MXFP8 for selected operations (bigchange.ai pt-BR, opening section).
+ * The pages give no formulas.  The definitions used (softmax over the experts, top k
+ * kept and renormalised, ties to the lower expert index, SwiGLU expert FFN with the
+ * gate applied at the combine) are stated with each call below.
+ *
+ * Conventions for every call
+ *   - Pointers named "device" are device memory owned by the caller.  The library
+ *     never allocates, frees or synchronises; every call is asynchronous on `stream`
+ *     (a cudaStream_t passed as void*; NULL is the legacy default stream).
+ *   - Matrices are row-major with the last index contiguous.  Tokens are rows.
+ *   - All device pointers must be 16-byte aligned (MOE_EALIGN otherwise).
+ *   - Element type of activations and weights ("act"): float for MOE_FP32, bfloat16
+ *     for MOE_BF16 and MOE_MXFP8 (MXFP8 quantises inside the grouped GEMM calls).
+ *     Logits, gates and d_logits are always float; indices are int32.
+ *   - Shapes: T >= 0 tokens, d = d_model (multiple of 128), d_ff (multiple of 64),
+ *     1 <= E <= 1024 experts, 1 <= k <= min(E, 32), T*k < 2^31.  R = T*k routed rows.
+ *   - Argument checks run on the host before any launch and return MOE_EINVAL,
+ *     MOE_EALIGN, MOE_EWORKSPACE or MOE_EUNSUPPORTED with nothing launched.  A failed
+ *     launch returns MOE_ECUDA.  Data-dependent faults found on the device (an index
+ *     or offset out of range, a device wait that timed out) set bits of the status
+ *     word in the workspace; they are read only by moe_read_device_status, an
+ *     explicit synchronisation point of the caller's choosing.
+ *   - `ws` is a device workspace of at least moe_workspace_size() bytes, prepared
+ *     once with moe_workspace_init.  Calls that overlap on the GPU must not share one.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_EINVAL = -1,        /* bad descriptor, size or null pointer */
+  MOE_EALIGN = -2,        /* a pointer is not 16-byte aligned */
+  MOE_EWORKSPACE = -3,    /* workspace or saved buffer too small */
+  MOE_EUNSUPPORTED = -4,  /* valid but not supported by this build or device */
+  MOE_ECUDA = -5,         /* a CUDA call or kernel launch failed */
+  MOE_EDEVICE = -6        /* moe_read_device_status found a device-side error */
+} moe_status;
+
+typedef enum moe_dtype {
+  MOE_FP32 = 0,   /* fp32 storage, TF32 tensor-core GEMMs with fp32 accumulation */
+  MOE_BF16 = 1,   /* bf16 storage, bf16 tensor-core GEMMs with fp32 accumulation */
+  MOE_MXFP8 = 2   /* bf16 storage, GEMM operands E4M3 with an E8M0 scale per 32 */
+} moe_dtype;
+
+/* moe_desc.flags */
+#define MOE_FLAG_ROUTER   1  /* logits = x . Wr computed on the device (else injected) */
+#define MOE_FLAG_DW_FP32  2  /* dW13 / dW2 are float (else act type) */
+#define MOE_FLAG_ACCUM_DW 4  /* add into existing float dW (requires MOE_FLAG_DW_FP32) */
+
+/* device status bits */
+#define MOE_DEV_BAD_INDEX   1  /* an expert index or slot was out of range; the row was skipped */
+#define MOE_DEV_BAD_OFFSETS 2  /* offsets not an exclusive scan ending at R; GEMM skipped */
+#define MOE_DEV_TIMEOUT     4  /* a bounded device wait gave up; results are invalid */
+
+typedef struct moe_desc {
+  int32_t T, d, d_ff, E, k;
+  int32_t dtype;   /* moe_dtype */
+  int32_t flags;   /* MOE_FLAG_* */
+} moe_desc;
+
+/* Byte offsets (from the start of the caller's `saved` buffer) of the tensors that
+ * moe_layer_fwd keeps for moe_layer_bwd.  Every offset is a multiple of 256. */
+typedef struct moe_saved_layout {
+  size_t topk_idx;   /* int32 [T,k] */
+  size_t gates;      /* float [T,k] */
+  size_t counts;     /* int32 [E] */
+  size_t offsets;    /* int32 [E+1] */
+  size_t slot;       /* int32 [T,k] */
+  size_t row_token;  /* int32 [R] */
+  size_t row_gate;   /* float [R] */
+  size_t logits;     /* float [T,E] (router on only; else equal to `x_perm`, unused) */
+  size_t x_perm;     /* act [R,d] */
+  size_t H13;        /* act [R,2*d_ff] */
+  size_t a;          /* act [R,d_ff] */
+  size_t y_perm;     /* act [R,d] */
+  size_t total;      /* bytes needed */
+} moe_saved_layout;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(int32_t status);
+
+/* Checks a descriptor; MOE_OK if every call below accepts it. */
+moe_status moe_check_desc(const moe_desc* desc);
+
+/* Workspace bytes that every call below needs for this descriptor (*bytes out). */
+moe_status moe_workspace_size(const moe_desc* desc, size_t* bytes);
+
+/* Layout and size of the `saved` buffer of moe_layer_fwd / moe_layer_bwd. */
+moe_status moe_saved_layout_get(const moe_desc* desc, moe_saved_layout* out);
+
+/* Zeroes the device status word of `ws` (asynchronous on `stream`).  Call once after
+ * allocating a workspace, and after handling an error reported by
+ * moe_read_device_status. */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/* Synchronises `stream`, then copies the device status word of `ws` to *bits (host).
+ * Returns MOE_OK when no bit is set, MOE_EDEVICE otherwise.  This is the only call
+ * that waits for the device. */
+moe_status moe_read_device_status(const void* ws, void* stream, int32_t* bits);
+
+/* S1, router projection: logits[T,E] (float, device) = x[T,d] (act) . Wr[d,E] (act),
+ * fp32 accumulation.  The pages measure their headline rows with random routing
+ * (bigchange.ai pt-BR, "Três números, três denominadores"); this call is the learned
+ * router's projection. */
+moe_status moe_router_logits(const moe_desc* desc, const void* x, const void* Wr,
+                             float* logits, void* stream);
+
+/* S2-S4, GPU-resident routing (deniz.in, "Yeni stack nasıl çalışıyor").
+ * In:  logits [T,E] float.
+ * Out: topk_idx [T,k] int32: per token the k experts of largest logit in descending
+ *      logit order, equal logits broken towards the lower expert index;
+ *      gates [T,k] float: softmax over the k kept logits (= full softmax
+ *      renormalised over the kept experts);
+ *      counts [E] int32: rows per expert;  offsets [E+1] int32: exclusive scan of counts;
+ *      slot [T,k] int32: row of pair (t,j) in the expert-sorted order, rows of one
+ *      expert in token order: slot[t,j] = offsets[e] + #{t' < t routed to e};
+ *      row_token [R] int32 and row_gate [R] float: token and gate of each sorted row.
+ * Every output is fully written; counts/offsets never leave the device. */
+moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_idx,
+                     float* gates, int32_t* counts, int32_t* offsets, int32_t* slot,
+                     int32_t* row_token, float* row_gate, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* S5, row-wise dispatch: x_perm[slot[t,j]] = x[t] for every (t,j)
+ * (unite.ai, "पैरालेलिज़्म, प्रिसीजन, और मेमोरी तकनीकें").  x [T,d] act, x_perm [R,d] act.
+ * x_perm_sf is reserved for the MXFP8 layout and must be NULL.  A slot outside
+ * [0,R) sets MOE_DEV_BAD_INDEX and that copy is skipped. */
+moe_status moe_dispatch(const moe_desc* desc, const void* x, const int32_t* slot,
+                        void* x_perm, void* x_perm_sf, void* ws, size_t ws_bytes,
+                        void* stream);
+
+/* S6-S7, device-scheduled grouped GEMM forward of the SwiGLU experts
+ * (deniz.in, "Yeni stack nasıl çalışıyor").  For each expert e, rows
+ * [offsets[e], offsets[e+1]) of x_perm form X_e:
+ *   H13_e = X_e . W13_e^T          (W13 [E, 2*d_ff, d]: rows 0..d_ff-1 gate W1, then up W3)
+ *   a_e   = silu(H1_e) * H3_e      (computed in fp32 from the accumulator)
+ *   Y_e   = a_e . W2_e^T           (W2 [E, d, d_ff])
+ * Out: H13 [R,2*d_ff], a [R,d_ff], y_perm [R,d], all act.  The tile schedule is read
+ * from `offsets` on the device.  Offsets that are not an exclusive scan ending at R
+ * set MOE_DEV_BAD_OFFSETS and nothing is written. */
+moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm,
+                                const void* x_perm_sf, const void* W13, const void* W2,
+                                const int32_t* offsets, void* H13, void* a, void* y_perm,
+                                void* ws, size_t ws_bytes, void* stream);
+
+/* S8, weighted combine: y[t] = sum_j gates[t,j] * y_perm[slot[t,j]], summed in fp32.
+ * y_perm [R,d] act -> y [T,d] act.  A gather: no atomics, deterministic. */
+moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* gates,
+                       const int32_t* slot, void* y, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* S9, backward of the combine and of the gate softmax:
+ *   dy_perm[slot[t,j]] = gates[t,j] * dy[t]                        (act [R,d])
+ *   dg[t,j] = <dy[t], y_perm[slot[t,j]]>                            (fp32)
+ *   d_logits[t, topk_idx[t,j]] = g_tj * (dg_tj - sum_i g_ti dg_ti), 0 elsewhere  ([T,E] float) */
+moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_perm,
+                           const float* gates, const int32_t* topk_idx, const int32_t* slot,
+                           void* dy_perm, float* d_logits, void* ws, size_t ws_bytes,
+                           void* stream);
+
+/* S10-S13, grouped GEMM backward of the SwiGLU experts, per expert e:
+ *   dA_e   = dY_e . W2_e                                   (dY_e = rows of dy_perm)
+ *   dH1_e  = dA_e * H3_e * s * (1 + H1_e * (1 - s)),  s = sigmoid(H1_e)
+ *   dH3_e  = dA_e * silu(H1_e)                            -> dH13 [R,2*d_ff] act
+ *   dW2_e  = dY_e^T . a_e                                  -> dW2  [E,d,d_ff]
+ *   dX_e   = dH13_e . W13_e                                -> dx_perm [R,d] act
+ *   dW13_e = dH13_e^T . X_e                                -> dW13 [E,2*d_ff,d]
+ * dW is act type, or float with MOE_FLAG_DW_FP32 (added into with MOE_FLAG_ACCUM_DW).
+ * An expert with no rows gets dW_e = 0 exactly (unchanged with MOE_FLAG_ACCUM_DW). */
+moe_status moe_grouped_gemm_bwd(const moe_desc* desc, const void* dy_perm, const void* x_perm,
+                                const void* H13, const void* a, const void* W13,
+                                const void* W2, const int32_t* offsets, void* dH13,
+                                void* dx_perm, void* dW13, void* dW2, void* ws,
+                                size_t ws_bytes, void* stream);
+
+/* S14, unpermute-reduce: dx[t] = sum_j dx_perm[slot[t,j]] (fp32 sum, act out). */
+moe_status moe_dispatch_bwd(const moe_desc* desc, const void* dx_perm, const int32_t* slot,
+                            void* dx, void* ws, size_t ws_bytes, void* stream);
+
+/* Router backward (MOE_FLAG_ROUTER): dx[T,d] += d_logits . Wr^T and
+ * dWr[d,E] (act) = x^T . d_logits, fp32 accumulation. */
+moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
+                          const float* d_logits, void* dx, void* dWr, void* ws,
+                          size_t ws_bytes, void* stream);
+
+/* Whole layer forward: [router] -> route -> dispatch -> grouped GEMM fwd -> combine.
+ * logits: injected routing logits [T,E] float, or NULL with MOE_FLAG_ROUTER and Wr.
+ * y [T,d] act.  `saved` (moe_saved_layout.total bytes) receives the tensors listed in
+ * moe_saved_layout, which moe_layer_bwd reads. */
+moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logits,
+                         const void* Wr, const void* W13, const void* W2, void* y,
+                         void* saved, size_t saved_bytes, void* ws, size_t ws_bytes,
+                         void* stream);
+
+/* Whole layer backward for upstream gradient dy [T,d] act.  Out: dx [T,d] act,
+ * d_logits [T,E] float, dW13, dW2 (see moe_grouped_gemm_bwd), and dWr [d,E] act when
+ * MOE_FLAG_ROUTER (x and Wr required then; x may be NULL otherwise). */
+moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x,
+                         const void* saved, size_t saved_bytes, const void* W13,
+                         const void* W2, const void* Wr, void* dx, float* d_logits,
+                         void* dW13, void* dW2, void* dWr, void* ws, size_t ws_bytes,
+                         void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

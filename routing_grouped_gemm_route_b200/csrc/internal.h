@@ -1,0 +1,60 @@
+// Internal launchers shared by the C-ABI entry points (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+int num_sms();
+
+// ----------------------------------------------------------------------------- routing
+// Tokens per routing CTA (8 warps x 32 tokens); the histogram has one row per CTA.
+constexpr int kRouteTokensPerCta = 256;
+inline int route_ctas(int T) { return (T + kRouteTokensPerCta - 1) / kRouteTokensPerCta; }
+
+cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
+                         int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                         float* row_gate, int32_t* hist, int32_t* cta_base, int* status,
+                         cudaStream_t s);
+
+// C[M,N] (fp32 out, or act out) = A . B with arbitrary element strides; a plain
+// CUDA-core kernel for the small router projections.
+cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A, int64_t sam,
+                               int64_t sak, bool a_is_act, const void* B, int64_t sbk,
+                               int64_t sbn, bool b_is_act, void* C, bool c_is_act,
+                               bool accumulate, cudaStream_t s);
+
+// ----------------------------------------------------------------------------- permute
+cudaError_t launch_dispatch(bool fp32, int T, int d, int k, const void* x, const int32_t* slot,
+                            void* x_perm, int* status, cudaStream_t s);
+// y[t] = sum_j w_tj * src[slot[t,j]] (+ extra[t] fp32 when given); w = gates or all ones.
+cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, const void* src,
+                              const float* gates, const int32_t* slot, const float* extra,
+                              void* y, int* status, cudaStream_t s);
+// y[i] += extra[i] for n elements (fp32 add, one rounding to the act type)
+cudaError_t launch_add_f32(bool fp32, int64_t n, void* y, const float* extra, cudaStream_t s);
+cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void* dy,
+                               const void* y_perm, const float* gates, const int32_t* topk_idx,
+                               const int32_t* slot, void* dy_perm, float* d_logits, int* status,
+                               cudaStream_t s);
+
+// ----------------------------------------------------------------------------- grouped GEMM
+struct GemmShape {
+  int E, R, d, f;
+  bool fp32;   // fp32 storage / TF32 MMA, else bf16
+};
+// FC1 (+SwiGLU epilogue) and FC2 forward.
+moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
+                    const int32_t* offsets, void* H13, void* a, void* y_perm, int* status,
+                    cudaStream_t s);
+// FC2 dgrad (+SwiGLU bwd), FC2 wgrad, FC1 dgrad, FC1 wgrad.
+moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm, const void* H13,
+                    const void* a, const void* W13, const void* W2, const int32_t* offsets,
+                    void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
+                    bool dw_accum, int* status, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,444 @@
+// C-ABI entry points: argument checks on the host, workspace carving and kernel
+// launches on the caller's stream.  No call allocates, frees or waits for the device
+// (except moe_read_device_status, whose purpose is to wait).
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "internal.h"
+#include "moe.h"
+
+namespace moe {
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline size_t act_bytes(const moe_desc& d) { return d.dtype == MOE_FP32 ? 4 : 2; }
+inline int64_t R_of(const moe_desc& d) { return (int64_t)d.T * d.k; }
+inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+struct WsLayout {
+  size_t status, hist, cta_base, dy_perm, dH13, dx_perm, dx_router, total;
+};
+
+WsLayout ws_layout(const moe_desc& d) {
+  WsLayout w;
+  const size_t es = act_bytes(d);
+  const size_t R = (size_t)R_of(d);
+  const size_t ctas = (size_t)route_ctas(d.T);
+  size_t o = 0;
+  w.status = o; o += kAlign;
+  w.hist = o; o = up(o + ctas * d.E * 4);
+  w.cta_base = o; o = up(o + ctas * d.E * 4);
+  w.dy_perm = o; o = up(o + R * d.d * es);
+  w.dH13 = o; o = up(o + R * 2 * (size_t)d.d_ff * es);
+  w.dx_perm = o; o = up(o + R * d.d * es);
+  w.dx_router = o;
+  if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.d * 4);
+  w.total = o;
+  return w;
+}
+
+moe_saved_layout saved_layout(const moe_desc& d) {
+  moe_saved_layout s;
+  const size_t es = act_bytes(d);
+  const size_t T = d.T, k = d.k, R = (size_t)R_of(d), E = d.E;
+  size_t o = 0;
+  s.topk_idx = o; o = up(o + T * k * 4);
+  s.gates = o; o = up(o + T * k * 4);
+  s.counts = o; o = up(o + E * 4);
+  s.offsets = o; o = up(o + (E + 1) * 4);
+  s.slot = o; o = up(o + T * k * 4);
+  s.row_token = o; o = up(o + R * 4);
+  s.row_gate = o; o = up(o + R * 4);
+  s.logits = o;
+  if (d.flags & MOE_FLAG_ROUTER) o = up(o + T * E * 4);
+  s.x_perm = o; o = up(o + R * d.d * es);
+  s.H13 = o; o = up(o + R * 2 * (size_t)d.d_ff * es);
+  s.a = o; o = up(o + R * (size_t)d.d_ff * es);
+  s.y_perm = o; o = up(o + R * d.d * es);
+  s.total = o;
+  return s;
+}
+
+moe_status check(const moe_desc* d) {
+  if (!d) return MOE_EINVAL;
+  if (d->T < 0 || d->d <= 0 || d->d_ff <= 0 || d->E < 1 || d->E > 1024 || d->k < 1 ||
+      d->k > 32 || d->k > d->E)
+    return MOE_EINVAL;
+  if (d->d % 128 != 0 || d->d_ff % 64 != 0) return MOE_EINVAL;
+  if ((int64_t)d->T * d->k >= (int64_t(1) << 31)) return MOE_EINVAL;
+  if ((int64_t)d->E * 2 * d->d_ff >= (int64_t(1) << 31) || (int64_t)d->E * d->d >= (int64_t(1) << 31))
+    return MOE_EINVAL;
+  if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
+  if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW)) return MOE_EINVAL;
+  if ((d->flags & MOE_FLAG_ACCUM_DW) && !(d->flags & MOE_FLAG_DW_FP32)) return MOE_EINVAL;
+  if (d->dtype == MOE_MXFP8) return MOE_EUNSUPPORTED;
+  return MOE_OK;
+}
+
+// Every pointer in the list must be non-null and 16-byte aligned.
+moe_status ptrs(std::initializer_list<const void*> ps) {
+  for (const void* p : ps) {
+    if (!p) return MOE_EINVAL;
+    if (!aligned16(p)) return MOE_EALIGN;
+  }
+  return MOE_OK;
+}
+// Pointers to buffers whose size is a multiple of T: with no tokens they may be null
+// (an empty tensor has no storage); otherwise as above.
+moe_status tptrs(const moe_desc& d, std::initializer_list<const void*> ps) {
+  if (d.T > 0) return ptrs(ps);
+  for (const void* p : ps)
+    if (p && !aligned16(p)) return MOE_EALIGN;
+  return MOE_OK;
+}
+
+moe_status ws_ok(const moe_desc& d, const void* ws, size_t ws_bytes) {
+  if (!ws) return MOE_EINVAL;
+  if (!aligned16(ws)) return MOE_EALIGN;
+  if (ws_bytes < ws_layout(d).total) return MOE_EWORKSPACE;
+  return MOE_OK;
+}
+
+inline int* status_ptr(void* ws) { return reinterpret_cast<int*>(ws); }
+template <typename P>
+inline P* at(void* base, size_t off) {
+  return reinterpret_cast<P*>(reinterpret_cast<char*>(base) + off);
+}
+template <typename P>
+inline const P* at(const void* base, size_t off) {
+  return reinterpret_cast<const P*>(reinterpret_cast<const char*>(base) + off);
+}
+inline moe_status cu(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+
+#define MOE_TRY(expr)                  \
+  do {                                 \
+    moe_status _st = (expr);           \
+    if (_st != MOE_OK) return _st;     \
+  } while (0)
+
+GemmShape gshape(const moe_desc& d) {
+  GemmShape g;
+  g.E = d.E;
+  g.R = (int)R_of(d);
+  g.d = d.d;
+  g.f = d.d_ff;
+  g.fp32 = d.dtype == MOE_FP32;
+  return g;
+}
+
+// ---------------------------------------------------------------------------- bodies
+moe_status route_body(const moe_desc& d, const float* logits, int32_t* idx, float* gates,
+                      int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                      float* row_gate, void* ws, cudaStream_t s) {
+  const WsLayout w = ws_layout(d);
+  if (d.T == 0) {
+    MOE_TRY(cu(cudaMemsetAsync(counts, 0, sizeof(int32_t) * d.E, s)));
+    return cu(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (d.E + 1), s));
+  }
+  return cu(launch_route(d, logits, idx, gates, counts, offsets, slot, row_token, row_gate,
+                         at<int32_t>(ws, w.hist), at<int32_t>(ws, w.cta_base), status_ptr(ws), s));
+}
+
+moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_perm,
+                         const void* H13, const void* a, const void* W13, const void* W2,
+                         const int32_t* offsets, void* dH13, void* dx_perm, void* dW13, void* dW2,
+                         void* ws, cudaStream_t s) {
+  const bool fp32_dw = d.flags & MOE_FLAG_DW_FP32;
+  const bool acc = d.flags & MOE_FLAG_ACCUM_DW;
+  if (R_of(d) == 0) {
+    if (acc) return MOE_OK;
+    const size_t es = fp32_dw ? 4 : act_bytes(d);
+    MOE_TRY(cu(cudaMemsetAsync(dW13, 0, (size_t)d.E * 2 * d.d_ff * d.d * es, s)));
+    return cu(cudaMemsetAsync(dW2, 0, (size_t)d.E * d.d * d.d_ff * es, s));
+  }
+  return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13, dW2,
+                  fp32_dw, acc, status_ptr(ws), s);
+}
+
+moe_status router_fwd_body(const moe_desc& d, const void* x, const void* Wr, float* logits,
+                           cudaStream_t s) {
+  if (d.T == 0) return MOE_OK;
+  const bool f32 = d.dtype == MOE_FP32;
+  // logits[T,E] = x[T,d] . Wr[d,E]
+  return cu(launch_router_gemm(f32, d.T, d.E, d.d, x, d.d, 1, true, Wr, d.E, 1, true, logits,
+                               false, false, s));
+}
+
+moe_status router_bwd_body(const moe_desc& d, const void* x, const void* Wr,
+                           const float* d_logits, float* dx_extra, void* dx_act, void* dWr,
+                           cudaStream_t s) {
+  const bool f32 = d.dtype == MOE_FP32;
+  if (d.T > 0) {
+    if (dx_extra) {
+      // dx_extra[T,d] (float) = d_logits[T,E] . Wr^T
+      MOE_TRY(cu(launch_router_gemm(f32, d.T, d.d, d.E, d_logits, d.E, 1, false, Wr, 1, d.E, true,
+                                    dx_extra, false, false, s)));
+    } else {
+      // dx[T,d] (act) += d_logits . Wr^T
+      if (!f32) return MOE_EUNSUPPORTED;   // bf16 in-place add goes through dx_extra
+      MOE_TRY(cu(launch_router_gemm(f32, d.T, d.d, d.E, d_logits, d.E, 1, false, Wr, 1, d.E, true,
+                                    dx_act, true, true, s)));
+    }
+  }
+  // dWr[d,E] = x^T . d_logits
+  if (d.T == 0) {
+    return cu(cudaMemsetAsync(dWr, 0, (size_t)d.d * d.E * act_bytes(d), s));
+  }
+  return cu(launch_router_gemm(f32, d.d, d.E, d.T, x, 1, d.d, true, d_logits, d.E, 1, false, dWr,
+                               true, false, s));
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int32_t st) {
+  switch (st) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument";
+    case MOE_EALIGN: return "pointer not 16-byte aligned";
+    case MOE_EWORKSPACE: return "workspace or saved buffer too small";
+    case MOE_EUNSUPPORTED: return "unsupported configuration";
+    case MOE_ECUDA: return "CUDA error";
+    case MOE_EDEVICE: return "device-side error flagged in the status word";
+    default: return "unknown status";
+  }
+}
+
+moe_status moe_check_desc(const moe_desc* desc) { return check(desc); }
+
+moe_status moe_workspace_size(const moe_desc* desc, size_t* bytes) {
+  MOE_TRY(check(desc));
+  if (!bytes) return MOE_EINVAL;
+  *bytes = ws_layout(*desc).total;
+  return MOE_OK;
+}
+
+moe_status moe_saved_layout_get(const moe_desc* desc, moe_saved_layout* out) {
+  MOE_TRY(check(desc));
+  if (!out) return MOE_EINVAL;
+  *out = saved_layout(*desc);
+  return MOE_OK;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws) return MOE_EINVAL;
+  if (!aligned16(ws)) return MOE_EALIGN;
+  if (ws_bytes < 256) return MOE_EWORKSPACE;
+  return cu(cudaMemsetAsync(ws, 0, 256, S(stream)));
+}
+
+moe_status moe_read_device_status(const void* ws, void* stream, int32_t* bits) {
+  if (!ws || !bits) return MOE_EINVAL;
+  int32_t v = 0;
+  if (cudaMemcpyAsync(&v, ws, sizeof(v), cudaMemcpyDeviceToHost, S(stream)) != cudaSuccess)
+    return MOE_ECUDA;
+  if (cudaStreamSynchronize(S(stream)) != cudaSuccess) return MOE_ECUDA;
+  *bits = v;
+  return v ? MOE_EDEVICE : MOE_OK;
+}
+
+moe_status moe_router_logits(const moe_desc* desc, const void* x, const void* Wr, float* logits,
+                             void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {x, logits}));
+  MOE_TRY(ptrs({Wr}));
+  return router_fwd_body(*desc, x, Wr, logits, S(stream));
+}
+
+moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_idx, float* gates,
+                     int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                     float* row_gate, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {logits, topk_idx, gates, slot, row_token, row_gate}));
+  MOE_TRY(ptrs({counts, offsets}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  return route_body(*desc, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate, ws,
+                    S(stream));
+}
+
+moe_status moe_dispatch(const moe_desc* desc, const void* x, const int32_t* slot, void* x_perm,
+                        void* x_perm_sf, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {x, slot, x_perm}));
+  if (x_perm_sf) return MOE_EINVAL;
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  const moe_desc& d = *desc;
+  return cu(launch_dispatch(d.dtype == MOE_FP32, d.T, d.d, d.k, x, slot, x_perm, status_ptr(ws),
+                            S(stream)));
+}
+
+moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const void* x_perm_sf,
+                                const void* W13, const void* W2, const int32_t* offsets, void* H13,
+                                void* a, void* y_perm, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {x_perm, H13, a, y_perm}));
+  MOE_TRY(ptrs({W13, W2, offsets}));
+  if (x_perm_sf) return MOE_EINVAL;
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  if (R_of(*desc) == 0) return MOE_OK;
+  return gemm_fwd(gshape(*desc), x_perm, W13, W2, offsets, H13, a, y_perm, status_ptr(ws),
+                  S(stream));
+}
+
+moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* gates,
+                       const int32_t* slot, void* y, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {y_perm, gates, slot, y}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  const moe_desc& d = *desc;
+  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, y_perm, gates, slot, nullptr, y,
+                              status_ptr(ws), S(stream)));
+}
+
+moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_perm,
+                           const float* gates, const int32_t* topk_idx, const int32_t* slot,
+                           void* dy_perm, float* d_logits, void* ws, size_t ws_bytes,
+                           void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  const moe_desc& d = *desc;
+  return cu(launch_combine_bwd(d.dtype == MOE_FP32, d.T, d.d, d.k, d.E, dy, y_perm, gates,
+                               topk_idx, slot, dy_perm, d_logits, status_ptr(ws), S(stream)));
+}
+
+moe_status moe_grouped_gemm_bwd(const moe_desc* desc, const void* dy_perm, const void* x_perm,
+                                const void* H13, const void* a, const void* W13, const void* W2,
+                                const int32_t* offsets, void* dH13, void* dx_perm, void* dW13,
+                                void* dW2, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {dy_perm, x_perm, H13, a, dH13, dx_perm}));
+  MOE_TRY(ptrs({W13, W2, offsets, dW13, dW2}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  return gemm_bwd_body(*desc, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13, dW2,
+                       ws, S(stream));
+}
+
+moe_status moe_dispatch_bwd(const moe_desc* desc, const void* dx_perm, const int32_t* slot,
+                            void* dx, void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {dx_perm, slot, dx}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  const moe_desc& d = *desc;
+  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, dx_perm, nullptr, slot, nullptr,
+                              dx, status_ptr(ws), S(stream)));
+}
+
+moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
+                          const float* d_logits, void* dx, void* dWr, void* ws, size_t ws_bytes,
+                          void* stream) {
+  MOE_TRY(check(desc));
+  MOE_TRY(tptrs(*desc, {x, d_logits, dx}));
+  MOE_TRY(ptrs({Wr, dWr}));
+  MOE_TRY(ws_ok(*desc, ws, ws_bytes));
+  const moe_desc& d = *desc;
+  if (d.dtype == MOE_FP32) return router_bwd_body(d, x, Wr, d_logits, nullptr, dx, dWr, S(stream));
+  // bf16: accumulate the router term in fp32, then add it to dx with one rounding
+  const WsLayout w = ws_layout(d);
+  if (!(d.flags & MOE_FLAG_ROUTER)) return MOE_EINVAL;
+  float* extra = at<float>(ws, w.dx_router);
+  MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, S(stream)));
+  return cu(launch_add_f32(false, (int64_t)d.T * d.d, dx, extra, S(stream)));
+}
+
+moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logits, const void* Wr,
+                         const void* W13, const void* W2, void* y, void* saved, size_t saved_bytes,
+                         void* ws, size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  const moe_desc& d = *desc;
+  const bool router = d.flags & MOE_FLAG_ROUTER;
+  MOE_TRY(tptrs(d, {x, y}));
+  MOE_TRY(ptrs({W13, W2, saved}));
+  if (router) MOE_TRY(ptrs({Wr}));
+  else MOE_TRY(tptrs(d, {logits}));
+  MOE_TRY(ws_ok(d, ws, ws_bytes));
+  const moe_saved_layout L = saved_layout(d);
+  if (saved_bytes < L.total) return MOE_EWORKSPACE;
+  cudaStream_t s = S(stream);
+  int* st = status_ptr(ws);
+
+  const float* lg = logits;
+  if (router) {
+    float* out = at<float>(saved, L.logits);
+    MOE_TRY(router_fwd_body(d, x, Wr, out, s));
+    lg = out;
+  }
+  int32_t* idx = at<int32_t>(saved, L.topk_idx);
+  float* gates = at<float>(saved, L.gates);
+  int32_t* slot = at<int32_t>(saved, L.slot);
+  int32_t* offsets = at<int32_t>(saved, L.offsets);
+  MOE_TRY(route_body(d, lg, idx, gates, at<int32_t>(saved, L.counts), offsets, slot,
+                     at<int32_t>(saved, L.row_token), at<float>(saved, L.row_gate), ws, s));
+  if (d.T == 0) return MOE_OK;
+  const bool f32 = d.dtype == MOE_FP32;
+  void* x_perm = at<char>(saved, L.x_perm);
+  void* y_perm = at<char>(saved, L.y_perm);
+  MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, x_perm, st, s)));
+  MOE_TRY(gemm_fwd(gshape(d), x_perm, W13, W2, offsets, at<char>(saved, L.H13),
+                   at<char>(saved, L.a), y_perm, st, s));
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, y_perm, gates, slot, nullptr, y, st, s));
+}
+
+moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, const void* saved,
+                         size_t saved_bytes, const void* W13, const void* W2, const void* Wr,
+                         void* dx, float* d_logits, void* dW13, void* dW2, void* dWr, void* ws,
+                         size_t ws_bytes, void* stream) {
+  MOE_TRY(check(desc));
+  const moe_desc& d = *desc;
+  const bool router = d.flags & MOE_FLAG_ROUTER;
+  MOE_TRY(tptrs(d, {dy, dx, d_logits}));
+  MOE_TRY(ptrs({saved, W13, W2, dW13, dW2}));
+  if (router) {
+    MOE_TRY(tptrs(d, {x}));
+    MOE_TRY(ptrs({Wr, dWr}));
+  }
+  MOE_TRY(ws_ok(d, ws, ws_bytes));
+  const moe_saved_layout L = saved_layout(d);
+  if (saved_bytes < L.total) return MOE_EWORKSPACE;
+  const WsLayout w = ws_layout(d);
+  cudaStream_t s = S(stream);
+  int* st = status_ptr(ws);
+  const bool f32 = d.dtype == MOE_FP32;
+
+  const int32_t* idx = at<int32_t>(saved, L.topk_idx);
+  const float* gates = at<float>(saved, L.gates);
+  const int32_t* slot = at<int32_t>(saved, L.slot);
+  const int32_t* offsets = at<int32_t>(saved, L.offsets);
+  void* dy_perm = at<char>(ws, w.dy_perm);
+  void* dH13 = at<char>(ws, w.dH13);
+  void* dx_perm = at<char>(ws, w.dx_perm);
+
+  MOE_TRY(cu(launch_combine_bwd(f32, d.T, d.d, d.k, d.E, dy, at<char>(saved, L.y_perm), gates,
+                                idx, slot, dy_perm, d_logits, st, s)));
+  MOE_TRY(gemm_bwd_body(d, dy_perm, at<char>(saved, L.x_perm), at<char>(saved, L.H13),
+                        at<char>(saved, L.a), W13, W2, offsets, dH13, dx_perm, dW13, dW2, ws, s));
+  float* extra = nullptr;
+  if (router) {
+    extra = at<float>(ws, w.dx_router);
+    MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, s));
+  }
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, dx_perm, nullptr, slot, extra, dx, st, s));
+}
+
+}  // extern "C"

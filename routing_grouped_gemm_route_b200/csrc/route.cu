@@ -1,0 +1,306 @@
+// GPU-resident routing: top-k selection, renormalised gates, per-expert counts and
+// offsets, and the expert-sorted slot of every (token, j) pair.
+//
+// The write-ups say the routing metadata now stays on the GPU, removing the old
+// path's host round trip for the expert-group sizes, so the CPU can queue work
+// without waiting for a copy back (deniz.in, "Ai2, Olmo-core 3'ü Apache 2.0 ile
+// yayınladı", section "Yeni stack nasıl çalışıyor"; unite.ai, "पैरालेलिज़्म, प्रिसीजन,
+// और मेमोरी तकनीकें").  Three launches, no atomics on global memory, no host sync:
+//   1. topk:  one warp per token, logits in registers, k rounds of warp arg-max
+//             (ties to the lower expert index); gates = softmax over the kept
+//             logits; a per-CTA expert histogram in shared memory.
+//   2. scan:  one CTA: per expert, an exclusive scan of the CTA histograms (the
+//             CTA's base inside the expert), counts, and offsets = exclusive scan
+//             of counts.
+//   3. slots: per warp of 32 tokens, a bitmask per expert of the lanes that chose
+//             it; a token's rank inside the expert is the population count of the
+//             lower lanes' bits plus the bases of earlier warps and CTAs.  So the
+//             rows of an expert come out in token order.
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <math.h>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kWarps = 8;
+static_assert(kWarps * 32 == kRouteTokensPerCta, "one token per lane in the slot pass");
+
+// a beats b: larger logit, or equal logit and smaller index
+__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
+  return va > vb || (va == vb && ia < ib);
+}
+
+template <int NPL>   // logits per lane = ceil(E / 32)
+__global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float* __restrict__ logits,
+                                                           int T, int E, int k,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ gates,
+                                                           int32_t* __restrict__ hist) {
+  extern __shared__ int s_hist[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+
+  const int t0 = blockIdx.x * kRouteTokensPerCta + warp * 32;
+  for (int i = 0; i < 32; ++i) {
+    const int t = t0 + i;
+    if (t >= T) break;
+    const float* row = logits + (int64_t)t * E;
+    float v[NPL];
+#pragma unroll
+    for (int c = 0; c < NPL; ++c) {
+      const int e = c * 32 + lane;
+      v[c] = e < E ? row[e] : -INFINITY;
+    }
+    unsigned taken = 0;           // bit c: v[c] already selected
+    float my_val = 0.f;
+    int my_idx = 0;
+    float top = 0.f;
+    for (int j = 0; j < k; ++j) {
+      // lane-local best among the not-yet-taken entries (index ascending on ties)
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        const int e = c * 32 + lane;
+        if (e < E && !(taken & (1u << c)) && better(v[c], e, bv, bi)) {
+          bv = v[c];
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+        if (better(ov, oi, bv, bi)) {
+          bv = ov;
+          bi = oi;
+        }
+      }
+      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+      if (j == 0) top = bv;
+      if (lane == j) {
+        my_val = bv;
+        my_idx = bi;
+      }
+    }
+    // gates: softmax over the kept logits, lane j holds entry j
+    const float z = lane < k ? expf(my_val - top) : 0.f;
+    const float sum = warp_sum(z);
+    if (lane < k) {
+      topk_idx[(int64_t)t * k + lane] = my_idx;
+      gates[(int64_t)t * k + lane] = z / sum;
+      atomicAdd(&s_hist[my_idx], 1);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
+}
+
+// One CTA of 1024 threads: per expert the scan over CTA histograms, then offsets.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ hist, int nctas,
+                                                    int E, int32_t* __restrict__ cta_base,
+                                                    int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets) {
+  __shared__ int s_part[1024];
+  __shared__ int s_carry;
+  if (threadIdx.x == 0) s_carry = 0;
+  __syncthreads();
+  for (int e0 = 0; e0 < E; e0 += 1024) {
+    const int e = e0 + threadIdx.x;
+    int run = 0;
+    if (e < E) {
+      int c = 0;
+      for (; c + 4 <= nctas; c += 4) {
+        const int h0 = hist[(int64_t)(c + 0) * E + e];
+        const int h1 = hist[(int64_t)(c + 1) * E + e];
+        const int h2 = hist[(int64_t)(c + 2) * E + e];
+        const int h3 = hist[(int64_t)(c + 3) * E + e];
+        cta_base[(int64_t)(c + 0) * E + e] = run;
+        cta_base[(int64_t)(c + 1) * E + e] = run + h0;
+        cta_base[(int64_t)(c + 2) * E + e] = run + h0 + h1;
+        cta_base[(int64_t)(c + 3) * E + e] = run + h0 + h1 + h2;
+        run += h0 + h1 + h2 + h3;
+      }
+      for (; c < nctas; ++c) {
+        const int h = hist[(int64_t)c * E + e];
+        cta_base[(int64_t)c * E + e] = run;
+        run += h;
+      }
+      counts[e] = run;
+    }
+    // block-wide inclusive scan of `run` (Hillis-Steele)
+    s_part[threadIdx.x] = run;
+    __syncthreads();
+    for (int o = 1; o < 1024; o <<= 1) {
+      const int add = threadIdx.x >= o ? s_part[threadIdx.x - o] : 0;
+      __syncthreads();
+      s_part[threadIdx.x] += add;
+      __syncthreads();
+    }
+    const int incl = s_part[threadIdx.x];
+    const int carry = s_carry;
+    if (e < E) offsets[e] = carry + incl - run;
+    __syncthreads();
+    if (threadIdx.x == 1023) s_carry = carry + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offsets[E] = s_carry;
+}
+
+__global__ void __launch_bounds__(kWarps * 32) slot_kernel(
+    const int32_t* __restrict__ topk_idx, const float* __restrict__ gates,
+    const int32_t* __restrict__ offsets, const int32_t* __restrict__ cta_base, int T, int E,
+    int k, int32_t* __restrict__ slot, int32_t* __restrict__ row_token,
+    float* __restrict__ row_gate, int* status) {
+  extern __shared__ unsigned s_mem[];
+  unsigned* masks = s_mem;                                          // [kWarps][E]
+  int* wbase = reinterpret_cast<int*>(s_mem + kWarps * E);          // [kWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
+  __syncthreads();
+  const int t = blockIdx.x * kRouteTokensPerCta + threadIdx.x;
+  const bool live = t < T;
+  if (live) {
+    for (int j = 0; j < k; ++j) {
+      const int e = topk_idx[(int64_t)t * k + j];
+      if (e >= 0 && e < E) atomicOr(&masks[warp * E + e], 1u << lane);
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = offsets[e] + cta_base[(int64_t)blockIdx.x * E + e];
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      wbase[w * E + e] = run;
+      run += __popc(masks[w * E + e]);
+    }
+  }
+  __syncthreads();
+  if (live) {
+    const unsigned lower = (1u << lane) - 1u;
+    for (int j = 0; j < k; ++j) {
+      const int e = topk_idx[(int64_t)t * k + j];
+      if (e < 0 || e >= E) {
+        set_status(status, MOE_DEV_BAD_INDEX);
+        slot[(int64_t)t * k + j] = -1;
+        continue;
+      }
+      const int s = wbase[warp * E + e] + __popc(masks[warp * E + e] & lower);
+      slot[(int64_t)t * k + j] = s;
+      row_token[s] = t;
+      row_gate[s] = gates[(int64_t)t * k + j];
+    }
+  }
+}
+
+template <int NPL>
+cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gates,
+                        int32_t* hist, cudaStream_t s) {
+  const int ctas = route_ctas(T);
+  topk_kernel<NPL><<<ctas, kWarps * 32, E * sizeof(int), s>>>(logits, T, E, k, idx, gates, hist);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------- router GEMM
+// C[m, n] = sum_k A[m*sam + k*sak] * B[k*sbk + n*sbn], 32x32 output tile per block of
+// 256 threads (4 outputs each), fp32 accumulation.
+template <typename TA, typename TB, typename TC>
+__global__ void __launch_bounds__(256) router_gemm_kernel(int M, int N, int K, const TA* A,
+                                                          int64_t sam, int64_t sak, const TB* B,
+                                                          int64_t sbk, int64_t sbn, TC* C,
+                                                          int accumulate) {
+  __shared__ float sA[32][33];
+  __shared__ float sB[32][33];
+  const int m0 = blockIdx.y * 32, n0 = blockIdx.x * 32;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;   // ty in 0..7
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int k0 = 0; k0 < K; k0 += 32) {
+    for (int r = ty; r < 32; r += 8) {
+      const int m = m0 + r, kk = k0 + tx;
+      sA[r][tx] = (m < M && kk < K) ? Elem<TA>::to_f(A[m * sam + kk * sak]) : 0.f;
+      const int kb = k0 + r, n = n0 + tx;
+      sB[r][tx] = (kb < K && n < N) ? Elem<TB>::to_f(B[kb * sbk + n * sbn]) : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < 32; ++kk) {
+      const float b = sB[kk][tx];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i] += sA[ty + 8 * i][kk] * b;
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int m = m0 + ty + 8 * i, n = n0 + tx;
+    if (m < M && n < N) {
+      float v = acc[i];
+      if (accumulate) v += Elem<TC>::to_f(C[(int64_t)m * N + n]);
+      C[(int64_t)m * N + n] = Elem<TC>::from_f(v);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
+                         int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
+                         float* row_gate, int32_t* hist, int32_t* cta_base, int* status,
+                         cudaStream_t s) {
+  const int T = d.T, E = d.E, k = d.k;
+  const int ctas = route_ctas(T);
+  cudaError_t err;
+  const int npl = (E + 31) / 32;
+  if (npl <= 1) err = launch_topk<1>(logits, T, E, k, topk_idx, gates, hist, s);
+  else if (npl <= 2) err = launch_topk<2>(logits, T, E, k, topk_idx, gates, hist, s);
+  else if (npl <= 4) err = launch_topk<4>(logits, T, E, k, topk_idx, gates, hist, s);
+  else if (npl <= 8) err = launch_topk<8>(logits, T, E, k, topk_idx, gates, hist, s);
+  else if (npl <= 16) err = launch_topk<16>(logits, T, E, k, topk_idx, gates, hist, s);
+  else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, s);
+  if (err != cudaSuccess) return err;
+  scan_kernel<<<1, 1024, 0, s>>>(hist, ctas, E, cta_base, counts, offsets);
+  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  const size_t smem = size_t(2) * kWarps * E * sizeof(int);
+  if (smem > 48 * 1024) {
+    err = cudaFuncSetAttribute(slot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
+    if (err != cudaSuccess) return err;
+  }
+  slot_kernel<<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, T, E, k, slot,
+                                              row_token, row_gate, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A, int64_t sam,
+                               int64_t sak, bool a_is_act, const void* B, int64_t sbk,
+                               int64_t sbn, bool b_is_act, void* C, bool c_is_act,
+                               bool accumulate, cudaStream_t s) {
+  dim3 grid((N + 31) / 32, (M + 31) / 32);
+  using bf = __nv_bfloat16;
+#define MOE_RG(TA, TB, TC)                                                                     \
+  router_gemm_kernel<TA, TB, TC><<<grid, 256, 0, s>>>(M, N, K, (const TA*)A, sam, sak,           \
+                                                      (const TB*)B, sbk, sbn, (TC*)C,             \
+                                                      accumulate ? 1 : 0)
+  if (fp32_act) {
+    // every operand is float
+    MOE_RG(float, float, float);
+  } else if (a_is_act && b_is_act && !c_is_act) {
+    MOE_RG(bf, bf, float);          // logits = x . Wr
+  } else if (!a_is_act && b_is_act && !c_is_act) {
+    MOE_RG(float, bf, float);       // d_logits . Wr^T into a float buffer
+  } else if (a_is_act && !b_is_act && c_is_act) {
+    MOE_RG(bf, float, bf);          // dWr = x^T . d_logits
+  } else {
+    return cudaErrorInvalidValue;
+  }
+#undef MOE_RG
+  return cudaGetLastError();
+}
+
+}  // namespace moe

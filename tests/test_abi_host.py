@@ -1,0 +1,118 @@
+"""Host-side checks of the C ABI that need no GPU: exports, descriptor and pointer
+validation, workspace and saved-buffer sizing.  No call here reaches a kernel."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+from routing_grouped_gemm_route_b200 import lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_symbols():
+    src = open(os.path.join(ROOT, "include", "moe.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:moe_status|const char\*)\s+(moe_\w+)\s*\(", src, re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from routing_grouped_gemm_route_b200 import build
+    build.build()
+    return lib.load()
+
+
+def test_every_declared_symbol_is_exported(L):
+    declared = header_symbols()
+    assert len(declared) >= 17
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r" T (moe_\w+)$", out, re.M))
+    assert set(declared) <= exported, set(declared) - exported
+    assert sorted(lib.EXPORTS) == declared
+
+
+@pytest.mark.parametrize("args,code", [
+    ((512, 128, 256, 8, 2, "fp32"), 0),
+    ((16384, 2048, 1024, 128, 4, "bf16"), 0),
+    ((0, 128, 64, 1, 1, "bf16"), 0),                  # no tokens is valid
+    ((10, 100, 64, 8, 2, "bf16"), lib.MOE_EINVAL),    # d not a multiple of 128
+    ((10, 128, 32, 8, 2, "bf16"), lib.MOE_EINVAL),    # d_ff not a multiple of 64
+    ((10, 128, 64, 8, 9, "bf16"), lib.MOE_EINVAL),    # k > E
+    ((10, 128, 64, 8, 0, "bf16"), lib.MOE_EINVAL),    # k < 1
+    ((10, 128, 64, 1025, 2, "bf16"), lib.MOE_EINVAL), # E > 1024
+    ((10, 128, 64, 64, 33, "bf16"), lib.MOE_EINVAL),  # k > 32
+    ((-1, 128, 64, 8, 2, "bf16"), lib.MOE_EINVAL),
+    ((2 ** 29, 128, 64, 8, 4, "bf16"), lib.MOE_EINVAL),  # T*k >= 2^31
+    ((10, 128, 64, 8, 2, "mxfp8"), lib.MOE_EUNSUPPORTED),
+])
+def test_descriptor_checks(L, args, code):
+    assert lib.moe_check_desc(lib.make_desc(*args)) == code
+
+
+def test_flag_checks(L):
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 8)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
+                                            lib.MOE_FLAG_ACCUM_DW)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
+                                            lib.MOE_FLAG_ACCUM_DW | lib.MOE_FLAG_DW_FP32)) == 0
+
+
+def test_sizes_grow_with_the_problem(L):
+    small = lib.moe_workspace_size(lib.make_desc(512, 128, 256, 8, 2, "fp32", lib.MOE_FLAG_ROUTER))
+    big = lib.moe_workspace_size(lib.make_desc(16384, 2048, 1024, 128, 4, "bf16"))
+    assert 0 < small < big
+    d = lib.make_desc(16384, 2048, 1024, 128, 4, "bf16")
+    s = lib.moe_saved_layout_get(d)
+    R = 16384 * 4
+    # every saved tensor is 256-byte aligned and the buffers do not overlap
+    offs = [s.topk_idx, s.gates, s.counts, s.offsets, s.slot, s.row_token, s.row_gate, s.x_perm,
+            s.H13, s.a, s.y_perm]
+    assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
+    assert s.y_perm + R * 2048 * 2 <= s.total
+    assert s.H13 - s.x_perm >= R * 2048 * 2 and s.a - s.H13 >= R * 2048 * 2
+
+
+def _p(v):
+    return ctypes.c_void_p(v)
+
+
+def test_pointer_and_workspace_errors_before_any_launch(L):
+    d = lib.make_desc(64, 128, 64, 8, 2, "bf16")
+    ws_need = lib.moe_workspace_size(d)
+    good, bad = 0x10000, 0x10008
+    args = [_p(good)] * 8
+    # null output pointer
+    st = L.moe_route(ctypes.byref(d), _p(good), None, *args[2:8], _p(good), ws_need, None)
+    assert st == lib.MOE_EINVAL
+    # misaligned pointer
+    st = L.moe_route(ctypes.byref(d), _p(bad), *args[1:8], _p(good), ws_need, None)
+    assert st == lib.MOE_EALIGN
+    # workspace too small
+    st = L.moe_route(ctypes.byref(d), *args, _p(good), ws_need - 1, None)
+    assert st == lib.MOE_EWORKSPACE
+    # null workspace
+    st = L.moe_dispatch(ctypes.byref(d), _p(good), _p(good), _p(good), None, None, ws_need, None)
+    assert st == lib.MOE_EINVAL
+    # the MXFP8 scale-factor buffer is reserved
+    st = L.moe_dispatch(ctypes.byref(d), _p(good), _p(good), _p(good), _p(good), _p(good),
+                        ws_need, None)
+    assert st == lib.MOE_EINVAL
+    # saved buffer too small for the layer forward
+    s = lib.moe_saved_layout_get(d)
+    st = L.moe_layer_fwd(ctypes.byref(d), _p(good), _p(good), None, _p(good), _p(good), _p(good),
+                         _p(good), s.total - 256, _p(good), ws_need, None)
+    assert st == lib.MOE_EWORKSPACE
+    # router flag requires Wr
+    dr = lib.make_desc(64, 128, 64, 8, 2, "bf16", lib.MOE_FLAG_ROUTER)
+    st = L.moe_layer_fwd(ctypes.byref(dr), _p(good), None, None, _p(good), _p(good), _p(good),
+                         _p(good), 1 << 40, _p(good), 1 << 40, None)
+    assert st == lib.MOE_EINVAL
+    assert L.moe_check_desc(None) == lib.MOE_EINVAL
+
+
+def test_status_strings(L):
+    for code in (0, -1, -2, -3, -4, -5, -6):
+        assert lib.status_string(code) not in ("", "unknown status")

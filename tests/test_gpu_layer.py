@@ -1,0 +1,160 @@
+"""End-to-end layer fwd+bwd through moe_layer_fwd / moe_layer_bwd against the oracle.
+
+Small workloads are compared in full.  The timed workloads run at their full sizes
+in the same calls the bench times; their outputs are checked on sampled tokens and
+sampled experts, each recomputed by the oracle from the same inputs (a token's y,
+dx and d_logits depend only on that token's row and logits; an expert's dW on the
+tokens routed to it)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routing_grouped_gemm_route_b200 import lib
+from routing_grouped_gemm_route_b200.inputs import WORKLOADS, make_inputs
+
+from helpers import TOL, f64, npi, rel, run_layer, workload
+
+pytestmark = pytest.mark.gpu
+
+
+def oracle_layer(w, inp, logits=None):
+    x = f64(inp["x"])
+    W13, W2 = inp["W13"].float().numpy(), inp["W2"].float().numpy()
+    Wr = None if inp["Wr"] is None else f64(inp["Wr"])
+    L = logits if logits is not None else (None if inp["logits"] is None else f64(inp["logits"]))
+    fwd = oracle.layer_fwd(x, W13, W2, logits=L, Wr=None if L is not None else Wr, k=w.k)
+    bwd = oracle.layer_bwd(fwd, f64(inp["dy"]), x, W13, W2, Wr=Wr)
+    return fwd, bwd
+
+
+def check_full(w, flags=0):
+    inp = make_inputs(w)
+    desc, layer, dv, y, g, status = run_layer(w, inp, flags)
+    assert status == 0
+    v = layer.views()
+    # routing is judged on the logits the GPU routed on (injected, or its own x . Wr)
+    logits = f64(v["logits"]) if w.router else None
+    if w.router:
+        assert rel(v["logits"], f64(inp["x"]) @ f64(inp["Wr"])) < 1e-5
+    fwd, bwd = oracle_layer(w, inp, logits)
+    assert np.array_equal(npi(v["topk_idx"]), fwd["topk_idx"])
+    assert np.array_equal(npi(v["offsets"]), fwd["offsets"])
+    assert np.array_equal(npi(v["slot"]), fwd["slot"])
+    assert rel(y, fwd["y"]) < TOL
+    for name in ("dx", "d_logits", "dW13", "dW2"):
+        assert rel(g[name], bwd[name]) < TOL, name
+    if w.router:
+        # with the router, x gets d_logits . Wr^T as well, and Wr its own gradient
+        dWr = f64(inp["x"]).T @ bwd["d_logits"]
+        assert rel(g["dWr"], dWr) < TOL
+    return desc, layer, g
+
+
+def test_tiny_fp32_workload(cuda_lib):
+    check_full(WORKLOADS["tiny_fp32"])
+
+
+@pytest.mark.parametrize("T,d,E,k,f,dt,router,skew", [
+    (1000, 256, 8, 4, 128, "bf16", False, False),
+    (777, 128, 8, 2, 256, "bf16", True, False),
+    (2000, 256, 128, 4, 128, "bf16", False, False),
+    (2000, 256, 128, 4, 128, "bf16", False, True),
+    (333, 384, 12, 3, 192, "fp32", False, False),
+    (1, 128, 4, 2, 64, "bf16", False, False),
+])
+def test_small_layers(cuda_lib, T, d, E, k, f, dt, router, skew):
+    check_full(workload(T, d, E, k, f, dt, router, skew, seed=T))
+
+
+def test_fp32_weight_grads(cuda_lib):
+    w = workload(500, 256, 8, 2, 128, "bf16", seed=4)
+    _, _, g = check_full(w, lib.MOE_FLAG_DW_FP32)
+    assert g["dW13"].dtype == torch.float32
+
+
+def test_no_tokens(cuda_lib):
+    w = workload(0, 128, 4, 2, 64, "bf16")
+    inp = make_inputs(w)
+    desc, layer, dv, y, g, status = run_layer(w, inp)
+    assert status == 0
+    assert torch.all(g["dW13"] == 0) and torch.all(g["dW2"] == 0)
+    assert int(layer.views()["offsets"].sum()) == 0
+
+
+def test_layer_replays_in_a_cuda_graph(cuda_lib):
+    """The whole fwd+bwd captures in one CUDA graph (no host round trip anywhere) and
+    replays with new logits, matching an uncaptured run."""
+    w = workload(3000, 256, 16, 4, 128, "bf16", seed=8)
+    inp = make_inputs(w)
+    desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, "bf16")
+    layer = lib.Layer(desc)
+    dv = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    y = torch.empty(w.T, w.d, dtype=torch.bfloat16, device="cuda")
+    out = dict(dx=torch.empty_like(y), d_logits=torch.empty(w.T, w.E, device="cuda"),
+               dW13=torch.empty_like(dv["W13"]), dW2=torch.empty_like(dv["W2"]))
+    layer.fwd(dv["x"], dv["W13"], dv["W2"], logits=dv["logits"], y=y)   # warm-up (attributes)
+    layer.bwd(dv["dy"], dv["W13"], dv["W2"], out=out)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        layer.fwd(dv["x"], dv["W13"], dv["W2"], logits=dv["logits"], y=y)
+        layer.bwd(dv["dy"], dv["W13"], dv["W2"], out=out)
+    for seed in (101, 102):
+        w2 = w.replace(seed=seed)
+        newL = make_inputs(w2)["logits"]
+        dv["logits"].copy_(newL)
+        g.replay()
+        torch.cuda.synchronize()
+        inp2 = dict(inp, logits=newL)
+        fwd, bwd = oracle_layer(w, inp2)
+        assert np.array_equal(npi(layer.views()["topk_idx"]), fwd["topk_idx"])
+        assert rel(y, fwd["y"]) < TOL
+        assert rel(out["dW2"], bwd["dW2"]) < TOL
+        assert rel(out["d_logits"], bwd["d_logits"]) < TOL
+    assert lib.moe_read_device_status(layer.ws) == 0
+
+
+@pytest.mark.parametrize("name", ["e8_bf16", "e128_bf16", "e128_skew_bf16"])
+def test_full_size_workloads_sampled(cuda_lib, name):
+    """Full-size workloads, one layer fwd+bwd exactly as the bench runs it; outputs
+    checked on sampled tokens and experts."""
+    w = WORKLOADS[name]
+    inp = make_inputs(w, device="cuda")
+    desc, layer, dv, y, g, status = run_layer(w, {k: v for k, v in inp.items()})
+    assert status == 0
+    v = layer.views()
+    L = inp["logits"].cpu()
+    # routing over all tokens: bit-exact
+    ref = oracle.route(L.numpy(), w.k, w.E)
+    assert np.array_equal(npi(v["topk_idx"]), ref["topk_idx"])
+    assert np.array_equal(npi(v["offsets"]), ref["offsets"])
+    assert np.array_equal(npi(v["slot"]), ref["slot"])
+    assert np.array_equal(npi(v["row_token"]), ref["row_token"])
+    W13 = inp["W13"].float().cpu().numpy()
+    W2 = inp["W2"].float().cpu().numpy()
+    x, dy = inp["x"].cpu(), inp["dy"].cpu()
+    rng = np.random.default_rng(0)
+    # sampled tokens: y, dx, d_logits
+    toks = np.sort(rng.choice(w.T, size=96, replace=False))
+    toks[0], toks[-1] = 0, w.T - 1
+    fw = oracle.layer_fwd(f64(x[toks]), W13, W2, logits=f64(L[toks]), k=w.k)
+    bw = oracle.layer_bwd(fw, f64(dy[toks]), f64(x[toks]), W13, W2)
+    assert rel(y[toks], fw["y"]) < TOL
+    assert rel(g["dx"][toks], bw["dx"]) < TOL
+    assert rel(g["d_logits"][toks], bw["d_logits"]) < TOL
+    # sampled experts: dW over every token routed to the expert; empty experts exactly 0
+    counts = ref["counts"]
+    picks = [int(np.argmax(counts)), int(np.argmin(counts)), int(rng.integers(w.E))]
+    for e in dict.fromkeys(picks):
+        if counts[e] == 0:
+            assert torch.all(g["dW13"][e] == 0) and torch.all(g["dW2"][e] == 0)
+            continue
+        te = np.unique(ref["row_token"][ref["offsets"][e]:ref["offsets"][e + 1]])
+        if len(te) > 3000:
+            te = te[:3000]                   # bound the oracle's work on the hot expert
+            continue
+        fe = oracle.layer_fwd(f64(x[te]), W13, W2, logits=f64(L[te]), k=w.k)
+        be = oracle.layer_bwd(fe, f64(dy[te]), f64(x[te]), W13, W2)
+        assert rel(g["dW2"][e], be["dW2"][e]) < TOL, e
+        assert rel(g["dW13"][e], be["dW13"][e]) < TOL, e
