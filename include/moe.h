@@ -143,6 +143,30 @@ moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_id
                      int32_t* row_token, float* row_gate, void* ws, size_t ws_bytes,
                      void* stream);
 
+/* Size of the device array that moe_route_noalloc uses for its scratch (4 MiB). */
+#define MOE_ROUTE_NOALLOC_SCRATCH_BYTES (4 * 1024 * 1024)
+
+/* moe_route without a workspace.  The paper has no counterpart: this entry point is a
+ * library convenience for callers that cannot give the library device memory of its
+ * own -- for example a host framework or plugin that plans every device buffer ahead
+ * and passes only its input and output tensors, or a latency-critical caller that
+ * must not call cudaMalloc because it synchronises the device.
+ * Same arguments, outputs and results as moe_route, minus ws/ws_bytes.  Its scratch
+ * (per-CTA expert histograms and bases, 2 * ceil(T/256) * E int32) lives in one
+ * static device array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU which loads
+ * this library holds until the process exits; a descriptor that needs more returns
+ * MOE_EWORKSPACE before any launch (with E = 128 that allows T up to about 1M tokens,
+ * with E = 1024 about 130k).  The call allocates nothing and frees nothing.
+ * The first call on a device looks up the array's device address (once per device,
+ * with that device current); make that first call before any stream capture.
+ * All calls share the one array and it keeps the last call's contents (every call
+ * overwrites what it reads, so nothing needs clearing): calls that overlap on the
+ * GPU -- on different streams, or from different host threads -- race and must be
+ * serialised by the caller. */
+moe_status moe_route_noalloc(const moe_desc* desc, const float* logits, int32_t* topk_idx,
+                             float* gates, int32_t* counts, int32_t* offsets, int32_t* slot,
+                             int32_t* row_token, float* row_gate, void* stream);
+
 /* S5, row-wise dispatch: x_perm[slot[t,j]] = x[t] for every (t,j)
  * (unite.ai, "पैरालेलिज़्म, प्रिसीजन, और मेमोरी तकनीकें").  x [T,d] act, x_perm [R,d] act.
  * x_perm_sf is reserved for the MXFP8 layout and must be NULL.  A slot outside

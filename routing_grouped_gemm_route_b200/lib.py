@@ -21,12 +21,14 @@ MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE
 MOE_FP32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
 MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW = 1, 2, 4
 MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4
+MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 DTYPES = {"fp32": MOE_FP32, "bf16": MOE_BF16, "mxfp8": MOE_MXFP8}
 
 # Every entry point that include/moe.h declares.
 EXPORTS = ["moe_status_string", "moe_check_desc", "moe_workspace_size", "moe_saved_layout_get",
            "moe_workspace_init", "moe_read_device_status", "moe_router_logits", "moe_route",
+           "moe_route_noalloc",
            "moe_dispatch", "moe_grouped_gemm_fwd", "moe_combine", "moe_combine_bwd",
            "moe_grouped_gemm_bwd", "moe_dispatch_bwd", "moe_router_bwd", "moe_layer_fwd",
            "moe_layer_bwd"]
@@ -75,6 +77,7 @@ def load():
         "moe_read_device_status": [_P, _P, ctypes.POINTER(_I)],
         "moe_router_logits": [_P, _P, _P, _P, _P],
         "moe_route": [_P] + [_P] * 8 + [_P, _S, _P],
+        "moe_route_noalloc": [_P] + [_P] * 8 + [_P],
         "moe_dispatch": [_P, _P, _P, _P, _P, _P, _S, _P],
         "moe_grouped_gemm_fwd": [_P] + [_P] * 8 + [_P, _S, _P],
         "moe_combine": [_P, _P, _P, _P, _P, _P, _S, _P],
@@ -182,6 +185,16 @@ def moe_route(desc, logits, topk_idx, gates, counts, offsets, slot, row_token, r
     _check(load().moe_route(ctypes.byref(desc), _ptr(logits), _ptr(topk_idx), _ptr(gates),
                             _ptr(counts), _ptr(offsets), _ptr(slot), _ptr(row_token),
                             _ptr(row_gate), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_route")
+
+
+def moe_route_noalloc(desc, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate,
+                      stream=None):
+    """moe_route for callers that cannot provide a workspace: the scratch lives in a
+    fixed static device array inside the library (see include/moe.h)."""
+    _check(load().moe_route_noalloc(ctypes.byref(desc), _ptr(logits), _ptr(topk_idx),
+                                    _ptr(gates), _ptr(counts), _ptr(offsets), _ptr(slot),
+                                    _ptr(row_token), _ptr(row_gate), _stream(stream)),
+           "moe_route_noalloc")
 
 
 def moe_dispatch(desc, x, slot, x_perm, ws, x_perm_sf=None, stream=None):
