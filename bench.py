@@ -45,7 +45,11 @@ def parse():
     ap.add_argument("--router", action="store_true", help="compute logits = x.Wr on the device")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
-    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--e2e-steps", type=int, default=30, help="0 skips the end-to-end leg")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="override T (a smaller case of the workload, for profiling)")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="override E (a smaller case of the workload, for profiling)")
     return ap.parse_args()
 
 
@@ -222,6 +226,64 @@ def run_reference(args, w, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d_logits, dW13,
+            dW2, dWr):
+    """Same metric through the public whole-layer calls, with the step's inputs copied
+    from pinned host memory and its results copied back, all inside the timed region."""
+    from routing_grouped_gemm_route_b200 import lib
+    T, d, E = w.T, w.d, w.E
+    es = 4 if act == torch.float32 else 2
+    E2E = max(3, args.e2e_steps)
+
+    def z(*shape, dt=act):
+        return torch.empty(*shape, dtype=dt, device=dev)
+    hx = torch.empty(T, d, dtype=act, pin_memory=True)
+    hx.copy_(x.cpu())
+    hdy = torch.empty(T, d, dtype=act, pin_memory=True)
+    hdy.copy_(dy.cpu())
+    hl = None
+    if not w.router:
+        hl = torch.empty(T, E, dtype=torch.float32, pin_memory=True)
+        hl.copy_(logits.cpu())
+    hy = torch.empty(T, d, dtype=act, pin_memory=True)
+    hdx = torch.empty(T, d, dtype=act, pin_memory=True)
+    layer = lib.Layer(desc, device=dev)
+    x_in, dl_in, dy_in = z(T, d), (z(T, E, dt=torch.float32) if not w.router else None), z(T, d)
+    outs = dict(dx=dx, d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
+
+    def e2e_step():
+        x_in.copy_(hx, non_blocking=True)
+        if dl_in is not None:
+            dl_in.copy_(hl, non_blocking=True)
+        dy_in.copy_(hdy, non_blocking=True)
+        layer.fwd(x_in, W13, W2, logits=dl_in, Wr=Wr, y=y)
+        layer.bwd(dy_in, W13, W2, x=x_in, Wr=Wr, out=outs)
+        hy.copy_(y, non_blocking=True)
+        hdx.copy_(dx, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(E2E):
+        e2e_step()
+    e1.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
+    h2d = T * d * es * 2 + (0 if w.router else T * E * 4)
+    d2h = T * d * es * 2
+    e2e = {"value": world * T * E2E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": E2E,
+           "api": "moe_layer_fwd + moe_layer_bwd with pinned-host x, logits, dy in and y, dx out"}
+    if lib.moe_read_device_status(layer.ws) != 0:
+        raise RuntimeError("device status set during the end-to-end run")
+
+    return e2e
+
+
 # ------------------------------------------------------------------------------ our arm
 def main():
     args = parse()
@@ -229,6 +291,10 @@ def main():
     w = WORKLOADS[args.workload]
     if args.router:
         w = w.replace(router=True)
+    if args.tokens is not None:
+        w = w.replace(T=args.tokens, name=w.name + f"[T={args.tokens}]")
+    if args.experts is not None:
+        w = w.replace(E=args.experts, name=w.name + f"[E={args.experts}]")
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, w, world, rank)
@@ -371,50 +437,10 @@ def main():
                 if pk["source"] == "measured" else "fallback 1.4 PFLOP/s sustained"}
 
     # ---------------------------------------------------------------- end to end (host buffers)
-    E2E = max(3, min(args.e2e_steps, K))
-    hx = torch.empty(T, d, dtype=act, pin_memory=True)
-    hx.copy_(x.cpu())
-    hdy = torch.empty(T, d, dtype=act, pin_memory=True)
-    hdy.copy_(dy.cpu())
-    hl = None
-    if not w.router:
-        hl = torch.empty(T, E, dtype=torch.float32, pin_memory=True)
-        hl.copy_(logits.cpu())
-    hy = torch.empty(T, d, dtype=act, pin_memory=True)
-    hdx = torch.empty(T, d, dtype=act, pin_memory=True)
-    layer = lib.Layer(desc, device=dev)
-    dx_in, dl_in, dy_in = z(T, d), (z(T, E, dt=torch.float32) if not w.router else None), z(T, d)
-    outs = dict(dx=dx, d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
-
-    def e2e_step():
-        dx_in.copy_(hx, non_blocking=True)
-        if dl_in is not None:
-            dl_in.copy_(hl, non_blocking=True)
-        dy_in.copy_(hdy, non_blocking=True)
-        layer.fwd(dx_in, W13, W2, logits=dl_in, Wr=Wr, y=y)
-        layer.bwd(dy_in, W13, W2, x=dx_in, Wr=Wr, out=outs)
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
-
-    for _ in range(2):
-        e2e_step()
-    torch.cuda.synchronize()
-    barrier(world)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(E2E):
-        e2e_step()
-    e1.record()
-    torch.cuda.synchronize()
-    barrier(world)
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
-    h2d = T * d * es * 2 + (0 if w.router else T * E * 4)
-    d2h = T * d * es * 2
-    e2e = {"value": world * T * E2E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "steps": E2E,
-           "api": "moe_layer_fwd + moe_layer_bwd with pinned-host x, logits, dy in and y, dx out"}
-    if lib.moe_read_device_status(layer.ws) != 0:
-        raise RuntimeError("device status set during the end-to-end run")
+    e2e = None
+    if args.e2e_steps > 0:
+        e2e = run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d_logits,
+                      dW13, dW2, dWr)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
