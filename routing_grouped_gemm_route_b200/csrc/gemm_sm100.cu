@@ -8,21 +8,26 @@
 // memory, builds the tile list itself and walks it; the host never learns the
 // per-expert sizes.
 //
-// Kernel structure (one CTA per SM, 192 threads):
+// Kernel structure (one CTA per SM):
 //   warp 0      TMA producer: 128-byte-swizzled operand tiles into a ring of stages
 //   warp 1      tcgen05.mma issuer (one thread) + tensor-memory allocation
-//   warps 2..5  epilogue: tensor memory -> registers -> fused math -> global memory
+//   warps 2..   epilogue (4 warps, 8 for the math-heavy SwiGLU backward: two per
+//               tensor-memory lane quadrant, splitting the columns): tensor memory ->
+//               registers -> fused math -> swizzled shared memory -> TMA bulk tensor
+//               stores, one 32x32 chunk at a time
 // Two fp32 accumulators of 128 x BN live in tensor memory so the epilogue of one
 // tile overlaps the main loop of the next.
 //
 // Two groupings:
 //   RAGGED_M  forward and dgrad: expert e owns rows [off_e, off_e+1) of the routed
 //             activations; tiles of 128 rows start at off_e and rows past the
-//             expert's end are computed but never stored.
-//   RAGGED_K  wgrad: dW_e = G_e^T . X_e sums over the expert's rows; the last
-//             K-block of an expert is partial and its foreign rows are zeroed in
-//             shared memory before the MMA reads them.  An expert with no rows
-//             writes dW_e = 0.
+//             expert's end are computed but never stored (a 32-row slice that ends
+//             inside the expert is written with plain stores, row by row).
+//   RAGGED_K  wgrad: dW_e = G_e^T . X_e sums over the expert's rows.  G is read
+//             through a per-expert tensor map whose row extent ends at the
+//             expert's last row (built on the device from the offsets), so the
+//             last, partial K-block arrives with its foreign rows zero-filled by
+//             the TMA unit.  An expert with no rows writes dW_e = 0.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
@@ -43,7 +48,7 @@ enum { RAGGED_M = 0, RAGGED_K = 1 };
 enum { EPI_STORE = 0, EPI_SWIGLU_FWD = 1, EPI_SWIGLU_BWD = 2 };
 
 constexpr int BM = 128;
-constexpr int kThreads = 192;
+constexpr int kMaxE = 1024;
 
 struct Params {
   const int32_t* offsets;  // [E+1]
@@ -53,29 +58,52 @@ struct Params {
   int K;                   // RAGGED_M: reduction length
   int b_rows_per_expert;   // expert e's rows start at e * b_rows_per_expert in B's tensor map
   int f;                   // d_ff (SwiGLU epilogues)
-  void* out;               // main output
-  int64_t ldo;             // its row stride in elements (RAGGED_M)
+  void* out;               // main output (plain-store path of partial row slices)
+  int64_t ldo;             // its row stride in elements
   void* out_a;             // SwiGLU forward: a [R, f]
-  const void* aux;         // SwiGLU backward: H13 [R, 2f]
-  int out_fp32;            // RAGGED_K: dW element type is float
   int accumulate;          // RAGGED_K: dW += result (float dW only)
+  const CUtensorMap* a_maps;  // RAGGED_K: per-expert maps of G (row extent = off_e+1)
   int* status;
 };
 
-template <typename T, int BN>
+// PAIR: a cluster of two CTAs on two SMs computes 256-row tiles with cta_group::2 MMAs;
+// each CTA loads its 128 rows of A and half of the BN rows of B, so each SM moves a
+// third fewer operand bytes per MMA flop than a lone CTA with a 128 x BN tile.
+template <typename T, typename OutT, int BN, int EPI, bool PAIR = false, int MODE = RAGGED_M>
 struct Cfg {
   static constexpr int ES = sizeof(T);
   static constexpr int KB = 128 / ES;     // K elements per stage (one 128-byte swizzle row)
   static constexpr int MNB = 128 / ES;    // M/N elements per 128-byte block (M/N-major tiles)
   static constexpr int UK = 32 / ES;      // K of one MMA instruction
+  static constexpr int TM = PAIR ? 2 * BM : BM;     // tile rows (M) of the whole cluster
+  static constexpr int BNC = PAIR ? BN / 2 : BN;    // rows of B held by one CTA
   static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BN * 128;
+  static constexpr int B_BYTES = BNC * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int STAGES = (196 * 1024) / STAGE > 8 ? 8 : (196 * 1024) / STAGE;
   static constexpr int TMEM_COLS = 2 * BN;
+  // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there);
+  // elsewhere 4 warps keep up and leave more shared memory to the operand ring
+  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD ? 8 : 4;
+  static constexpr int THREADS = 64 + 32 * EPI_WARPS;
+  static constexpr int COLGRP = EPI_WARPS / 4;          // warps sharing one lane quadrant
+  static constexpr int NCH = BN / 32;                   // 32-column chunks per tile
+  static constexpr int WCH = NCH / COLGRP;              // chunks per epilogue warp
+  // epilogue shared memory per warp: output staging chunks of 32 rows x 32 columns
+  static constexpr int CH = 32 * 32 * sizeof(OutT);
+  static constexpr int NBUF = EPI == EPI_SWIGLU_FWD ? 3 : EPI == EPI_SWIGLU_BWD ? 0 : 2;
+  // SwiGLU backward: slots of prefetched H1/H3 input chunks (32 x 32 each); the dH1/dH3
+  // results are staged in place in the slot they were computed from
+  static constexpr int IN_SLOTS = EPI == EPI_SWIGLU_BWD ? (ES == 2 ? (WCH < 2 ? WCH : 2) : 1) : 0;
+  static constexpr int IN_CH = 2 * 32 * 32 * ES;
+  static constexpr int EPI_WARP = ((NBUF * CH + IN_SLOTS * IN_CH) + 1023) / 1024 * 1024;
+  static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP;
+  static constexpr int BAR_BYTES = 512;
+  static constexpr int BUDGET =
+      227 * 1024 - 1024 /*alignment*/ - BAR_BYTES - (2 * (kMaxE + 1) + 8) * 4 - EPI_BYTES;
+  static constexpr int STAGES = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
+  static_assert(STAGES >= 2, "shared memory budget");
   static constexpr size_t smem_bytes(int E) {
-    return 1024 /*alignment slack*/ + size_t(STAGES) * STAGE + 256 /*barriers, flags*/ +
-           size_t(2 * (E + 1) + 4) * sizeof(int);
+    return 1024 + size_t(STAGES) * STAGE + EPI_BYTES + BAR_BYTES + size_t(2 * (E + 1) + 8) * 4;
   }
 };
 
@@ -83,7 +111,7 @@ struct Tile {
   int e, n0, m0, row0, rows_end, kb, cnt;
 };
 
-template <int MODE, int BN, int KB>
+template <int MODE, int BN, int KB, int TM>
 __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int m_tiles, const int* s_off,
                                             const int* s_mt, int E, int K) {
   Tile tl;
@@ -96,7 +124,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int m_tiles, con
       if (s_mt[mid] <= mtg) lo = mid; else hi = mid;
     }
     tl.e = lo;
-    tl.m0 = (mtg - s_mt[lo]) * BM;
+    tl.m0 = (mtg - s_mt[lo]) * TM;
     tl.row0 = s_off[lo] + tl.m0;
     tl.rows_end = s_off[lo + 1];
     tl.n0 = nt * BN;
@@ -107,7 +135,7 @@ __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int m_tiles, con
     tl.e = t / per;
     const int r = t - tl.e * per;
     const int mt = r / n_tiles;
-    tl.m0 = mt * BM;
+    tl.m0 = mt * TM;
     tl.n0 = (r - mt * n_tiles) * BN;
     tl.row0 = s_off[tl.e];
     tl.rows_end = s_off[tl.e + 1];
@@ -127,31 +155,79 @@ __device__ __forceinline__ void store32(T* dst, const float* v) {
     stg16(dst + i, pk.raw);
   }
 }
+
+// One row of a 32 x 32 staging chunk in shared memory, laid out for a TMA box of
+// 32 x 32 elements: 64-byte rows with the 64-byte swizzle (16-bit elements) or 128-byte
+// rows with the 128-byte swizzle (32-bit elements).  Thread `r` owns row r; the XOR
+// spreads the 32 rows' 16-byte pieces over all banks.
 template <typename T>
-__device__ __forceinline__ void load32(const T* src, float* v) {
+__device__ __forceinline__ int swz_chunk(int j, int r) {
+  return sizeof(T) == 4 ? (j ^ (r & 7)) : (j ^ ((r >> 1) & 3));
+}
+template <typename T>
+__device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float* v) {
+  constexpr int RB = 32 * sizeof(T);
   constexpr int PER = 16 / sizeof(T);
+  uint8_t* row = buf + r * RB;
 #pragma unroll
-  for (int i = 0; i < 32; i += PER) {
+  for (int j = 0; j < RB / 16; ++j) {
     Vec16<T> pk;
-    pk.raw = *reinterpret_cast<const uint4*>(src + i);
-    pk.to_float(v + i);
+    pk.from_float(v + j * PER);
+    *reinterpret_cast<uint4*>(row + swz_chunk<T>(j, r) * 16) = pk.raw;
+  }
+}
+template <typename T>
+__device__ __forceinline__ void unstage_row(const uint8_t* buf, int r, float* v) {
+  constexpr int RB = 32 * sizeof(T);
+  constexpr int PER = 16 / sizeof(T);
+  const uint8_t* row = buf + r * RB;
+#pragma unroll
+  for (int j = 0; j < RB / 16; ++j) {
+    Vec16<T> pk;
+    pk.raw = *reinterpret_cast<const uint4*>(row + swz_chunk<T>(j, r) * 16);
+    pk.to_float(v + j * PER);
   }
 }
 
-__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + __expf(-z)); }
+// Logistic function with the fast exponential and fast division intrinsics; the exponent
+// is capped at 80 so the denominator stays finite (the result is then below 1e-34).
+__device__ __forceinline__ float sigmoid_f(float z) {
+  return __fdividef(1.0f, 1.0f + __expf(fminf(-z, 80.0f)));
+}
 
 __device__ __forceinline__ void bits_to_f32(const uint32_t* v, float* f) {
 #pragma unroll
   for (int i = 0; i < 32; ++i) f[i] = __uint_as_float(v[i]);
 }
 
-template <typename T, int BN, bool A_MN, bool B_MN, int MODE, int EPI>
-__global__ void __launch_bounds__(kThreads, 1)
+// Writes the 32 x 32 chunk held one row per lane through staging buffer `buf` with a TMA
+// store (or reduce-add) at (x, y).  `lane 0` owns the bulk groups; before refilling a
+// buffer it waits until at most NBUF-1 earlier groups still read shared memory.
+template <typename OutT, int NBUF>
+__device__ __forceinline__ void staged_store(uint8_t* buf, const float* v, int lane,
+                                             const void* tmap, int x, int y, bool reduce) {
+  if (lane == 0) bulk_wait_read<NBUF - 1>();
+  __syncwarp();
+  stage_row<OutT>(buf, lane, v);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    if (reduce) tma_reduce_add_2d(tmap, buf, x, y);
+    else tma_store_2d(tmap, buf, x, y);
+    bulk_commit();
+  }
+}
+
+template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
+__global__ void __launch_bounds__(Cfg<T, OutT, BN, EPI, PAIR, MODE>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                    const Params p) {
-  using C = Cfg<T, BN>;
+                    const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
+                    const __grid_constant__ CUtensorMap tmI, const Params p) {
+  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
   constexpr bool kTF32 = sizeof(T) == 4;
-  constexpr uint32_t IDESC = idesc_f32acc(BM, BN, kTF32 ? 2u : 1u, A_MN, B_MN);
+  constexpr uint32_t IDESC = idesc_f32acc(C::TM, BN, kTF32 ? 2u : 1u, A_MN, B_MN);
+  static_assert(!PAIR || !kTF32, "CTA pairs run the 16-bit kernels");
+  static_assert(!B_MN || C::BNC % C::MNB == 0, "an M/N-major B half is whole 128-byte blocks");
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
   static_assert(MODE == RAGGED_M || (A_MN && B_MN && EPI == EPI_STORE), "wgrad layout");
 
@@ -159,24 +235,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint64_t* full = reinterpret_cast<uint64_t*>(tiles + C::STAGES * C::STAGE);
+  uint8_t* epi_smem = tiles + C::STAGES * C::STAGE;
+  uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* fin = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
+  uint64_t* in_full = fin + 1;                                   // [EPI_WARPS][IN_SLOTS]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(full) + C::BAR_BYTES / 4 - 4;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_total = reinterpret_cast<int*>(tmem_slot + 2);
-  int* s_off = s_total + 2;
+  int* s_off = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(full) + C::BAR_BYTES);
   int* s_mt = s_off + (p.E + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int E = p.E;
   const int n_tiles = p.N / BN;
-  const int m_tiles = MODE == RAGGED_K ? p.M / BM : 0;
+  const int m_tiles = MODE == RAGGED_K ? p.M / C::TM : 0;
+  // CTA pair: rank 0 (leader) issues the MMAs and owns the shared full/tempty barriers
+  const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+  const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
+  const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-  for (int i = threadIdx.x; i <= E; i += kThreads) s_off[i] = p.offsets[i];
+  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = p.offsets[i];
   __syncthreads();
 
   if (warp == 0) {
@@ -188,7 +270,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       if (e < E) {
         const int c = s_off[e + 1] - s_off[e];
         if (c < 0) ok = 0;
-        mt = c > 0 ? (c + BM - 1) / BM : 0;
+        mt = c > 0 ? (c + C::TM - 1) / C::TM : 0;
       }
       int incl = mt;
 #pragma unroll
@@ -214,21 +296,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       }
       for (int a = 0; a < 2; ++a) {
         mbar_init(&tfull[a], 1);
-        mbar_init(&tempty[a], 4);
+        mbar_init(&tempty[a], C::EPI_WARPS * (PAIR ? 2 : 1));
       }
       mbar_init(fin, 1);
+      for (int i = 0; i < C::EPI_WARPS * C::IN_SLOTS; ++i) mbar_init(&in_full[i], 1);
       fence_mbar_init();
     }
   }
   __syncthreads();
   const int total = s_total[0];
-  if (static_cast<int>(blockIdx.x) >= total) return;   // uniform over the CTA
+  if (unit >= total) return;   // uniform over the CTA (and over a CTA pair)
 
-  if (warp == 1) tmem_alloc(tmem_slot, C::TMEM_COLS);
+  if (warp == 1) {
+    if (PAIR) tmem_alloc_pair(tmem_slot, C::TMEM_COLS);
+    else tmem_alloc(tmem_slot, C::TMEM_COLS);
+  }
   tc_fence_before();
-  __syncthreads();
+  if (PAIR) cluster_sync();   // barriers of both CTAs initialised, TMEM allocated
+  else __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  const bool leader = rank == 0;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -239,42 +327,60 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
       bool stop = false;
-      for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-        const Tile tl = decode_tile<MODE, BN, C::KB>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
+      // In a pair, both CTAs' loads complete on the leader's full barrier; only the
+      // leader arms it (with both CTAs' bytes).  The follower may land its bytes before
+      // the leader arms the phase: the transaction count goes transiently negative and
+      // the phase still waits for the leader's arrival.
+      const uint32_t full_leader = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;
+      const int arow = PAIR ? static_cast<int>(rank) * BM : 0;         // my rows of A
+      const int bcol = PAIR ? static_cast<int>(rank) * C::BNC : 0;     // my rows of B
+      for (int t = unit; t < total && !stop; t += n_units) {
+        const Tile tl = decode_tile<MODE, BN, C::KB, C::TM>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
         for (int kb = 0; kb < tl.kb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { stop = true; break; }
           uint8_t* sA = tiles + stage * C::STAGE;
           uint8_t* sB = sA + C::A_BYTES;
-          mbar_arrive_expect_tx(&full[stage], C::STAGE);
-          armed |= 1u << stage;
-          armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          if (leader) {
+            mbar_arrive_expect_tx(&full[stage], C::STAGE * (PAIR ? 2 : 1));
+            armed |= 1u << stage;
+            armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
+          }
+          const uint32_t fb = full_leader + static_cast<uint32_t>(stage) * 8u;
+          auto load = [&](void* dst, const CUtensorMap* tm, int x, int y) {
+            if (PAIR) tma_load_2d_pair(dst, tm, fb, x, y);
+            else tma_load_2d(dst, tm, &full[stage], x, y);
+          };
           const int k0 = kb * C::KB;
           if (MODE == RAGGED_M) {
-            tma_load_2d(sA, &tmA, &full[stage], k0, tl.row0);
+            load(sA, &tmA, k0, tl.row0 + arow);
             const int brow = tl.e * p.b_rows_per_expert;
             if (!B_MN) {
               if (EPI == EPI_SWIGLU_FWD) {
+                // B rows: the gate block W1[h0, h0+BN/2) then the up block W3[h0, ...)
                 const int h0 = tl.n0 / 2;
-                tma_load_2d(sB, &tmB, &full[stage], k0, brow + h0);
-                tma_load_2d(sB + (BN / 2) * 128, &tmB, &full[stage], k0, brow + p.f + h0);
+                if (PAIR) {
+                  load(sB, &tmB, k0, brow + (rank ? p.f : 0) + h0);
+                } else {
+                  load(sB, &tmB, k0, brow + h0);
+                  load(sB + (BN / 2) * 128, &tmB, k0, brow + p.f + h0);
+                }
               } else {
-                tma_load_2d(sB, &tmB, &full[stage], k0, brow + tl.n0);
+                load(sB, &tmB, k0, brow + tl.n0 + bcol);
               }
             } else {
 #pragma unroll
-              for (int i = 0; i < BN / C::MNB; ++i)
-                tma_load_2d(sB + i * C::KB * 128, &tmB, &full[stage], tl.n0 + i * C::MNB,
-                            brow + k0);
+              for (int i = 0; i < C::BNC / C::MNB; ++i)
+                load(sB + i * C::KB * 128, &tmB, tl.n0 + bcol + i * C::MNB, brow + k0);
             }
           } else {
+            const CUtensorMap* am = p.a_maps + tl.e;
+            if (kb == 0) fence_tmap_acquire(am);   // written by the map-building kernel
 #pragma unroll
             for (int i = 0; i < BM / C::MNB; ++i)
-              tma_load_2d(sA + i * C::KB * 128, &tmA, &full[stage], tl.m0 + i * C::MNB,
-                          tl.row0 + k0);
+              load(sA + i * C::KB * 128, am, tl.m0 + arow + i * C::MNB, tl.row0 + k0);
 #pragma unroll
-            for (int i = 0; i < BN / C::MNB; ++i)
-              tma_load_2d(sB + i * C::KB * 128, &tmB, &full[stage], tl.n0 + i * C::MNB,
-                          tl.row0 + k0);
+            for (int i = 0; i < C::BNC / C::MNB; ++i)
+              load(sB + i * C::KB * 128, &tmB, tl.n0 + bcol + i * C::MNB, tl.row0 + k0);
           }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -284,187 +390,275 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (armed & (1u << s)) mbar_wait_teardown(&full[s], (armed_par >> s) & 1u);
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == 1 && leader) {
     // ------------------------------------------------------------------ MMA issuer
-    int stage = 0;
-    uint32_t phase = 0;
-    int acc = 0;
-    uint32_t acc_phase = 0;
-    bool stop = false;
-    for (int t = blockIdx.x; t < total && !stop; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE, BN, C::KB>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
-      if (!mbar_wait_warp(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
-      for (int kb = 0; kb < tl.kb; ++kb) {
-        if (!mbar_wait_warp(&full[stage], phase, abort_flag, p.status)) { stop = true; break; }
+    if (lane == 0) {
+      // Descriptors of stage 0; a stage or K step only moves the start-address field
+      // (bits [0,14) in 16-byte units; shared addresses stay below 256 KB).
+      constexpr uint32_t MN_LAYOUT = kTF32 ? kLayoutSW128Atom32 : kLayoutSW128;
+      constexpr uint32_t MN_SBO = kTF32 ? 512 : 1024;   // M/N-major TF32: 4-row K groups
+      const uint32_t a0 = smem_u32(tiles);
+      const uint64_t a_desc0 = A_MN ? sdesc(a0, C::KB * 128, MN_SBO, MN_LAYOUT)
+                                    : sdesc(a0, 16, 1024, kLayoutSW128);
+      const uint64_t b_desc0 = B_MN ? sdesc(a0 + C::A_BYTES, C::KB * 128, MN_SBO, MN_LAYOUT)
+                                    : sdesc(a0 + C::A_BYTES, 16, 1024, kLayoutSW128);
+      constexpr uint32_t A_STEP = (A_MN ? C::UK * 128 : 32) >> 4;   // per MMA along K
+      constexpr uint32_t B_STEP = (B_MN ? C::UK * 128 : 32) >> 4;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      bool stop = false;
+      for (int t = unit; t < total && !stop; t += n_units) {
+        const Tile tl =
+            decode_tile<MODE, BN, C::KB, C::TM>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
         tc_fence_after();
-        uint8_t* sA = tiles + stage * C::STAGE;
-        if (MODE == RAGGED_K && kb == tl.kb - 1) {
-          const int valid = tl.cnt - kb * C::KB;
-          if (valid < C::KB) {
-            // Rows [valid, KB) of this K-block belong to later experts: zero them in A.
-            const int rows = C::KB - valid;
-            const int per_blk = rows * 8;   // 16-byte chunks per M block
-            for (int i = lane; i < (BM / C::MNB) * per_blk; i += 32) {
-              const int blk = i / per_blk;
-              const int rem = i - blk * per_blk;
-              uint8_t* dst = sA + blk * C::KB * 128 + (valid + (rem >> 3)) * 128 + (rem & 7) * 16;
-              *reinterpret_cast<uint4*>(dst) = make_uint4(0u, 0u, 0u, 0u);
-            }
-            fence_proxy_async_smem();
-          }
-          __syncwarp();
-        }
-        if (lane == 0) {
-          const uint32_t a_base = smem_u32(sA);
-          const uint32_t b_base = a_base + C::A_BYTES;
-          // M/N-major TF32 tiles use the 32-byte-atom swizzle (4-row K groups)
-          constexpr uint32_t MN_LAYOUT = kTF32 ? kLayoutSW128Atom32 : kLayoutSW128;
-          constexpr uint32_t MN_SBO = kTF32 ? 512 : 1024;
+        const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
+        for (int kb = 0; kb < tl.kb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { stop = true; break; }
+          tc_fence_after();
+          const uint32_t so = static_cast<uint32_t>(stage * C::STAGE) >> 4;
 #pragma unroll
           for (int kk = 0; kk < C::KB / C::UK; ++kk) {
-            const uint64_t ad =
-                A_MN ? sdesc(a_base + kk * C::UK * 128, C::KB * 128, MN_SBO, MN_LAYOUT)
-                     : sdesc(a_base + kk * 32, 16, 1024, kLayoutSW128);
-            const uint64_t bd =
-                B_MN ? sdesc(b_base + kk * C::UK * 128, C::KB * 128, MN_SBO, MN_LAYOUT)
-                     : sdesc(b_base + kk * 32, 16, 1024, kLayoutSW128);
-            umma<kTF32>(d_tmem, ad, bd, IDESC, (kb | kk) != 0 ? 1u : 0u);
+            const uint64_t ad = a_desc0 + so + kk * A_STEP;
+            const uint64_t bd = b_desc0 + so + kk * B_STEP;
+            const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
+            if (PAIR) umma_pair(d_tmem, ad, bd, IDESC, accum);
+            else umma<kTF32>(d_tmem, ad, bd, IDESC, accum);
           }
-          umma_commit(&empty[stage]);
+          if (PAIR) umma_commit_pair(&empty[stage], 3);   // frees the stage in both CTAs
+          else umma_commit(&empty[stage]);
+          if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
-        __syncwarp();
-        if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
+        if (PAIR) umma_commit_pair(&tfull[acc], 3);
+        else umma_commit(&tfull[acc]);
+        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
       }
-      if (lane == 0) umma_commit(&tfull[acc]);
-      __syncwarp();
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
-    }
-    if (lane == 0) {
-      umma_commit(fin);
+      // (a kernel's tcgen05 instructions all use one cta_group)
+      if (PAIR) umma_commit_pair(fin, 1);
+      else umma_commit(fin);
       mbar_wait_teardown(fin, 0);
     }
     __syncwarp();
-  } else {
+  } else if (warp >= 2) {
     // ------------------------------------------------------------------ epilogue
     const int q = warp & 3;                 // tensor-memory lane quadrant of this warp
-    const int r = q * 32 + lane;            // tile row
+    const int ew = warp - 2;                // epilogue warp index (shared-memory slice)
+    const int cg = ew >> 2;                 // column group: chunks [cg*WCH, (cg+1)*WCH)
+    uint8_t* stage_buf = epi_smem + ew * C::EPI_WARP;
+    uint8_t* in_buf = stage_buf + C::NBUF * C::CH;
+    constexpr int INS = C::IN_SLOTS > 0 ? C::IN_SLOTS : 1;   // slot-ring modulus
+    uint64_t* my_in_full = in_full + ew * INS;
+    int sbuf = 0;
+    uint32_t in_issued = 0, in_used = 0;    // SwiGLU-backward input chunks
     int acc = 0;
     uint32_t acc_phase = 0;
-    for (int t = blockIdx.x; t < total; t += gridDim.x) {
-      const Tile tl = decode_tile<MODE, BN, C::KB>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
+    uint32_t v[32];
+    float fv[32];
+    const uint32_t tempty_leader = PAIR ? map_to_rank(smem_u32(tempty), 0) : 0u;
+    const int myrow = PAIR ? static_cast<int>(rank) * BM : 0;      // my 128 rows of the tile
+    for (int t = unit; t < total; t += n_units) {
+      const Tile tl = decode_tile<MODE, BN, C::KB, C::TM>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
+      const int rbase = MODE == RAGGED_M ? tl.row0 + myrow + q * 32 : 0;   // first row of my slice
+      int nvalid = 32;
+      if (MODE == RAGGED_M) {
+        nvalid = tl.rows_end - rbase;
+        nvalid = nvalid < 0 ? 0 : (nvalid > 32 ? 32 : nvalid);
+      }
+      const bool whole = nvalid == 32;
+      const int cfirst = cg * C::WCH;       // my first 32-column chunk
+      if (EPI == EPI_SWIGLU_BWD && nvalid > 0) {
+        // prefetch this slice's H1/H3 chunks while the main loop still runs (the slots'
+        // previous results must have been read out by their TMA stores first)
+        if (lane == 0) {
+          bulk_wait_read<0>();
+          for (int i = 0; i < C::WCH && i < C::IN_SLOTS; ++i) {
+            const int slot = in_issued % INS;
+            const int x = tl.n0 + (cfirst + i) * 32;
+            uint8_t* dst = in_buf + slot * C::IN_CH;
+            mbar_arrive_expect_tx(&my_in_full[slot], C::IN_CH);
+            tma_load_2d(dst, &tmI, &my_in_full[slot], x, rbase);
+            tma_load_2d(dst + C::IN_CH / 2, &tmI, &my_in_full[slot], p.f + x, rbase);
+            ++in_issued;
+          }
+        }
+        in_issued = __shfl_sync(0xffffffffu, in_issued, 0);
+      }
       if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, p.status)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
-      uint32_t v[32];
       if (MODE == RAGGED_M) {
-        const int64_t grow = tl.row0 + r;
-        const bool valid = grow < tl.rows_end;
-        if (EPI == EPI_STORE) {
-          T* out = reinterpret_cast<T*>(p.out) + grow * p.ldo + tl.n0;
+        const int64_t grow = rbase + lane;
+        const bool valid = lane < nvalid;
+        if (nvalid > 0) {
+          if (EPI == EPI_STORE) {
 #pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
-            tmem_ld32(tb + c, v);
-            tmem_ld_wait();
-            reg_fence32(v);
-            if (valid) {
-              float fv[32];
+            for (int c = 0; c < BN; c += 32) {
+              tmem_ld32(tb + c, v);
+              tmem_ld_wait();
+              reg_fence32(v);
               bits_to_f32(v, fv);
-              store32<T>(out + c, fv);
-            }
-          }
-        } else if (EPI == EPI_SWIGLU_FWD) {
-          const int h0 = tl.n0 / 2;
-          T* h13 = reinterpret_cast<T*>(p.out) + grow * (2 * (int64_t)p.f) + h0;
-          T* aa = reinterpret_cast<T*>(p.out_a) + grow * (int64_t)p.f + h0;
-          uint32_t v3[32];
-#pragma unroll 1
-          for (int c = 0; c < BN / 2; c += 32) {
-            tmem_ld32(tb + c, v);
-            tmem_ld32(tb + BN / 2 + c, v3);
-            tmem_ld_wait();
-            reg_fence32(v);
-            reg_fence32(v3);
-            if (valid) {
-              float h1[32], h3[32];
-              bits_to_f32(v, h1);
-              bits_to_f32(v3, h3);
-              store32<T>(h13 + c, h1);
-              store32<T>(h13 + p.f + c, h3);
-              float av[32];
-#pragma unroll
-              for (int i = 0; i < 32; ++i) av[i] = h1[i] * sigmoid_f(h1[i]) * h3[i];
-              store32<T>(aa + c, av);
-            }
-          }
-        } else {  // EPI_SWIGLU_BWD: accumulator = dA
-          const T* h13 = reinterpret_cast<const T*>(p.aux) + grow * (2 * (int64_t)p.f) + tl.n0;
-          T* dh = reinterpret_cast<T*>(p.out) + grow * (2 * (int64_t)p.f) + tl.n0;
-#pragma unroll 1
-          for (int c = 0; c < BN; c += 32) {
-            tmem_ld32(tb + c, v);
-            tmem_ld_wait();
-            reg_fence32(v);
-            if (valid) {
-              float h1[32], h3[32], d1[32], d3[32], da[32];
-              load32<T>(h13 + c, h1);
-              load32<T>(h13 + p.f + c, h3);
-              bits_to_f32(v, da);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) {
-                const float s = sigmoid_f(h1[i]);
-                d1[i] = da[i] * h3[i] * s * (1.0f + h1[i] * (1.0f - s));
-                d3[i] = da[i] * h1[i] * s;
+              if (whole) {
+                staged_store<OutT, C::NBUF>(stage_buf + sbuf * C::CH, fv, lane, &tmO, tl.n0 + c,
+                                            rbase, false);
+                sbuf = sbuf + 1 == C::NBUF ? 0 : sbuf + 1;
+              } else if (valid) {
+                store32<OutT>(reinterpret_cast<OutT*>(p.out) + grow * p.ldo + tl.n0 + c, fv);
               }
-              store32<T>(dh + c, d1);
-              store32<T>(dh + p.f + c, d3);
+            }
+          } else if (EPI == EPI_SWIGLU_FWD) {
+            const int h0 = tl.n0 / 2;
+            uint32_t v3[32];
+            float h3[32], av[32];
+#pragma unroll 1
+            for (int c = 0; c < BN / 2; c += 32) {
+              tmem_ld32(tb + c, v);
+              tmem_ld32(tb + BN / 2 + c, v3);
+              tmem_ld_wait();
+              reg_fence32(v);
+              reg_fence32(v3);
+              bits_to_f32(v, fv);
+              bits_to_f32(v3, h3);
+#pragma unroll
+              for (int i = 0; i < 32; ++i) av[i] = fv[i] * sigmoid_f(fv[i]) * h3[i];
+              if (whole) {
+                staged_store<OutT, C::NBUF>(stage_buf + 0 * C::CH, fv, lane, &tmO, h0 + c, rbase,
+                                            false);
+                staged_store<OutT, C::NBUF>(stage_buf + 1 * C::CH, h3, lane, &tmO, p.f + h0 + c,
+                                            rbase, false);
+                staged_store<OutT, C::NBUF>(stage_buf + 2 * C::CH, av, lane, &tmO2, h0 + c, rbase,
+                                            false);
+              } else if (valid) {
+                OutT* h13 = reinterpret_cast<OutT*>(p.out) + grow * (2 * (int64_t)p.f) + h0 + c;
+                store32<OutT>(h13, fv);
+                store32<OutT>(h13 + p.f, h3);
+                store32<OutT>(reinterpret_cast<OutT*>(p.out_a) + grow * (int64_t)p.f + h0 + c, av);
+              }
+            }
+          } else {  // EPI_SWIGLU_BWD: accumulator = dA; H1/H3 prefetched in in_buf
+            float h1[32], h3[32], d3[32];
+#pragma unroll 1
+            for (int i = 0; i < C::WCH; ++i) {
+              const int c = (cfirst + i) * 32;
+              const int slot = in_used % INS;
+              const uint32_t par = (in_used / INS) & 1u;
+              tmem_ld32(tb + c, v);
+              tmem_ld_wait();
+              reg_fence32(v);
+              bits_to_f32(v, fv);
+              if (!mbar_wait_warp(&my_in_full[slot], par, abort_flag, p.status)) break;
+              uint8_t* sl = in_buf + slot * C::IN_CH;
+              unstage_row<T>(sl, lane, h1);
+              unstage_row<T>(sl + C::IN_CH / 2, lane, h3);
+              ++in_used;
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                const float sg = sigmoid_f(h1[j]);
+                const float da = fv[j];
+                d3[j] = da * h1[j] * sg;
+                fv[j] = da * h3[j] * sg * (1.0f + h1[j] * (1.0f - sg));
+              }
+              if (whole) {
+                // each lane rewrites only the row it read, so no barrier is needed first
+                stage_row<OutT>(sl, lane, fv);
+                stage_row<OutT>(sl + C::IN_CH / 2, lane, d3);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                  tma_store_2d(&tmO, sl, tl.n0 + c, rbase);
+                  tma_store_2d(&tmO, sl + C::IN_CH / 2, p.f + tl.n0 + c, rbase);
+                  bulk_commit();
+                }
+              } else if (valid) {
+                OutT* dh = reinterpret_cast<OutT*>(p.out) + grow * (2 * (int64_t)p.f) + tl.n0 + c;
+                store32<OutT>(dh, fv);
+                store32<OutT>(dh + p.f, d3);
+              }
+              if (i + C::IN_SLOTS < C::WCH) {
+                // refill the slot with the chunk IN_SLOTS ahead once its stores read it out
+                __syncwarp();
+                if (lane == 0) {
+                  bulk_wait_read<0>();
+                  const int x = tl.n0 + (cfirst + i + C::IN_SLOTS) * 32;
+                  mbar_arrive_expect_tx(&my_in_full[slot], C::IN_CH);
+                  tma_load_2d(sl, &tmI, &my_in_full[slot], x, rbase);
+                  tma_load_2d(sl + C::IN_CH / 2, &tmI, &my_in_full[slot], p.f + x, rbase);
+                }
+                ++in_issued;
+              }
             }
           }
         }
       } else {
-        // RAGGED_K: dW_e[m0 + r, n0 .. n0 + BN)
-        const int64_t off = (int64_t)tl.e * p.M * p.N + (int64_t)(tl.m0 + r) * p.N + tl.n0;
+        // RAGGED_K: dW_e[m0 + 32q .. +32, n0 .. n0 + BN), a [E*M, N] tensor
         const bool has = tl.kb > 0;
+        const int y = tl.e * p.M + tl.m0 + myrow + q * 32;
+        if (has || !p.accumulate) {
 #pragma unroll 1
-        for (int c = 0; c < BN; c += 32) {
-          if (has) {
-            tmem_ld32(tb + c, v);
-            tmem_ld_wait();
-            reg_fence32(v);
-          } else {
+          for (int c = cfirst * 32; c < (cfirst + C::WCH) * 32; c += 32) {
+            if (has) {
+              tmem_ld32(tb + c, v);
+              tmem_ld_wait();
+              reg_fence32(v);
+              bits_to_f32(v, fv);
+            } else {
 #pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0u;
-          }
-          float fv[32];
-          bits_to_f32(v, fv);
-          if (p.out_fp32) {
-            float* o = reinterpret_cast<float*>(p.out) + off + c;
-            if (p.accumulate) {
-              float old[32];
-              load32<float>(o, old);
-#pragma unroll
-              for (int i = 0; i < 32; ++i) fv[i] += old[i];
+              for (int i = 0; i < 32; ++i) fv[i] = 0.f;
             }
-            store32<float>(o, fv);
-          } else {
-            store32<T>(reinterpret_cast<T*>(p.out) + off + c, fv);
+            staged_store<OutT, C::NBUF>(stage_buf + sbuf * C::CH, fv, lane, &tmO, tl.n0 + c, y,
+                                        p.accumulate != 0);
+            sbuf = sbuf + 1 == C::NBUF ? 0 : sbuf + 1;
           }
         }
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[acc]);
+      if (lane == 0) {
+        if (PAIR) mbar_arrive_remote(tempty_leader + static_cast<uint32_t>(acc) * 8u);
+        else mbar_arrive(&tempty[acc]);
+      }
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
     }
+    if (lane == 0) {
+      bulk_wait_all();
+      // input chunks still in flight (only after an abort) must land before exit
+      for (; in_used < in_issued; ++in_used)
+        mbar_wait_teardown(&my_in_full[in_used % INS], (in_used / INS) & 1u);
+    }
+    __syncwarp();
   }
 
-  __syncthreads();
+  // A pair's leader reads the follower's shared memory and writes its TMEM until its
+  // last MMA completes (the leader waited for that above): neither CTA leaves before.
+  tc_fence_before();
+  if (PAIR) cluster_sync();
+  else __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, C::TMEM_COLS);
+    if (PAIR) tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+    else tmem_dealloc(tmem_base, C::TMEM_COLS);
   }
+}
+
+// Per-expert views of G [R, M] for the ragged-K wgrad: maps[e] = tmpl with its row
+// extent cut at off_e+1, so TMA zero-fills every row past expert e's last one.  (A view
+// needs at least one row; an expert with no rows never loads through its map.)
+__global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
+                                   const __grid_constant__ CUtensorMap tmpl1,
+                                   const int32_t* __restrict__ offsets, int E,
+                                   CUtensorMap* maps) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= 2 * E) return;
+  const int e = i < E ? i : i - E;
+  const uint4* src = reinterpret_cast<const uint4*>(i < E ? &tmpl0 : &tmpl1);
+  uint4* dst = reinterpret_cast<uint4*>(maps + i);
+#pragma unroll
+  for (int j = 0; j < 8; ++j) dst[j] = src[j];
+  const int rows = offsets[e + 1];
+  tmap_replace_outer_dim(maps + i, static_cast<uint32_t>(rows > 0 ? rows : 1));
+  fence_tmap_release();
 }
 
 // =============================================================================== host side
@@ -488,11 +682,15 @@ static EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 2-D row-major tensor [rows, cols] with 128-byte swizzled boxes of [box_rows, box_cols].
-// `mn_major` boxes of 32-bit elements use the 32-byte-atom variant of the swizzle, the
-// layout the tensor core accepts for M/N-major TF32 operands.
+enum class Box { KMajor, MNMajor, Chunk };
+
+// 2-D row-major tensor [rows, cols] of bf16 or fp32 with box [box_rows, box_cols]:
+//   KMajor / MNMajor operand tiles: 128-byte rows, 128-byte swizzle (M/N-major fp32
+//   tiles: the 32-byte-atom variant, the layout the tensor core takes for M/N-major
+//   TF32 operands);
+//   Chunk: 32 x 32 epilogue chunks, 64-byte swizzle for 16-bit, 128-byte for 32-bit.
 static bool make_tmap(CUtensorMap* m, const void* base, bool fp32, uint64_t cols, uint64_t rows,
-                      uint32_t box_cols, uint32_t box_rows, bool mn_major = false) {
+                      uint32_t box_cols, uint32_t box_rows, Box kind) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const uint64_t es = fp32 ? 4 : 2;
@@ -500,58 +698,96 @@ static bool make_tmap(CUtensorMap* m, const void* base, bool fp32, uint64_t cols
   cuuint64_t strides[1] = {cols * es};
   cuuint32_t box[2] = {box_cols, box_rows};
   cuuint32_t estr[2] = {1, 1};
+  CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B;
+  if (kind == Box::MNMajor && fp32) swz = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
+  if (kind == Box::Chunk && !fp32) swz = CU_TENSOR_MAP_SWIZZLE_64B;
   CUresult r = enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    const_cast<void*>(base), dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   (fp32 && mn_major) ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B
-                                      : CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
-template <typename T, int BN, bool A_MN, bool B_MN, int MODE, int EPI>
-static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const Params& p,
+template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
+static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
+                         const CUtensorMap& to2, const CUtensorMap& ti, const Params& p,
                          int max_tiles, cudaStream_t s) {
-  using C = Cfg<T, BN>;
-  auto kern = grouped_gemm_kernel<T, BN, A_MN, B_MN, MODE, EPI>;
+  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
+  auto kern = grouped_gemm_kernel<T, OutT, BN, A_MN, B_MN, MODE, EPI, PAIR>;
   const size_t smem = C::smem_bytes(p.E);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ECUDA;
-  int grid = num_sms();
-  if (max_tiles < grid) grid = max_tiles;
-  if (grid < 1) return MOE_OK;
-  kern<<<grid, kThreads, smem, s>>>(ta, tb, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  int units = num_sms();
+  if (PAIR) {
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    // how many CTA pairs fit at once (one CTA per SM: the shared memory takes it all)
+    static int max_pairs[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MOE_ECUDA;
+    if (max_pairs[dev] == 0) {
+      cfg.gridDim = dim3(2, 1, 1);
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) n = num_sms() / 2;
+      max_pairs[dev] = n;
+    }
+    units = max_pairs[dev];
+  }
+  if (max_tiles < units) units = max_tiles;
+  if (units < 1) return MOE_OK;
+  cfg.gridDim = dim3(PAIR ? 2 * units : units, 1, 1);
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, ti, p) != cudaSuccess) return MOE_ECUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 static int pick_bn(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
 
-// Upper bound of the ragged-M tile count: sum_e ceil(cnt_e / BM) <= R / BM + E.
-static int ragged_m_tiles(const GemmShape& g, int n_tiles) {
-  const long long mt = (long long)g.R / BM + g.E;
+// Upper bound of the ragged-M tile count: sum_e ceil(cnt_e / TM) <= R / TM + E.
+static int ragged_m_tiles(const GemmShape& g, int n_tiles, int tm) {
+  const long long mt = (long long)g.R / tm + g.E;
   const long long t = mt * n_tiles;
   return t > (1 << 30) ? (1 << 30) : static_cast<int>(t);
 }
 
 // RAGGED_M GEMM, A K-major [R, K] act, B K-major weights [E*N_rows, K] (B_MN = false)
-// or M/N-major weights [E*K, N] (B_MN = true).
-template <typename T, bool B_MN, int EPI, int BN>
+// or M/N-major weights [E*K, N] (B_MN = true).  Output `out` [R, out_cols]; SwiGLU
+// forward also writes out_a [R, f]; SwiGLU backward reads aux [R, 2f].
+template <typename T, bool B_MN, int EPI, int BN, bool PAIR>
 static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B, int N,
-                        int b_rows_per_expert, int b_cols, void* out, int64_t ldo, void* out_a,
+                        int b_rows_per_expert, int b_cols, void* out, int out_cols, void* out_a,
                         const void* aux, const int32_t* offsets, int* status, cudaStream_t s) {
-  using C = Cfg<T, BN>;
+  using C = Cfg<T, T, BN, EPI, PAIR>;
   const bool fp32 = sizeof(T) == 4;
-  CUtensorMap ta, tb;
-  if (!make_tmap(&ta, A, fp32, K, g.R, C::KB, BM)) return MOE_ECUDA;
+  CUtensorMap ta, tb, to, to2, ti;
+  if (!make_tmap(&ta, A, fp32, K, g.R, C::KB, BM, Box::KMajor)) return MOE_ECUDA;
   if (!B_MN) {
-    const int box_rows = EPI == EPI_SWIGLU_FWD ? BN / 2 : BN;
-    if (!make_tmap(&tb, B, fp32, K, (uint64_t)g.E * b_rows_per_expert, C::KB, box_rows))
+    const int box_rows = EPI == EPI_SWIGLU_FWD ? BN / 2 : C::BNC;
+    if (!make_tmap(&tb, B, fp32, K, (uint64_t)g.E * b_rows_per_expert, C::KB, box_rows,
+                   Box::KMajor))
       return MOE_ECUDA;
   } else {
-    if (!make_tmap(&tb, B, fp32, b_cols, (uint64_t)g.E * b_rows_per_expert, C::MNB, C::KB, true))
+    if (!make_tmap(&tb, B, fp32, b_cols, (uint64_t)g.E * b_rows_per_expert, C::MNB, C::KB,
+                   Box::MNMajor))
       return MOE_ECUDA;
   }
+  if (!make_tmap(&to, out, fp32, out_cols, g.R, 32, 32, Box::Chunk)) return MOE_ECUDA;
+  to2 = to;
+  ti = to;
+  if (EPI == EPI_SWIGLU_FWD && !make_tmap(&to2, out_a, fp32, g.f, g.R, 32, 32, Box::Chunk))
+    return MOE_ECUDA;
+  if (EPI == EPI_SWIGLU_BWD && !make_tmap(&ti, aux, fp32, 2 * (uint64_t)g.f, g.R, 32, 32,
+                                          Box::Chunk))
+    return MOE_ECUDA;
   Params p{};
   p.offsets = offsets;
   p.E = g.E;
@@ -561,23 +797,25 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.b_rows_per_expert = b_rows_per_expert;
   p.f = g.f;
   p.out = out;
-  p.ldo = ldo;
+  p.ldo = out_cols;
   p.out_a = out_a;
-  p.aux = aux;
   p.status = status;
-  return launch<T, BN, false, B_MN, RAGGED_M, EPI>(ta, tb, p, ragged_m_tiles(g, N / BN), s);
+  return launch<T, T, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
+      ta, tb, to, to2, ti, p, ragged_m_tiles(g, N / BN, C::TM), s);
 }
 
 // RAGGED_K GEMM: dW_e[M, N] = G_e^T . X_e with G [R, M] and X [R, N] (both act, M/N-major).
-template <typename T, int BN>
+template <typename T, typename OutT, int BN, bool PAIR>
 static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X, int N, void* dW,
-                        bool dw_fp32, bool accum, const int32_t* offsets, int* status,
-                        cudaStream_t s) {
-  using C = Cfg<T, BN>;
+                        bool accum, const int32_t* offsets, const CUtensorMap* g_maps,
+                        int* status, cudaStream_t s) {
+  using C = Cfg<T, OutT, BN, EPI_STORE, PAIR, RAGGED_K>;
   const bool fp32 = sizeof(T) == 4;
-  CUtensorMap ta, tb;
-  if (!make_tmap(&ta, G, fp32, M, g.R, C::MNB, C::KB, true)) return MOE_ECUDA;
-  if (!make_tmap(&tb, X, fp32, N, g.R, C::MNB, C::KB, true)) return MOE_ECUDA;
+  CUtensorMap ta, tb, to;
+  if (!make_tmap(&ta, G, fp32, M, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&tb, X, fp32, N, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&to, dW, sizeof(OutT) == 4, N, (uint64_t)g.E * M, 32, 32, Box::Chunk))
+    return MOE_ECUDA;
   Params p{};
   p.offsets = offsets;
   p.E = g.E;
@@ -586,41 +824,45 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
   p.N = N;
   p.f = g.f;
   p.out = dW;
-  p.out_fp32 = dw_fp32 ? 1 : 0;
   p.accumulate = accum ? 1 : 0;
+  p.a_maps = g_maps;
   p.status = status;
-  const long long tiles = (long long)g.E * (M / BM) * (N / BN);
-  return launch<T, BN, true, true, RAGGED_K, EPI_STORE>(
-      ta, tb, p, tiles > (1 << 30) ? (1 << 30) : (int)tiles, s);
+  const long long tiles = (long long)g.E * (M / C::TM) * (N / BN);
+  return launch<T, OutT, BN, true, true, RAGGED_K, EPI_STORE, PAIR>(
+      ta, tb, to, to, to, p, tiles > (1 << 30) ? (1 << 30) : (int)tiles, s);
 }
 
-#define MOE_DISPATCH_BN(bn, CALL)           \
-  do {                                      \
+#define MOE_DISPATCH_BN(bn, CALL)                             \
+  do {                                                        \
     if ((bn) == 256) { constexpr int BN = 256; return CALL; } \
     if ((bn) == 128) { constexpr int BN = 128; return CALL; } \
     { constexpr int BN = 64; return CALL; }                   \
   } while (0)
 
+// CTA pairs for the 16-bit kernels; the TF32 kernels run one CTA per tile.
+template <typename T>
+constexpr bool kPair = sizeof(T) == 2;
+
 template <typename T>
 static moe_status fc1_fwd(const GemmShape& g, const void* x_perm, const void* W13,
                           const int32_t* off, void* H13, void* a, int* st, cudaStream_t s) {
   // accumulator grid: 2f columns, each tile = BN/2 gate columns + the matching BN/2 up columns
-  const int bn = g.f % 128 == 0 ? 256 : 128;
-  if (bn == 256)
-    return run_m<T, false, EPI_SWIGLU_FWD, 256>(g, x_perm, g.d, W13, 2 * g.f, 2 * g.f, g.d, H13,
-                                                 2 * (int64_t)g.f, a, nullptr, off, st, s);
-  return run_m<T, false, EPI_SWIGLU_FWD, 128>(g, x_perm, g.d, W13, 2 * g.f, 2 * g.f, g.d, H13,
-                                               2 * (int64_t)g.f, a, nullptr, off, st, s);
+  if (g.f % 128 == 0)
+    return run_m<T, false, EPI_SWIGLU_FWD, 256, kPair<T>>(g, x_perm, g.d, W13, 2 * g.f, 2 * g.f,
+                                                           g.d, H13, 2 * g.f, a, nullptr, off, st,
+                                                           s);
+  return run_m<T, false, EPI_SWIGLU_FWD, 128, kPair<T>>(g, x_perm, g.d, W13, 2 * g.f, 2 * g.f, g.d,
+                                                         H13, 2 * g.f, a, nullptr, off, st, s);
 }
 
 template <typename T>
 static moe_status fc2_fwd(const GemmShape& g, const void* a, const void* W2, const int32_t* off,
                           void* y_perm, int* st, cudaStream_t s) {
   if (g.d % 256 == 0)
-    return run_m<T, false, EPI_STORE, 256>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d, nullptr,
-                                            nullptr, off, st, s);
-  return run_m<T, false, EPI_STORE, 128>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d, nullptr,
-                                          nullptr, off, st, s);
+    return run_m<T, false, EPI_STORE, 256, kPair<T>>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d,
+                                                      nullptr, nullptr, off, st, s);
+  return run_m<T, false, EPI_STORE, 128, kPair<T>>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d,
+                                                    nullptr, nullptr, off, st, s);
 }
 
 template <typename T>
@@ -628,9 +870,16 @@ static moe_status fc2_dgrad(const GemmShape& g, const void* dy_perm, const void*
                             const void* H13, const int32_t* off, void* dH13, int* st,
                             cudaStream_t s) {
   // dA = dY . W2_e: K = d, N = f; B[n, k] = W2[e*d + k, n] (M/N-major)
-  MOE_DISPATCH_BN(pick_bn(g.f),
-                  (run_m<T, true, EPI_SWIGLU_BWD, BN>(g, dy_perm, g.d, W2, g.f, g.d, g.f, dH13,
-                                                      2 * (int64_t)g.f, nullptr, H13, off, st, s)));
+  if constexpr (kPair<T>) {
+    if (g.f % 256 == 0)
+      return run_m<T, true, EPI_SWIGLU_BWD, 256, true>(g, dy_perm, g.d, W2, g.f, g.d, g.f, dH13,
+                                                        2 * g.f, nullptr, H13, off, st, s);
+  }
+  if (g.f % 128 == 0)
+    return run_m<T, true, EPI_SWIGLU_BWD, 128, kPair<T>>(g, dy_perm, g.d, W2, g.f, g.d, g.f, dH13,
+                                                          2 * g.f, nullptr, H13, off, st, s);
+  return run_m<T, true, EPI_SWIGLU_BWD, 64, false>(g, dy_perm, g.d, W2, g.f, g.d, g.f, dH13,
+                                                    2 * g.f, nullptr, H13, off, st, s);
 }
 
 template <typename T>
@@ -638,16 +887,48 @@ static moe_status fc1_dgrad(const GemmShape& g, const void* dH13, const void* W1
                             const int32_t* off, void* dx_perm, int* st, cudaStream_t s) {
   // dX = dH13 . W13_e: K = 2f, N = d; B[n, k] = W13[e*2f + k, n] (M/N-major)
   if (g.d % 256 == 0)
-    return run_m<T, true, EPI_STORE, 256>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d, dx_perm, g.d,
-                                           nullptr, nullptr, off, st, s);
-  return run_m<T, true, EPI_STORE, 128>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d, dx_perm, g.d,
-                                         nullptr, nullptr, off, st, s);
+    return run_m<T, true, EPI_STORE, 256, kPair<T>>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
+                                                     dx_perm, g.d, nullptr, nullptr, off, st, s);
+  return run_m<T, true, EPI_STORE, 128, kPair<T>>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
+                                                   dx_perm, g.d, nullptr, nullptr, off, st, s);
+}
+
+template <typename T, typename OutT>
+static moe_status wgrad_t(const GemmShape& g, const void* G, int M, const void* X, int N, void* dW,
+                          bool accum, const int32_t* off, const CUtensorMap* maps, int* st,
+                          cudaStream_t s) {
+  // pairs need 256-row output tiles and B halves of whole 64-column blocks (BN >= 128)
+  const int bn = pick_bn(N);
+  if (kPair<T> && M % 256 == 0 && bn >= 128) {
+    if (bn == 256)
+      return run_k<T, OutT, 256, kPair<T>>(g, G, M, X, N, dW, accum, off, maps, st, s);
+    return run_k<T, OutT, 128, kPair<T>>(g, G, M, X, N, dW, accum, off, maps, st, s);
+  }
+  MOE_DISPATCH_BN(bn, (run_k<T, OutT, BN, false>(g, G, M, X, N, dW, accum, off, maps, st, s)));
 }
 
 template <typename T>
 static moe_status wgrad(const GemmShape& g, const void* G, int M, const void* X, int N, void* dW,
-                        bool dw_fp32, bool accum, const int32_t* off, int* st, cudaStream_t s) {
-  MOE_DISPATCH_BN(pick_bn(N), (run_k<T, BN>(g, G, M, X, N, dW, dw_fp32, accum, off, st, s)));
+                        bool dw_fp32, bool accum, const int32_t* off, const CUtensorMap* maps,
+                        int* st, cudaStream_t s) {
+  if (dw_fp32) return wgrad_t<T, float>(g, G, M, X, N, dW, accum, off, maps, st, s);
+  return wgrad_t<T, T>(g, G, M, X, N, dW, false, off, maps, st, s);
+}
+
+// Builds the per-expert maps of both wgrad G operands (dY for FC2, dH13 for FC1) into
+// `maps` [2E] before either wgrad runs.
+template <typename T>
+static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, const void* dH13,
+                                   const int32_t* off, CUtensorMap* maps, cudaStream_t s) {
+  using C = Cfg<T, T, 128, EPI_STORE>;
+  const bool fp32 = sizeof(T) == 4;
+  CUtensorMap t0, t1;
+  if (!make_tmap(&t0, dy_perm, fp32, g.d, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&t1, dH13, fp32, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
+    return MOE_ECUDA;
+  const int threads = 2 * g.E;
+  expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, maps);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 }  // namespace gemm
@@ -670,25 +951,30 @@ template <typename T>
 static moe_status gemm_bwd_t(const GemmShape& g, const void* dy_perm, const void* x_perm,
                              const void* H13, const void* a, const void* W13, const void* W2,
                              const int32_t* off, void* dH13, void* dx_perm, void* dW13, void* dW2,
-                             bool dw_fp32, bool dw_accum, int* st, cudaStream_t s) {
-  moe_status r = gemm::fc2_dgrad<T>(g, dy_perm, W2, H13, off, dH13, st, s);
+                             bool dw_fp32, bool dw_accum, void* maps_ws, int* st,
+                             cudaStream_t s) {
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_ws);
+  moe_status r = gemm::build_wgrad_maps<T>(g, dy_perm, dH13, off, maps, s);
   if (r != MOE_OK) return r;
-  r = gemm::wgrad<T>(g, dy_perm, g.d, a, g.f, dW2, dw_fp32, dw_accum, off, st, s);
+  r = gemm::fc2_dgrad<T>(g, dy_perm, W2, H13, off, dH13, st, s);
+  if (r != MOE_OK) return r;
+  r = gemm::wgrad<T>(g, dy_perm, g.d, a, g.f, dW2, dw_fp32, dw_accum, off, maps, st, s);
   if (r != MOE_OK) return r;
   r = gemm::fc1_dgrad<T>(g, dH13, W13, off, dx_perm, st, s);
   if (r != MOE_OK) return r;
-  return gemm::wgrad<T>(g, dH13, 2 * g.f, x_perm, g.d, dW13, dw_fp32, dw_accum, off, st, s);
+  return gemm::wgrad<T>(g, dH13, 2 * g.f, x_perm, g.d, dW13, dw_fp32, dw_accum, off, maps + g.E,
+                        st, s);
 }
 
 moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm, const void* H13,
                     const void* a, const void* W13, const void* W2, const int32_t* offsets,
                     void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
-                    bool dw_accum, int* status, cudaStream_t s) {
+                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s) {
   if (g.fp32)
     return gemm_bwd_t<float>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13,
-                             dW2, dw_fp32, dw_accum, status, s);
+                             dW2, dw_fp32, dw_accum, maps_ws, status, s);
   return gemm_bwd_t<__nv_bfloat16>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm,
-                                   dW13, dW2, dw_fp32, dw_accum, status, s);
+                                   dW13, dW2, dw_fp32, dw_accum, maps_ws, status, s);
 }
 
 }  // namespace moe

@@ -51,10 +51,12 @@ struct GemmShape {
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
                     const int32_t* offsets, void* H13, void* a, void* y_perm, int* status,
                     cudaStream_t s);
-// FC2 dgrad (+SwiGLU bwd), FC2 wgrad, FC1 dgrad, FC1 wgrad.
+// FC2 dgrad (+SwiGLU bwd), FC2 wgrad, FC1 dgrad, FC1 wgrad.  `maps_ws`: 2*E*128 bytes
+// of 128-byte-aligned device scratch for the per-expert tensor maps of the wgrads.
+constexpr size_t kTensorMapBytes = 128;
 moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm, const void* H13,
                     const void* a, const void* W13, const void* W2, const int32_t* offsets,
                     void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
-                    bool dw_accum, int* status, cudaStream_t s);
+                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s);
 
 }  // namespace moe

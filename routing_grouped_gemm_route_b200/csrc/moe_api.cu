@@ -33,7 +33,7 @@ inline int64_t R_of(const moe_desc& d) { return (int64_t)d.T * d.k; }
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 struct WsLayout {
-  size_t status, hist, cta_base, dy_perm, dH13, dx_perm, dx_router, total;
+  size_t status, hist, cta_base, maps, dy_perm, dH13, dx_perm, dx_router, total;
 };
 
 WsLayout ws_layout(const moe_desc& d) {
@@ -45,6 +45,7 @@ WsLayout ws_layout(const moe_desc& d) {
   w.status = o; o += kAlign;
   w.hist = o; o = up(o + ctas * d.E * 4);
   w.cta_base = o; o = up(o + ctas * d.E * 4);
+  w.maps = o; o = up(o + 2 * (size_t)d.E * kTensorMapBytes);
   w.dy_perm = o; o = up(o + R * d.d * es);
   w.dH13 = o; o = up(o + R * 2 * (size_t)d.d_ff * es);
   w.dx_perm = o; o = up(o + R * d.d * es);
@@ -169,7 +170,7 @@ moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_p
     return cu(cudaMemsetAsync(dW2, 0, (size_t)d.E * d.d * d.d_ff * es, s));
   }
   return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13, dW2,
-                  fp32_dw, acc, status_ptr(ws), s);
+                  fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s);
 }
 
 moe_status router_fwd_body(const moe_desc& d, const void* x, const void* Wr, float* logits,
