@@ -204,6 +204,27 @@ moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_p
                            void* dy_perm, float* d_logits, void* ws, size_t ws_bytes,
                            void* stream);
 
+/* S15, MXFP8 quantisation (bigchange.ai pt-BR, opening section: MXFP8 for selected
+ * operations; OCP MX v1.0 rule, since the pages give none).  x [rows, cols] bf16 (device)
+ * is split into row segments [seg_offsets[e], seg_offsets[e+1]) (e < num_segments; one per
+ * expert; seg_offsets[num_segments] = rows).  Per block of 32 elements -- along cols
+ * (colwise = 0) or along the rows of one segment starting at its first row (colwise = 1;
+ * a segment's last block may be partial) -- the shared exponent is
+ * s = floor(log2(amax)) - 8 clamped to [-127, 127] (-127 for an all-zero block) and each
+ * element becomes E4M3(x / 2^s), round to nearest even, saturated to +-448.
+ * Out: codes [rows, cols] uint8 (device, x's layout); scales: E8M0 bytes s + 127 in
+ * 512-byte chunks (moe_mx_scale_bytes), chunk (tile_pref[e] + p/128) * (cols/128) +
+ * col/128 with tile_pref the prefix over segments of ceil(rows_e/128) and p the row
+ * inside its segment; inside a chunk the byte of (index i, block b) is
+ * 16*(i%32) + 4*((i%128)/32) + b, with i = p and b = (col%128)/32 rowwise, i = col and
+ * b = (p%128)/32 colwise.  Scale bytes of chunk slots that no block reaches are left
+ * untouched.  cols must be a multiple of 128.  ws: at least 256 + 8*(num_segments+1)
+ * bytes of device scratch. */
+moe_status moe_mx_scale_bytes(int64_t rows, int32_t cols, int32_t num_segments, size_t* bytes);
+moe_status moe_mx_quantize(const void* x, int64_t rows, int32_t cols, const int32_t* seg_offsets,
+                           int32_t num_segments, int32_t colwise, uint8_t* codes, uint8_t* scales,
+                           void* ws, size_t ws_bytes, void* stream);
+
 /* S10-S13, grouped GEMM backward of the SwiGLU experts, per expert e:
  *   dA_e   = dY_e . W2_e                                   (dY_e = rows of dy_perm)
  *   dH1_e  = dA_e * H3_e * s * (1 + H1_e * (1 - s)),  s = sigmoid(H1_e)

@@ -42,6 +42,13 @@ cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void
                                const int32_t* slot, void* dy_perm, float* d_logits, int* status,
                                cudaStream_t s);
 
+// ----------------------------------------------------------------------------- MXFP8
+size_t mx_sf_bytes(int64_t R, int C, int E);
+// `scratch`: 2*(E+1) int32 of device memory (segment prefixes).
+cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
+                               bool colwise, uint8_t* codes, uint8_t* sf, int32_t* scratch,
+                               cudaStream_t s);
+
 // ----------------------------------------------------------------------------- grouped GEMM
 struct GemmShape {
   int E, R, d, f;

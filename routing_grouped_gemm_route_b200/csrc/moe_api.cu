@@ -324,6 +324,29 @@ moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_p
                                topk_idx, slot, dy_perm, d_logits, status_ptr(ws), S(stream)));
 }
 
+moe_status moe_mx_scale_bytes(int64_t rows, int32_t cols, int32_t num_segments, size_t* bytes) {
+  if (!bytes || rows < 0 || cols <= 0 || cols % 128 != 0 || num_segments < 1 ||
+      num_segments > 1024)
+    return MOE_EINVAL;
+  *bytes = mx_sf_bytes(rows, cols, num_segments);
+  return MOE_OK;
+}
+
+moe_status moe_mx_quantize(const void* x, int64_t rows, int32_t cols, const int32_t* seg_offsets,
+                           int32_t num_segments, int32_t colwise, uint8_t* codes, uint8_t* scales,
+                           void* ws, size_t ws_bytes, void* stream) {
+  if (rows < 0 || rows >= (int64_t(1) << 31) || cols <= 0 || cols % 128 != 0 ||
+      num_segments < 1 || num_segments > 1024 || (colwise != 0 && colwise != 1))
+    return MOE_EINVAL;
+  if (rows * (int64_t)cols >= (int64_t(1) << 40)) return MOE_EINVAL;
+  MOE_TRY(ptrs({seg_offsets, ws}));
+  if (rows > 0) MOE_TRY(ptrs({x, codes, scales}));
+  if (ws_bytes < 256 + 8 * (size_t)(num_segments + 1)) return MOE_EWORKSPACE;
+  int32_t* scratch = at<int32_t>(ws, 256);
+  return cu(launch_mx_quantize(x, rows, cols, seg_offsets, num_segments, colwise != 0, codes,
+                               scales, scratch, S(stream)));
+}
+
 moe_status moe_grouped_gemm_bwd(const moe_desc* desc, const void* dy_perm, const void* x_perm,
                                 const void* H13, const void* a, const void* W13, const void* W2,
                                 const int32_t* offsets, void* dH13, void* dx_perm, void* dW13,

@@ -28,7 +28,7 @@ DTYPES = {"fp32": MOE_FP32, "bf16": MOE_BF16, "mxfp8": MOE_MXFP8}
 # Every entry point that include/moe.h declares.
 EXPORTS = ["moe_status_string", "moe_check_desc", "moe_workspace_size", "moe_saved_layout_get",
            "moe_workspace_init", "moe_read_device_status", "moe_router_logits", "moe_route",
-           "moe_route_noalloc",
+           "moe_route_noalloc", "moe_mx_scale_bytes", "moe_mx_quantize",
            "moe_dispatch", "moe_grouped_gemm_fwd", "moe_combine", "moe_combine_bwd",
            "moe_grouped_gemm_bwd", "moe_dispatch_bwd", "moe_router_bwd", "moe_layer_fwd",
            "moe_layer_bwd"]
@@ -78,6 +78,8 @@ def load():
         "moe_router_logits": [_P, _P, _P, _P, _P],
         "moe_route": [_P] + [_P] * 8 + [_P, _S, _P],
         "moe_route_noalloc": [_P] + [_P] * 8 + [_P],
+        "moe_mx_scale_bytes": [ctypes.c_int64, _I, _I, ctypes.POINTER(_S)],
+        "moe_mx_quantize": [_P, ctypes.c_int64, _I, _P, _I, _I, _P, _P, _P, _S, _P],
         "moe_dispatch": [_P, _P, _P, _P, _P, _P, _S, _P],
         "moe_grouped_gemm_fwd": [_P] + [_P] * 8 + [_P, _S, _P],
         "moe_combine": [_P, _P, _P, _P, _P, _P, _S, _P],
@@ -195,6 +197,22 @@ def moe_route_noalloc(desc, logits, topk_idx, gates, counts, offsets, slot, row_
                                     _ptr(gates), _ptr(counts), _ptr(offsets), _ptr(slot),
                                     _ptr(row_token), _ptr(row_gate), _stream(stream)),
            "moe_route_noalloc")
+
+
+def moe_mx_scale_bytes(rows, cols, num_segments) -> int:
+    n = _S(0)
+    _check(load().moe_mx_scale_bytes(rows, cols, num_segments, ctypes.byref(n)),
+           "moe_mx_scale_bytes")
+    return n.value
+
+
+def moe_mx_quantize(x, seg_offsets, colwise, codes, scales, ws, stream=None):
+    """MXFP8 quantisation of bf16 x [rows, cols] in row segments (see include/moe.h)."""
+    rows, cols = x.shape
+    _check(load().moe_mx_quantize(_ptr(x), rows, cols, _ptr(seg_offsets),
+                                  seg_offsets.numel() - 1, 1 if colwise else 0, _ptr(codes),
+                                  _ptr(scales), _ptr(ws), _nbytes(ws), _stream(stream)),
+           "moe_mx_quantize")
 
 
 def moe_dispatch(desc, x, slot, x_perm, ws, x_perm_sf=None, stream=None):
