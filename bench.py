@@ -175,8 +175,9 @@ def oracle_sample_run(w, inp_cpu: dict, T_s: int):
     Wr = None if inp_cpu["Wr"] is None else inp_cpu["Wr"].double().numpy()
     L = None if inp_cpu["logits"] is None else inp_cpu["logits"][:T_s].double().numpy()
     t0 = time.perf_counter()
-    fwd = oracle.layer_fwd(x, W13, W2, logits=L, Wr=Wr if L is None else None, k=w.k)
-    oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr)
+    fwd = oracle.layer_fwd(x, W13, W2, logits=L, Wr=Wr if L is None else None, k=w.k,
+                           mx=w.dtype == "mxfp8")
+    oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr, mx=w.dtype == "mxfp8")
     return time.perf_counter() - t0
 
 
@@ -202,16 +203,19 @@ def host_inputs(w, dev_inp: dict) -> dict:
 def cpu_baseline(w, inp_cpu, target_s: float) -> dict:
     """Oracle tokens/s on a bounded token sample: grown (at most 4 calls, each at most 4x
     the last) until one call takes about target_s seconds."""
-    T_s = min(64, w.T)
+    # MXFP8: the oracle quantises the weights of every expert a sample touches (several
+    # seconds per expert at d=4096), so the sample is one token (its k experts) and stays so
+    mx = w.dtype == "mxfp8"
+    T_s = min(1 if mx else 64, w.T)
     t = oracle_sample_run(w, inp_cpu, T_s)
-    for _ in range(3):
+    for _ in range(0 if mx else 3):
         if t >= 0.6 * target_s or T_s >= w.T:
             break
         T_s = int(min(w.T, max(T_s + 1, T_s * min(4.0, target_s / max(t, 1e-3)))))
         t = oracle_sample_run(w, inp_cpu, T_s)
     return {"value": T_s / t, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"fp64 NumPy oracle fwd+bwd on the first {T_s} of {w.T} tokens of the same "
-                      f"workload (all {w.E} experts' weights), one call, {t:.1f} s"}
+                      f"workload (the experts those tokens select), one call, {t:.1f} s"}
 
 
 # ------------------------------------------------------------------------------ reference arm
@@ -222,14 +226,14 @@ def run_reference(args, w, world, rank):
     inp = make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     inp_cpu = host_inputs(w, inp)
     del inp
-    T_s = min(128, w.T)
+    T_s = min(1 if w.dtype == "mxfp8" else 128, w.T)
     for _ in range(args.warmup):
         oracle_sample_run(w, inp_cpu, T_s)
     times = [oracle_sample_run(w, inp_cpu, T_s) for _ in range(args.steps)]
     tot = sum(times)
     value = T_s * args.steps / tot
     sample = (f"fp64 NumPy oracle fwd+bwd on the first {T_s} of {w.T} tokens of the workload per "
-              f"step (all {w.E} experts' weights)")
+              f"step (the experts those tokens select)")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * tot / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -349,8 +353,12 @@ def main():
               "dispatch_bwd"]
     if w.router:
         stages = ["router"] + stages + ["router_bwd"]
-    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 2, "combine": 1,
-                "combine_bwd": 1, "gemm_bwd": 4, "dispatch_bwd": 1, "router_bwd": 3}
+    mx = w.dtype == "mxfp8"
+    # GEMM stages: bf16/fp32 fwd = 2 GEMMs, bwd = tensor-map builder + 4 GEMMs; MXFP8 adds
+    # the quantisers (segment prefix + quantise per operand) and two offset fills per stage
+    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 12 if mx else 2,
+                "combine": 1, "combine_bwd": 1, "gemm_bwd": 23 if mx else 5, "dispatch_bwd": 1,
+                "router_bwd": 3}
 
     def run_stage(name):
         if name == "router":
@@ -432,8 +440,13 @@ def main():
     gemm_ms = stage_ms["gemm_fwd"] + stage_ms["gemm_bwd"]
     gemm_tflops = (gemm_flops["gemm_fwd"] + gemm_flops["gemm_bwd"]) / (gemm_ms * 1e-3) / 1e12
     peak_tf = pk["bf16_sustained"]
+    peak_kind = "sustained dense bf16"
     if act == torch.float32:
         peak_tf = pk["bf16_sustained"] * 1.1 / 2.25     # TF32 = bf16 x nominal ratio
+        peak_kind = "sustained dense bf16 x 1.1/2.25 (nominal tf32/bf16)"
+    elif mx:
+        peak_tf = pk["bf16_sustained"] * 4.5 / 2.25     # FP8 = bf16 x nominal ratio
+        peak_kind = "sustained dense bf16 x 4.5/2.25 (nominal fp8/bf16)"
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
     if os.path.exists(tfile):
@@ -449,8 +462,10 @@ def main():
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / peak_tf, 4), "traffic": traffic,
                 "kernel": "grouped GEMM, 6 launches per step (FC1+SwiGLU, FC2, FC2 dgrad+SwiGLU "
                           "bwd, FC2 wgrad, FC1 dgrad, FC1 wgrad), algorithmic 18*T*k*d*d_ff flops",
-                "peak_source": f"{pk['source']} sustained dense bf16 (MEASURED_PEAKS.json)"
-                if pk["source"] == "measured" else "fallback 1.4 PFLOP/s sustained"}
+                "peak_source": f"{pk['source']} {peak_kind} (MEASURED_PEAKS.json)"
+                if pk["source"] == "measured" else f"fallback 1.4 PFLOP/s, {peak_kind}"}
+    if mx:
+        roofline["kernel"] += "; the GEMM stages include the MXFP8 quantisers of their operands"
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -467,7 +482,7 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16" if act == torch.bfloat16 else "f32",
+            "vs_baseline": None, "dtype": ("mxfp8-e4m3" if mx else "bf16") if act == torch.bfloat16 else "f32",
             "data": "synthetic (seeded N(0,1) activations/logits, N(0,0.02) weights)",
             "config": {"workload": workload_desc(w), "T": T, "d_model": d, "E": E, "top_k": k,
                        "d_ff": f, "router_on_device": w.router,

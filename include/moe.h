@@ -61,7 +61,9 @@ typedef enum moe_status {
 typedef enum moe_dtype {
   MOE_FP32 = 0,   /* fp32 storage, TF32 tensor-core GEMMs with fp32 accumulation */
   MOE_BF16 = 1,   /* bf16 storage, bf16 tensor-core GEMMs with fp32 accumulation */
-  MOE_MXFP8 = 2   /* bf16 storage, GEMM operands E4M3 with an E8M0 scale per 32 */
+  MOE_MXFP8 = 2   /* bf16 storage; the grouped GEMMs quantise their operands to E4M3 with
+                     an E8M0 scale per 32 along K (moe_mx_quantize) and run block-scaled
+                     tensor-core MMAs with fp32 accumulation; d_ff a multiple of 128 */
 } moe_dtype;
 
 /* moe_desc.flags */
@@ -168,9 +170,9 @@ moe_status moe_route_noalloc(const moe_desc* desc, const float* logits, int32_t*
                              int32_t* row_token, float* row_gate, void* stream);
 
 /* S5, row-wise dispatch: x_perm[slot[t,j]] = x[t] for every (t,j)
- * (unite.ai, "पैरालेलिज़्म, प्रिसीजन, और मेमोरी तकनीकें").  x [T,d] act, x_perm [R,d] act.
- * x_perm_sf is reserved for the MXFP8 layout and must be NULL.  A slot outside
- * [0,R) sets MOE_DEV_BAD_INDEX and that copy is skipped. */
+ * (unite.ai, "पैरालेलिज़्म, प्रिसीजन, और मेमोरी तकनीकें").  x [T,d] act, x_perm [R,d] act
+ * (bf16 also for MOE_MXFP8: the grouped GEMM quantises it).  x_perm_sf is reserved and
+ * must be NULL.  A slot outside [0,R) sets MOE_DEV_BAD_INDEX and that copy is skipped. */
 moe_status moe_dispatch(const moe_desc* desc, const void* x, const int32_t* slot,
                         void* x_perm, void* x_perm_sf, void* ws, size_t ws_bytes,
                         void* stream);
@@ -217,7 +219,9 @@ moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_p
  * col/128 with tile_pref the prefix over segments of ceil(rows_e/128) and p the row
  * inside its segment; inside a chunk the byte of (index i, block b) is
  * 16*(i%32) + 4*((i%128)/32) + b, with i = p and b = (col%128)/32 rowwise, i = col and
- * b = (p%128)/32 colwise.  Scale bytes of chunk slots that no block reaches are left
+ * b = (p%128)/32 colwise.  Colwise, the slots of a segment's last chunk past its last
+ * block are written as 0 (scale 2^-127), so a reader of whole chunks sees finite scales;
+ * other slots that no block reaches (rowwise rows past a segment's end) are left
  * untouched.  cols must be a multiple of 128.  ws: at least 256 + 8*(num_segments+1)
  * bytes of device scratch. */
 moe_status moe_mx_scale_bytes(int64_t rows, int32_t cols, int32_t num_segments, size_t* bytes);

@@ -35,7 +35,7 @@ from __future__ import annotations
 
 import numpy as np
 
-from .mx import mx_quantize_dequantize
+from .mx import bf16_round, mx_quantize_dequantize
 
 
 def _f64(a) -> np.ndarray:
@@ -178,7 +178,9 @@ def dispatch_bwd(dx_perm, slot) -> np.ndarray:
 # --------------------------------------------------------------------------- expert FFN
 
 def _mx(a, axis, mx: bool):
-    return mx_quantize_dequantize(a, axis=axis) if mx else a
+    """An MXFP8 GEMM operand: the operand as the BF16 tensor the GEMM reads (BF16 I/O),
+    quantised with blocks of 32 along ``axis``.  Without ``mx``, ``a`` unchanged."""
+    return mx_quantize_dequantize(bf16_round(a), axis=axis) if mx else a
 
 
 def experts_fwd(x_perm, offsets, W13, W2, mx: bool = False):
@@ -186,7 +188,8 @@ def experts_fwd(x_perm, offsets, W13, W2, mx: bool = False):
 
     H_e = X_e W13_e^T, a_e = silu(H_e[:, :f]) * H_e[:, f:], Y_e = a_e W2_e^T.
     With ``mx`` the GEMM operands are MX-quantised (E4M3 + E8M0 per 32 along the
-    GEMM's K) at the points the MXFP8 path quantises them; the rest stays fp64.
+    GEMM's K) at the points the MXFP8 path quantises them, each taken as the BF16
+    tensor the GEMM reads; the rest stays fp64.
     Returns (H13 [R,2f], a [R,f], y_perm [R,d]).
     """
     X = _f64(x_perm)

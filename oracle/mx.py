@@ -17,6 +17,11 @@ definition for MXFP8 with E4M3 elements:
 E4M3 ("FN" variant): 1 sign bit, 4 exponent bits with bias 7, 3 mantissa bits;
 normals 2**(E-7) * (1 + m/8) for E in 1..15 (E=15, m=7 is NaN, so the largest
 normal is 448); subnormals 2**-6 * m/8.
+
+The MXFP8 workload keeps BF16 inputs and outputs around its block-scaled GEMMs ("fp32
+accumulate, BF16 I/O"), so the tensor a quantiser sees is a BF16 tensor: ``bf16_round``
+gives that rounding (IEEE round to nearest even, 8 significant bits) for the layer
+oracle to apply before quantising an operand.
 """
 from __future__ import annotations
 
@@ -26,6 +31,22 @@ BLOCK = 32
 E4M3_MAX = 448.0
 E4M3_EMAX = 8
 E4M3_EMIN = -6
+
+
+def bf16_round(v) -> np.ndarray:
+    """fp64 values rounded once to the nearest bfloat16 value (ties to even).
+
+    bfloat16 has 8 significant bits and the exponent range of fp32: the spacing of
+    values in the binade [2**(e-1), 2**e) is 2**(e-8), down to 2**-133 for the
+    subnormals below 2**-126.  Magnitudes that round above the largest finite value
+    (2**128 - 2**120) become infinite.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    _, ex = np.frexp(v)
+    spacing = np.ldexp(1.0, np.maximum(ex, -125) - 8)
+    r = np.rint(v / spacing) * spacing          # np.rint rounds halves to even
+    big = np.abs(r) > np.ldexp(255.0, 120)
+    return np.where(big, np.copysign(np.inf, v), r)
 
 
 def _floor_log2(a: np.ndarray) -> np.ndarray:

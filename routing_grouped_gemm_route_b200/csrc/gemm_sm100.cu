@@ -31,8 +31,10 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "internal.h"
@@ -42,6 +44,7 @@ namespace moe {
 namespace gemm {
 
 using bf16 = __nv_bfloat16;
+using fp8 = __nv_fp8_e4m3;     // MXFP8 operand codes (with E8M0 scales per 32 along K)
 using namespace moe::sm100;
 
 enum { RAGGED_M = 0, RAGGED_K = 1 };
@@ -63,8 +66,25 @@ struct Params {
   void* out_a;             // SwiGLU forward: a [R, f]
   int accumulate;          // RAGGED_K: dW += result (float dW only)
   const CUtensorMap* a_maps;  // RAGGED_K: per-expert maps of G (row extent = off_e+1)
+  // MXFP8: where each operand's 512-byte scale chunks are (see csrc/mx.cu for the
+  // layout).  Chunk of (expert e, M/N index mn, K-stage kb):
+  //   k_major: (seg(e) + mn/128) * W + kb     otherwise: (seg(e) + kb) * W + mn/128
+  // with seg(e) = e * seg_uniform, or tile_pref[e] when seg_uniform is 0.
+  struct Sf {
+    const uint8_t* base;
+    int seg_uniform;
+    int k_major;
+    int W;
+  } sfa, sfb;
+  const int32_t* tile_pref;  // [E+1] prefix of ceil(count_e / 128)
   int* status;
 };
+
+__device__ __forceinline__ int64_t sf_chunk(const Params::Sf& f, const int32_t* tile_pref, int e,
+                                            int mn, int kb) {
+  const int64_t seg = f.seg_uniform > 0 ? (int64_t)e * f.seg_uniform : (int64_t)tile_pref[e];
+  return f.k_major ? (seg + mn / 128) * f.W + kb : (seg + kb) * f.W + mn / 128;
+}
 
 // PAIR: a cluster of two CTAs on two SMs computes 256-row tiles with cta_group::2 MMAs;
 // each CTA loads its 128 rows of A and half of the BN rows of B, so each SM moves a
@@ -80,7 +100,12 @@ struct Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BNC * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  static constexpr int TMEM_COLS = 2 * BN;
+  // MXFP8: one 512-byte scale chunk for A's 128 rows and one per 128 rows of B, per stage
+  static constexpr bool MX = ES == 1;
+  static constexpr int SF_CHUNKS_B = MX ? BNC / 128 : 0;
+  static constexpr int SF_STAGE = MX ? 512 * (1 + SF_CHUNKS_B) : 0;
+  static constexpr int SFC = MX ? 4 * (1 + SF_CHUNKS_B) : 0;      // TMEM columns per stage
+  static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
   // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there);
   // elsewhere 4 warps keep up and leave more shared memory to the operand ring
   static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD ? 8 : 4;
@@ -91,19 +116,25 @@ struct Cfg {
   // epilogue shared memory per warp: output staging chunks of 32 rows x 32 columns
   static constexpr int CH = 32 * 32 * sizeof(OutT);
   static constexpr int NBUF = EPI == EPI_SWIGLU_FWD ? 3 : EPI == EPI_SWIGLU_BWD ? 0 : 2;
-  // SwiGLU backward: slots of prefetched H1/H3 input chunks (32 x 32 each); the dH1/dH3
-  // results are staged in place in the slot they were computed from
-  static constexpr int IN_SLOTS = EPI == EPI_SWIGLU_BWD ? (ES == 2 ? (WCH < 2 ? WCH : 2) : 1) : 0;
-  static constexpr int IN_CH = 2 * 32 * 32 * ES;
+  // SwiGLU backward: slots of prefetched H1/H3 input chunks (32 x 32 each, in the
+  // activation type: bf16 for the 16-bit and MXFP8 kernels); the dH1/dH3 results are
+  // staged in place in the slot they were computed from
+  static constexpr int AES = ES == 4 ? 4 : 2;
+  static constexpr int IN_SLOTS = EPI == EPI_SWIGLU_BWD ? (AES == 2 ? (WCH < 2 ? WCH : 2) : 1) : 0;
+  static constexpr int IN_CH = 2 * 32 * 32 * AES;
   static constexpr int EPI_WARP = ((NBUF * CH + IN_SLOTS * IN_CH) + 1023) / 1024 * 1024;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP;
   static constexpr int BAR_BYTES = 512;
   static constexpr int BUDGET =
       227 * 1024 - 1024 /*alignment*/ - BAR_BYTES - (2 * (kMaxE + 1) + 8) * 4 - EPI_BYTES;
-  static constexpr int STAGES = BUDGET / STAGE > 8 ? 8 : BUDGET / STAGE;
+  static constexpr int STAGES =
+      BUDGET / (STAGE + SF_STAGE) > 8 ? 8 : BUDGET / (STAGE + SF_STAGE);
   static_assert(STAGES >= 2, "shared memory budget");
+  static_assert(!MX || 2 * BN + STAGES * SFC <= 512, "tensor memory budget");
+  static constexpr int SF_COL0 = 2 * BN;                          // first scale column
   static constexpr size_t smem_bytes(int E) {
-    return 1024 + size_t(STAGES) * STAGE + EPI_BYTES + BAR_BYTES + size_t(2 * (E + 1) + 8) * 4;
+    return 1024 + size_t(STAGES) * (STAGE + SF_STAGE) + EPI_BYTES + BAR_BYTES +
+           size_t(2 * (E + 1) + 8) * 4;
   }
 };
 
@@ -224,8 +255,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                     const __grid_constant__ CUtensorMap tmI, const Params p) {
   using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
+  using ActT = typename std::conditional<sizeof(T) == 4, float, bf16>::type;  // epilogue inputs
   constexpr bool kTF32 = sizeof(T) == 4;
-  constexpr uint32_t IDESC = idesc_f32acc(C::TM, BN, kTF32 ? 2u : 1u, A_MN, B_MN);
+  constexpr bool kMX = C::MX;
+  constexpr uint32_t IDESC = kMX ? idesc_mxf8(C::TM, BN, A_MN, B_MN)
+                                 : idesc_f32acc(C::TM, BN, kTF32 ? 2u : 1u, A_MN, B_MN);
+  static_assert(!(kMX && PAIR), "MXFP8 tiles run one CTA per tile");
   static_assert(!PAIR || !kTF32, "CTA pairs run the 16-bit kernels");
   static_assert(!B_MN || C::BNC % C::MNB == 0, "an M/N-major B half is whole 128-byte blocks");
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
@@ -235,7 +270,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   uint8_t* tiles = smem;
-  uint8_t* epi_smem = tiles + C::STAGES * C::STAGE;
+  uint8_t* sf_smem = tiles + C::STAGES * C::STAGE;                 // MXFP8 scale chunks
+  uint8_t* epi_smem = sf_smem + C::STAGES * C::SF_STAGE;
   uint64_t* full = reinterpret_cast<uint64_t*>(epi_smem + C::EPI_BYTES);
   uint64_t* empty = full + C::STAGES;
   uint64_t* tfull = empty + C::STAGES;
@@ -341,7 +377,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           uint8_t* sA = tiles + stage * C::STAGE;
           uint8_t* sB = sA + C::A_BYTES;
           if (leader) {
-            mbar_arrive_expect_tx(&full[stage], C::STAGE * (PAIR ? 2 : 1));
+            mbar_arrive_expect_tx(&full[stage], (C::STAGE + C::SF_STAGE) * (PAIR ? 2 : 1));
             armed |= 1u << stage;
             armed_par = (armed_par & ~(1u << stage)) | (phase << stage);
           }
@@ -351,6 +387,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             else tma_load_2d(dst, tm, &full[stage], x, y);
           };
           const int k0 = kb * C::KB;
+          if constexpr (kMX) {
+            // this stage's scale chunks: A's 128 rows, then B's rows 128 at a time
+            uint8_t* sfs = sf_smem + stage * C::SF_STAGE;
+            const int a_mn = MODE == RAGGED_M ? tl.m0 + arow : tl.m0 + arow;
+            bulk_load(sfs, p.sfa.base + 512 * sf_chunk(p.sfa, p.tile_pref, tl.e, a_mn, kb), 512,
+                      &full[stage]);
+#pragma unroll
+            for (int j = 0; j < C::SF_CHUNKS_B; ++j)
+              bulk_load(sfs + 512 * (1 + j),
+                        p.sfb.base + 512 * sf_chunk(p.sfb, p.tile_pref, tl.e, tl.n0 + bcol + 128 * j, kb),
+                        512, &full[stage]);
+          }
           if (MODE == RAGGED_M) {
             load(sA, &tmA, k0, tl.row0 + arow);
             const int brow = tl.e * p.b_rows_per_expert;
@@ -419,12 +467,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { stop = true; break; }
           tc_fence_after();
           const uint32_t so = static_cast<uint32_t>(stage * C::STAGE) >> 4;
+          uint32_t sfa_t = 0, sfb_t = 0;
+          if constexpr (kMX) {
+            // scales of this stage into its TMEM slot (4 columns per 512-byte chunk); the
+            // MMAs below run after these copies (same issuing thread)
+            const uint32_t col = static_cast<uint32_t>(C::SF_COL0 + stage * C::SFC);
+            const uint32_t src = smem_u32(sf_smem + stage * C::SF_STAGE);
+            sfa_t = tmem_base + col;
+            sfb_t = tmem_base + col + 4;
+#pragma unroll
+            for (int j = 0; j <= C::SF_CHUNKS_B; ++j)
+              tmem_cp_scales(tmem_base + col + 4 * j, sdesc(src + 512 * j, 128, 128, 0));
+          }
 #pragma unroll
           for (int kk = 0; kk < C::KB / C::UK; ++kk) {
             const uint64_t ad = a_desc0 + so + kk * A_STEP;
             const uint64_t bd = b_desc0 + so + kk * B_STEP;
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if (PAIR) umma_pair(d_tmem, ad, bd, IDESC, accum);
+            if constexpr (kMX)
+              umma_mx(d_tmem, ad, bd, IDESC | idesc_sf_ids(kk, kk), sfa_t, sfb_t, accum);
+            else if (PAIR) umma_pair(d_tmem, ad, bd, IDESC, accum);
             else umma<kTF32>(d_tmem, ad, bd, IDESC, accum);
           }
           if (PAIR) umma_commit_pair(&empty[stage], 3);   // frees the stage in both CTAs
@@ -550,8 +612,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               bits_to_f32(v, fv);
               if (!mbar_wait_warp(&my_in_full[slot], par, abort_flag, p.status)) break;
               uint8_t* sl = in_buf + slot * C::IN_CH;
-              unstage_row<T>(sl, lane, h1);
-              unstage_row<T>(sl + C::IN_CH / 2, lane, h3);
+              unstage_row<ActT>(sl, lane, h1);
+              unstage_row<ActT>(sl + C::IN_CH / 2, lane, h3);
               ++in_used;
 #pragma unroll
               for (int j = 0; j < 32; ++j) {
@@ -689,11 +751,12 @@ enum class Box { KMajor, MNMajor, Chunk };
 //   tiles: the 32-byte-atom variant, the layout the tensor core takes for M/N-major
 //   TF32 operands);
 //   Chunk: 32 x 32 epilogue chunks, 64-byte swizzle for 16-bit, 128-byte for 32-bit.
-static bool make_tmap(CUtensorMap* m, const void* base, bool fp32, uint64_t cols, uint64_t rows,
+static bool make_tmap(CUtensorMap* m, const void* base, int es_, uint64_t cols, uint64_t rows,
                       uint32_t box_cols, uint32_t box_rows, Box kind) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const uint64_t es = fp32 ? 4 : 2;
+  const uint64_t es = static_cast<uint64_t>(es_);
+  const bool fp32 = es == 4;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {cols * es};
   cuuint32_t box[2] = {box_cols, box_rows};
@@ -701,7 +764,10 @@ static bool make_tmap(CUtensorMap* m, const void* base, bool fp32, uint64_t cols
   CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B;
   if (kind == Box::MNMajor && fp32) swz = CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B;
   if (kind == Box::Chunk && !fp32) swz = CU_TENSOR_MAP_SWIZZLE_64B;
-  CUresult r = enc(m, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+  const CUtensorMapDataType dt = es == 4   ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : es == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                           : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  CUresult r = enc(m, dt, 2,
                    const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -762,30 +828,37 @@ static int ragged_m_tiles(const GemmShape& g, int n_tiles, int tm) {
 // RAGGED_M GEMM, A K-major [R, K] act, B K-major weights [E*N_rows, K] (B_MN = false)
 // or M/N-major weights [E*K, N] (B_MN = true).  Output `out` [R, out_cols]; SwiGLU
 // forward also writes out_a [R, f]; SwiGLU backward reads aux [R, 2f].
-template <typename T, bool B_MN, int EPI, int BN, bool PAIR>
+struct MxRefs {             // MXFP8 scale chunks of both operands (unused otherwise)
+  Params::Sf a{}, b{};
+  const int32_t* tile_pref = nullptr;
+};
+
+template <typename T, bool B_MN, int EPI, int BN, bool PAIR, typename OutT = T>
 static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B, int N,
                         int b_rows_per_expert, int b_cols, void* out, int out_cols, void* out_a,
-                        const void* aux, const int32_t* offsets, int* status, cudaStream_t s) {
-  using C = Cfg<T, T, BN, EPI, PAIR>;
-  const bool fp32 = sizeof(T) == 4;
+                        const void* aux, const int32_t* offsets, int* status, cudaStream_t s,
+                        const MxRefs& mx = MxRefs()) {
+  using C = Cfg<T, OutT, BN, EPI, PAIR>;
+  constexpr int ES = sizeof(T);
+  constexpr int OES = sizeof(OutT);
   CUtensorMap ta, tb, to, to2, ti;
-  if (!make_tmap(&ta, A, fp32, K, g.R, C::KB, BM, Box::KMajor)) return MOE_ECUDA;
+  if (!make_tmap(&ta, A, ES, K, g.R, C::KB, BM, Box::KMajor)) return MOE_ECUDA;
   if (!B_MN) {
     const int box_rows = EPI == EPI_SWIGLU_FWD ? BN / 2 : C::BNC;
-    if (!make_tmap(&tb, B, fp32, K, (uint64_t)g.E * b_rows_per_expert, C::KB, box_rows,
+    if (!make_tmap(&tb, B, ES, K, (uint64_t)g.E * b_rows_per_expert, C::KB, box_rows,
                    Box::KMajor))
       return MOE_ECUDA;
   } else {
-    if (!make_tmap(&tb, B, fp32, b_cols, (uint64_t)g.E * b_rows_per_expert, C::MNB, C::KB,
+    if (!make_tmap(&tb, B, ES, b_cols, (uint64_t)g.E * b_rows_per_expert, C::MNB, C::KB,
                    Box::MNMajor))
       return MOE_ECUDA;
   }
-  if (!make_tmap(&to, out, fp32, out_cols, g.R, 32, 32, Box::Chunk)) return MOE_ECUDA;
+  if (!make_tmap(&to, out, OES, out_cols, g.R, 32, 32, Box::Chunk)) return MOE_ECUDA;
   to2 = to;
   ti = to;
-  if (EPI == EPI_SWIGLU_FWD && !make_tmap(&to2, out_a, fp32, g.f, g.R, 32, 32, Box::Chunk))
+  if (EPI == EPI_SWIGLU_FWD && !make_tmap(&to2, out_a, OES, g.f, g.R, 32, 32, Box::Chunk))
     return MOE_ECUDA;
-  if (EPI == EPI_SWIGLU_BWD && !make_tmap(&ti, aux, fp32, 2 * (uint64_t)g.f, g.R, 32, 32,
+  if (EPI == EPI_SWIGLU_BWD && !make_tmap(&ti, aux, OES, 2 * (uint64_t)g.f, g.R, 32, 32,
                                           Box::Chunk))
     return MOE_ECUDA;
   Params p{};
@@ -799,8 +872,11 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.out = out;
   p.ldo = out_cols;
   p.out_a = out_a;
+  p.sfa = mx.a;
+  p.sfb = mx.b;
+  p.tile_pref = mx.tile_pref;
   p.status = status;
-  return launch<T, T, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
+  return launch<T, OutT, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
       ta, tb, to, to2, ti, p, ragged_m_tiles(g, N / BN, C::TM), s);
 }
 
@@ -808,13 +884,13 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
 template <typename T, typename OutT, int BN, bool PAIR>
 static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X, int N, void* dW,
                         bool accum, const int32_t* offsets, const CUtensorMap* g_maps,
-                        int* status, cudaStream_t s) {
+                        int* status, cudaStream_t s, const MxRefs& mx = MxRefs()) {
   using C = Cfg<T, OutT, BN, EPI_STORE, PAIR, RAGGED_K>;
-  const bool fp32 = sizeof(T) == 4;
+  constexpr int ES = sizeof(T);
   CUtensorMap ta, tb, to;
-  if (!make_tmap(&ta, G, fp32, M, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
-  if (!make_tmap(&tb, X, fp32, N, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
-  if (!make_tmap(&to, dW, sizeof(OutT) == 4, N, (uint64_t)g.E * M, 32, 32, Box::Chunk))
+  if (!make_tmap(&ta, G, ES, M, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&tb, X, ES, N, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&to, dW, (int)sizeof(OutT), N, (uint64_t)g.E * M, 32, 32, Box::Chunk))
     return MOE_ECUDA;
   Params p{};
   p.offsets = offsets;
@@ -826,6 +902,9 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
   p.out = dW;
   p.accumulate = accum ? 1 : 0;
   p.a_maps = g_maps;
+  p.sfa = mx.a;
+  p.sfb = mx.b;
+  p.tile_pref = mx.tile_pref;
   p.status = status;
   const long long tiles = (long long)g.E * (M / C::TM) * (N / BN);
   return launch<T, OutT, BN, true, true, RAGGED_K, EPI_STORE, PAIR>(
@@ -921,21 +1000,128 @@ template <typename T>
 static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, const void* dH13,
                                    const int32_t* off, CUtensorMap* maps, cudaStream_t s) {
   using C = Cfg<T, T, 128, EPI_STORE>;
-  const bool fp32 = sizeof(T) == 4;
+  constexpr int ES = sizeof(T);
   CUtensorMap t0, t1;
-  if (!make_tmap(&t0, dy_perm, fp32, g.d, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
-  if (!make_tmap(&t1, dH13, fp32, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
+  if (!make_tmap(&t0, dy_perm, ES, g.d, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap(&t1, dH13, ES, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
     return MOE_ECUDA;
   const int threads = 2 * g.E;
   expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, maps);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
+// ------------------------------------------------------------------------ MXFP8 GEMMs
+// Operands are quantised (E4M3 + E8M0 per 32 along each GEMM's K) right before the GEMM
+// that reads them; all quantised tensors and scales live in the workspace (MxWork).
+// One CTA per 128 x 128 tile; scales stream through shared memory into TMEM per stage.
+static inline moe_status cuq(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
+#define MOE_MX_TRY(x)              \
+  do {                             \
+    moe_status _r = (x);           \
+    if (_r != MOE_OK) return _r;   \
+  } while (0)
+
+static Params::Sf sf_ref(const uint8_t* base, int seg_uniform, bool k_major, int W) {
+  Params::Sf f;
+  f.base = base;
+  f.seg_uniform = seg_uniform;
+  f.k_major = k_major ? 1 : 0;
+  f.W = W;
+  return f;
+}
+
+static moe_status mx_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
+                         const int32_t* off, void* H13, void* a, void* y_perm, int* st,
+                         cudaStream_t s, const MxWork& w) {
+  const int E = g.E, d = g.d, f = g.f;
+  const int32_t* tp = w.act_pref;
+  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w13_off, E, 2 * f, s)));
+  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w2_off, E, d, s)));
+  // FC1: x_perm and W13 rowwise along d; W13's scales in the gate/up tile order
+  MOE_MX_TRY(cuq(launch_mx_quantize(x_perm, g.R, d, off, E, false, w.xr, w.xr_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(W13, (int64_t)E * 2 * f, d, w.w13_off, E, false, w.w13r,
+                                    w.w13r_sf, w.w_scratch, s, f)));
+  MxRefs m1;
+  m1.a = sf_ref(w.xr_sf, 0, true, d / 128);
+  m1.b = sf_ref(w.w13r_sf, 2 * f / 128, true, d / 128);
+  m1.tile_pref = tp;
+  MOE_MX_TRY((run_m<fp8, false, EPI_SWIGLU_FWD, 128, false, bf16>(
+      g, w.xr, d, w.w13r, 2 * f, 2 * f, d, H13, 2 * f, a, nullptr, off, st, s, m1)));
+  // FC2: a and W2 rowwise along d_ff
+  MOE_MX_TRY(cuq(launch_mx_quantize(a, g.R, f, off, E, false, w.ar, w.ar_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(W2, (int64_t)E * d, f, w.w2_off, E, false, w.w2r, w.w2r_sf,
+                                    w.w_scratch, s)));
+  MxRefs m2;
+  m2.a = sf_ref(w.ar_sf, 0, true, f / 128);
+  m2.b = sf_ref(w.w2r_sf, d / 128, true, f / 128);
+  m2.tile_pref = tp;
+  return run_m<fp8, false, EPI_STORE, 128, false, bf16>(g, w.ar, f, w.w2r, d, d, f, y_perm, d,
+                                                         nullptr, nullptr, off, st, s, m2);
+}
+
+template <typename OutT>
+static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm,
+                         const void* H13, const void* a, const void* W13, const void* W2,
+                         const int32_t* off, void* dH13, void* dx_perm, void* dW13, void* dW2,
+                         bool accum, CUtensorMap* maps, int* st, cudaStream_t s, const MxWork& w) {
+  const int E = g.E, d = g.d, f = g.f;
+  const int32_t* tp = w.act_pref;
+  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w13_off, E, 2 * f, s)));
+  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w2_off, E, d, s)));
+  // FC2 dgrad (dA = dY . W2_e, K = d): dY rowwise along d, W2 colwise along its d rows
+  MOE_MX_TRY(cuq(launch_mx_quantize(dy_perm, g.R, d, off, E, false, w.dyr, w.dyr_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(W2, (int64_t)E * d, f, w.w2_off, E, true, w.w2c, w.w2c_sf,
+                                    w.w_scratch, s)));
+  MxRefs m1;
+  m1.a = sf_ref(w.dyr_sf, 0, true, d / 128);
+  m1.b = sf_ref(w.w2c_sf, d / 128, false, f / 128);
+  m1.tile_pref = tp;
+  MOE_MX_TRY((run_m<fp8, true, EPI_SWIGLU_BWD, 128, false, bf16>(
+      g, w.dyr, d, w.w2c, f, d, f, dH13, 2 * f, nullptr, H13, off, st, s, m1)));
+  // FC2 wgrad (dW2_e = dY_e^T . a_e, K = the expert's tokens): both colwise along tokens
+  MOE_MX_TRY(cuq(launch_mx_quantize(dy_perm, g.R, d, off, E, true, w.dyc, w.dyc_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(a, g.R, f, off, E, true, w.ac, w.ac_sf, w.act_pref, s)));
+  // FC1 operands of the backward: dH13 both ways, W13 colwise along its 2*d_ff rows,
+  // x_perm colwise along tokens
+  // (dH13 is quantised after the FC2 dgrad that writes it)
+  MOE_MX_TRY(build_wgrad_maps<fp8>(g, w.dyc, w.dhc, off, maps, s));
+  MxRefs m2;
+  m2.a = sf_ref(w.dyc_sf, 0, false, d / 128);
+  m2.b = sf_ref(w.ac_sf, 0, false, f / 128);
+  m2.tile_pref = tp;
+  MOE_MX_TRY((run_k<fp8, OutT, 128, false>(g, w.dyc, d, w.ac, f, dW2, accum, off, maps, st, s,
+                                           m2)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(dH13, g.R, 2 * f, off, E, false, w.dhr, w.dhr_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(dH13, g.R, 2 * f, off, E, true, w.dhc, w.dhc_sf, w.act_pref, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(W13, (int64_t)E * 2 * f, d, w.w13_off, E, true, w.w13c,
+                                    w.w13c_sf, w.w_scratch, s)));
+  MOE_MX_TRY(cuq(launch_mx_quantize(x_perm, g.R, d, off, E, true, w.xc, w.xc_sf, w.act_pref, s)));
+  // FC1 dgrad (dX = dH13 . W13_e, K = 2*d_ff)
+  MxRefs m3;
+  m3.a = sf_ref(w.dhr_sf, 0, true, 2 * f / 128);
+  m3.b = sf_ref(w.w13c_sf, 2 * f / 128, false, d / 128);
+  m3.tile_pref = tp;
+  MOE_MX_TRY((run_m<fp8, true, EPI_STORE, 128, false, bf16>(g, w.dhr, 2 * f, w.w13c, d, 2 * f, d,
+                                                            dx_perm, d, nullptr, nullptr, off, st,
+                                                            s, m3)));
+  // FC1 wgrad (dW13_e = dH13_e^T . X_e)
+  MxRefs m4;
+  m4.a = sf_ref(w.dhc_sf, 0, false, 2 * f / 128);
+  m4.b = sf_ref(w.xc_sf, 0, false, d / 128);
+  m4.tile_pref = tp;
+  return run_k<fp8, OutT, 128, false>(g, w.dhc, 2 * f, w.xc, d, dW13, accum, off, maps + E, st, s,
+                                      m4);
+}
+
 }  // namespace gemm
 
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
                     const int32_t* offsets, void* H13, void* a, void* y_perm, int* status,
-                    cudaStream_t s) {
+                    cudaStream_t s, const MxWork* mx) {
+  if (g.mx) {
+    if (!mx) return MOE_EINVAL;
+    return gemm::mx_fwd(g, x_perm, W13, W2, offsets, H13, a, y_perm, status, s, *mx);
+  }
   moe_status st;
   if (g.fp32) {
     st = gemm::fc1_fwd<float>(g, x_perm, W13, offsets, H13, a, status, s);
@@ -969,7 +1155,17 @@ static moe_status gemm_bwd_t(const GemmShape& g, const void* dy_perm, const void
 moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm, const void* H13,
                     const void* a, const void* W13, const void* W2, const int32_t* offsets,
                     void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
-                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s) {
+                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s,
+                    const MxWork* mx) {
+  if (g.mx) {
+    if (!mx) return MOE_EINVAL;
+    CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_ws);
+    if (dw_fp32)
+      return gemm::mx_bwd<float>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13,
+                                 dW2, dw_accum, maps, status, s, *mx);
+    return gemm::mx_bwd<__nv_bfloat16>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13,
+                                       dx_perm, dW13, dW2, false, maps, status, s, *mx);
+  }
   if (g.fp32)
     return gemm_bwd_t<float>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13,
                              dW2, dw_fp32, dw_accum, maps_ws, status, s);

@@ -44,26 +44,45 @@ cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void
 
 // ----------------------------------------------------------------------------- MXFP8
 size_t mx_sf_bytes(int64_t R, int C, int E);
-// `scratch`: 2*(E+1) int32 of device memory (segment prefixes).
+// `scratch`: 2*(E+1) int32 of device memory; receives tile_pref (prefix of
+// ceil(rows_e/128)) then the prefix of ceil(rows_e/32).  perm_f > 0: SwiGLU weight scale
+// order (see quant_rows_kernel).
 cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
                                bool colwise, uint8_t* codes, uint8_t* sf, int32_t* scratch,
-                               cudaStream_t s);
+                               cudaStream_t s, int perm_f = 0);
+cudaError_t launch_uniform_offsets(int32_t* seg_off, int E, int rows, cudaStream_t s);
+
+// Device buffers of the MXFP8 grouped GEMMs (codes + 512-byte scale chunks).
+struct MxWork {
+  int32_t* act_pref;      // [2(E+1)]: tile prefix (then 32-row prefix) of the experts' rows
+  int32_t* w13_off;       // [E+1] uniform segments of 2*d_ff rows
+  int32_t* w2_off;        // [E+1] uniform segments of d rows
+  int32_t* w_scratch;     // [2(E+1)]
+  uint8_t *xr, *xr_sf, *xc, *xc_sf;       // x_perm rowwise / colwise
+  uint8_t *ar, *ar_sf, *ac, *ac_sf;       // a
+  uint8_t *dyr, *dyr_sf, *dyc, *dyc_sf;   // dy_perm
+  uint8_t *dhr, *dhr_sf, *dhc, *dhc_sf;   // dH13
+  uint8_t *w13r, *w13r_sf, *w13c, *w13c_sf;
+  uint8_t *w2r, *w2r_sf, *w2c, *w2c_sf;
+};
 
 // ----------------------------------------------------------------------------- grouped GEMM
 struct GemmShape {
   int E, R, d, f;
   bool fp32;   // fp32 storage / TF32 MMA, else bf16
+  bool mx;     // bf16 storage, MXFP8 (E4M3 + E8M0 per 32) GEMM operands
 };
 // FC1 (+SwiGLU epilogue) and FC2 forward.
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
                     const int32_t* offsets, void* H13, void* a, void* y_perm, int* status,
-                    cudaStream_t s);
+                    cudaStream_t s, const MxWork* mx = nullptr);
 // FC2 dgrad (+SwiGLU bwd), FC2 wgrad, FC1 dgrad, FC1 wgrad.  `maps_ws`: 2*E*128 bytes
 // of 128-byte-aligned device scratch for the per-expert tensor maps of the wgrads.
 constexpr size_t kTensorMapBytes = 128;
 moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm, const void* H13,
                     const void* a, const void* W13, const void* W2, const int32_t* offsets,
                     void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
-                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s);
+                    bool dw_accum, void* maps_ws, int* status, cudaStream_t s,
+                    const MxWork* mx = nullptr);
 
 }  // namespace moe

@@ -33,7 +33,9 @@ inline int64_t R_of(const moe_desc& d) { return (int64_t)d.T * d.k; }
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 struct WsLayout {
-  size_t status, hist, cta_base, maps, dy_perm, dH13, dx_perm, dx_router, total;
+  size_t status, hist, cta_base, maps, dy_perm, dH13, dx_perm, dx_router;
+  size_t mx_ints, mx_bytes[24];   // MXFP8 operands (codes and scale chunks), see MxWork
+  size_t total;
 };
 
 WsLayout ws_layout(const moe_desc& d) {
@@ -51,9 +53,25 @@ WsLayout ws_layout(const moe_desc& d) {
   w.dx_perm = o; o = up(o + R * d.d * es);
   w.dx_router = o;
   if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.d * 4);
+  w.mx_ints = o;
+  if (d.dtype == MOE_MXFP8) {
+    const size_t E = d.E, f = d.d_ff, dm = d.d;
+    o = up(o + 6 * (E + 1) * 4);
+    // (rows, cols, segments) of x_perm r/c, a r/c, dy r/c, dH13 r/c, W13 r/c, W2 r/c
+    const size_t rows[12] = {R, R, R, R, R, R, R, R, E * 2 * f, E * 2 * f, E * dm, E * dm};
+    const size_t cols[12] = {dm, dm, f, f, dm, dm, 2 * f, 2 * f, dm, dm, f, f};
+    for (int i = 0; i < 12; ++i) {
+      w.mx_bytes[2 * i] = o;
+      o = up(o + rows[i] * cols[i]);
+      w.mx_bytes[2 * i + 1] = o;
+      o = up(o + mx_sf_bytes((int64_t)rows[i], (int)cols[i], d.E));
+    }
+  }
   w.total = o;
   return w;
 }
+
+
 
 moe_saved_layout saved_layout(const moe_desc& d) {
   moe_saved_layout s;
@@ -89,7 +107,7 @@ moe_status check(const moe_desc* d) {
   if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
   if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW)) return MOE_EINVAL;
   if ((d->flags & MOE_FLAG_ACCUM_DW) && !(d->flags & MOE_FLAG_DW_FP32)) return MOE_EINVAL;
-  if (d->dtype == MOE_MXFP8) return MOE_EUNSUPPORTED;
+  if (d->dtype == MOE_MXFP8 && d->d_ff % 128 != 0) return MOE_EUNSUPPORTED;
   return MOE_OK;
 }
 
@@ -128,6 +146,26 @@ inline const P* at(const void* base, size_t off) {
 }
 inline moe_status cu(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 
+MxWork mx_work(const moe_desc& d, void* ws) {
+  const WsLayout w = ws_layout(d);
+  MxWork m;
+  int32_t* ints = at<int32_t>(ws, w.mx_ints);
+  const int E1 = d.E + 1;
+  m.act_pref = ints;
+  m.w_scratch = ints + 2 * E1;
+  m.w13_off = ints + 4 * E1;
+  m.w2_off = ints + 5 * E1;
+  uint8_t* b[24];
+  for (int i = 0; i < 24; ++i) b[i] = at<uint8_t>(ws, w.mx_bytes[i]);
+  m.xr = b[0]; m.xr_sf = b[1]; m.xc = b[2]; m.xc_sf = b[3];
+  m.ar = b[4]; m.ar_sf = b[5]; m.ac = b[6]; m.ac_sf = b[7];
+  m.dyr = b[8]; m.dyr_sf = b[9]; m.dyc = b[10]; m.dyc_sf = b[11];
+  m.dhr = b[12]; m.dhr_sf = b[13]; m.dhc = b[14]; m.dhc_sf = b[15];
+  m.w13r = b[16]; m.w13r_sf = b[17]; m.w13c = b[18]; m.w13c_sf = b[19];
+  m.w2r = b[20]; m.w2r_sf = b[21]; m.w2c = b[22]; m.w2c_sf = b[23];
+  return m;
+}
+
 #define MOE_TRY(expr)                  \
   do {                                 \
     moe_status _st = (expr);           \
@@ -141,6 +179,7 @@ GemmShape gshape(const moe_desc& d) {
   g.d = d.d;
   g.f = d.d_ff;
   g.fp32 = d.dtype == MOE_FP32;
+  g.mx = d.dtype == MOE_MXFP8;
   return g;
 }
 
@@ -169,8 +208,9 @@ moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_p
     MOE_TRY(cu(cudaMemsetAsync(dW13, 0, (size_t)d.E * 2 * d.d_ff * d.d * es, s)));
     return cu(cudaMemsetAsync(dW2, 0, (size_t)d.E * d.d * d.d_ff * es, s));
   }
+  MxWork mx = mx_work(d, ws);
   return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13, dW2,
-                  fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s);
+                  fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s, &mx);
 }
 
 moe_status router_fwd_body(const moe_desc& d, const void* x, const void* Wr, float* logits,
@@ -298,8 +338,9 @@ moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const 
   if (x_perm_sf) return MOE_EINVAL;
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   if (R_of(*desc) == 0) return MOE_OK;
+  MxWork mx = mx_work(*desc, ws);
   return gemm_fwd(gshape(*desc), x_perm, W13, W2, offsets, H13, a, y_perm, status_ptr(ws),
-                  S(stream));
+                  S(stream), &mx);
 }
 
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* gates,
@@ -419,8 +460,9 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   void* x_perm = at<char>(saved, L.x_perm);
   void* y_perm = at<char>(saved, L.y_perm);
   MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, x_perm, st, s)));
+  MxWork mx = mx_work(d, ws);
   MOE_TRY(gemm_fwd(gshape(d), x_perm, W13, W2, offsets, at<char>(saved, L.H13),
-                   at<char>(saved, L.a), y_perm, st, s));
+                   at<char>(saved, L.a), y_perm, st, s, &mx));
   return cu(launch_gather_sum(f32, d.T, d.d, d.k, y_perm, gates, slot, nullptr, y, st, s));
 }
 

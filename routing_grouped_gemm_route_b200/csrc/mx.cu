@@ -73,14 +73,19 @@ __global__ void seg_prefix_kernel(const int32_t* __restrict__ seg_off, int E,
 }
 
 // Rowwise: one warp per row, lane l handles blocks l, l+32, ... (64 contiguous bytes each).
+// perm_f > 0 (SwiGLU weights [W1; W3], d_ff = perm_f rows each): the scale of row p is
+// filed under the row order gate[0:64], up[0:64], gate[64:128], up[64:128], ..., the order
+// in which a 128-row B tile of the fused SwiGLU GEMM takes 64 gate and 64 up rows.
 __global__ void __launch_bounds__(256) quant_rows_kernel(
     const __nv_bfloat16* __restrict__ x, int R, int C, const int32_t* __restrict__ seg_off, int E,
-    const int32_t* __restrict__ tile_pref, uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
+    const int32_t* __restrict__ tile_pref, int perm_f, uint8_t* __restrict__ codes,
+    uint8_t* __restrict__ sf) {
   const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= R) return;
   const int e = segment_of(seg_off, E, r);
-  const int p = r - seg_off[e];
+  int p = r - seg_off[e];
+  if (perm_f > 0) p = p < perm_f ? (p / 64) * 128 + (p % 64) : ((p - perm_f) / 64) * 128 + 64 + (p - perm_f) % 64;
   const int64_t group = (int64_t)tile_pref[e] + p / 128;
   const int nb = C / 32;
   const __nv_bfloat16* row = x + (int64_t)r * C;
@@ -103,7 +108,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
              ((uint32_t)e4m3(scalbnf(v[4 * j + 2], -s)) << 16) |
              ((uint32_t)e4m3(scalbnf(v[4 * j + 3], -s)) << 24);
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes + (int64_t)r * C + b * 32);
+    uint4* dst = reinterpret_cast<uint4*>(codes + (int64_t)r * C + b * 32);   // codes stay in x's row order
     dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
     dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
     const int64_t chunk = group * (C / 128) + (b * 32) / 128;
@@ -142,9 +147,25 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
     if (j < nrows) codes[(int64_t)(r0 + j) * C + c] = e4m3(scalbnf(v[j], -s));
   const int64_t chunk = ((int64_t)tile_pref[e] + p0 / 128) * (C / 128) + c / 128;
   sf[sf_byte(chunk, c, (p0 & 127) >> 5)] = static_cast<uint8_t>(s + 127);
+  // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad GEMM
+  // still reads all four scales (its rows past the segment are zero codes), so the absent
+  // blocks get the finite scale 2^-127 rather than whatever the buffer held (0xFF = NaN).
+  if (p0 + 32 >= seg_off[e + 1] - seg_off[e])
+    for (int b = ((p0 & 127) >> 5) + 1; b < 4; ++b) sf[sf_byte(chunk, c, b)] = 0;
+}
+
+// seg_off[e] = e * rows (uniform segments: one per expert's weight matrix)
+__global__ void uniform_offsets_kernel(int32_t* seg_off, int E, int rows) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e <= E) seg_off[e] = e * rows;
 }
 
 }  // namespace
+
+cudaError_t launch_uniform_offsets(int32_t* seg_off, int E, int rows, cudaStream_t s) {
+  uniform_offsets_kernel<<<(E + 1 + 255) / 256, 256, 0, s>>>(seg_off, E, rows);
+  return cudaGetLastError();
+}
 
 size_t mx_sf_bytes(int64_t R, int C, int E) {
   // chunks: (sum_e ceil(rows_e/128)) * (C/128) <= (R/128 + E) * (C/128)
@@ -153,7 +174,7 @@ size_t mx_sf_bytes(int64_t R, int C, int E) {
 
 cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
                                bool colwise, uint8_t* codes, uint8_t* sf, int32_t* scratch,
-                               cudaStream_t s) {
+                               cudaStream_t s, int perm_f) {
   if (R == 0) return cudaSuccess;
   int32_t* tile_pref = scratch;               // [E+1]
   int32_t* blk_pref = scratch + (E + 1);      // [E+1]
@@ -163,7 +184,7 @@ cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* s
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   if (!colwise) {
     quant_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(xb, (int)R, C, seg_off, E, tile_pref,
-                                                            codes, sf);
+                                                            perm_f, codes, sf);
   } else {
     // one CTA row per possible 32-row block: sum_e ceil(rows_e/32) <= R/32 + E
     dim3 grid((C + 255) / 256, (unsigned)((R + 31) / 32 + E));

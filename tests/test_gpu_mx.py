@@ -80,6 +80,19 @@ def test_mx_quantize_bit_exact(cuda_lib, counts, colwise):
         ref_codes, ref_sf, _ = oracle.mx_quantize(X[r0:r1], axis=0 if colwise else 1)
         assert np.array_equal(got_codes[r0:r1], ref_codes), ("codes", e)
         assert np.array_equal(got_sfs[e], ref_sf), ("scales", e)
+    if colwise:
+        # slots of each segment's last chunk past its last 32-row block hold 0 (2^-127)
+        tile = 0
+        for e in range(E):
+            cnt = int(seg_off[e + 1] - seg_off[e])
+            if cnt:
+                last = (cnt - 1) // 32
+                c = np.arange(C)
+                chunk = (tile + last // 4) * (C // 128) + c // 128
+                for b in range(last % 4 + 1, 4):
+                    idx = chunk * 512 + 16 * (c % 32) + 4 * ((c % 128) // 32) + b
+                    assert np.all(got_sf[idx] == 0), ("pad", e, b)
+            tile += (cnt + 127) // 128
 
 
 def test_mx_quantize_rejects_bad_shapes(cuda_lib):

@@ -1,0 +1,162 @@
+"""MXFP8 grouped GEMMs and layer on the GPU against the oracle's MXFP8 arithmetic
+(operands rounded through E4M3 + E8M0 per 32 along each GEMM's K at the same points,
+then exact fp64).  Bound: relative Frobenius error <= 3e-2."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle.mx import mx_quantize_dequantize as mxq
+from routing_grouped_gemm_route_b200 import lib
+from routing_grouped_gemm_route_b200.inputs import Workload, make_inputs, normal_tensor, random_logits
+
+from helpers import f64, npi, rel, run_layer, run_route
+
+pytestmark = pytest.mark.gpu
+TOL_MX = 3e-2
+
+CASES = [(600, 256, 128, 6, 2, None), (1000, 512, 256, 8, 4, "empty"), (96, 256, 128, 4, 4, None),
+         (3000, 1024, 512, 16, 4, None)]
+
+
+def make(T, d, f, E, k, mode, seed=0):
+    desc = lib.make_desc(T, d, f, E, k, "mxfp8")
+    L = random_logits(T, E, seed=seed + 11)
+    if mode == "empty":
+        L[:, ::3] -= 50.0
+    r = run_route(desc, L.cuda())
+    x = normal_tensor((T, d), seed=seed + 12).cuda()
+    W13 = normal_tensor((E, 2 * f, d), seed=seed + 13, std=0.02).cuda()
+    W2 = normal_tensor((E, d, f), seed=seed + 14, std=0.02).cuda()
+    ws = lib.alloc_workspace(desc)
+    xp = torch.empty(T * k, d, dtype=torch.bfloat16, device="cuda")
+    lib.moe_dispatch(desc, x, r["slot"], xp, ws)
+    return desc, r, W13, W2, ws, xp
+
+
+def gpu_fwd(desc, r, W13, W2, ws, xp):
+    R, d, f = desc.T * desc.k, desc.d, desc.d_ff
+    H13 = torch.full((R, 2 * f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    a = torch.full((R, f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    yp = torch.full((R, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lib.moe_grouped_gemm_fwd(desc, xp, W13, W2, r["offsets"], H13, a, yp, ws)
+    torch.cuda.synchronize()
+    assert lib.moe_read_device_status(ws) == 0
+    return H13, a, yp
+
+
+@pytest.mark.parametrize("T,d,f,E,k,mode", CASES)
+def test_mxfp8_grouped_gemm_fwd(cuda_lib, T, d, f, E, k, mode):
+    desc, r, W13, W2, ws, xp = make(T, d, f, E, k, mode)
+    H13, a, yp = gpu_fwd(desc, r, W13, W2, ws, xp)
+    off = npi(r["offsets"])
+    W13h, W2h, X, A = f64(W13), f64(W2), f64(xp), f64(a)
+    refH = np.zeros((T * k, 2 * f))
+    refY = np.zeros((T * k, d))
+    for e in range(E):
+        s = slice(off[e], off[e + 1])
+        if off[e + 1] == off[e]:
+            continue
+        refH[s] = mxq(X[s], 1) @ mxq(W13h[e], 1).T
+        refY[s] = mxq(A[s], 1) @ mxq(W2h[e], 1).T
+    assert rel(H13, refH) < TOL_MX
+    h1, h3 = refH[:, :f], refH[:, f:]
+    assert rel(a, oracle.silu(h1) * h3) < TOL_MX
+    assert rel(yp, refY) < TOL_MX
+    assert not torch.isnan(yp).any()
+
+
+@pytest.mark.parametrize("T,d,f,E,k,mode", CASES)
+def test_mxfp8_grouped_gemm_bwd(cuda_lib, T, d, f, E, k, mode):
+    desc, r, W13, W2, ws, xp = make(T, d, f, E, k, mode, seed=3)
+    H13, a, yp = gpu_fwd(desc, r, W13, W2, ws, xp)
+    R = T * k
+    dyp = normal_tensor((R, d), seed=21).cuda()
+    dH13 = torch.full((R, 2 * f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dxp = torch.full((R, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dW13 = torch.full((E, 2 * f, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    dW2 = torch.full((E, d, f), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lib.moe_grouped_gemm_bwd(desc, dyp, xp, H13, a, W13, W2, r["offsets"], dH13, dxp, dW13, dW2, ws)
+    torch.cuda.synchronize()
+    assert lib.moe_read_device_status(ws) == 0
+    off = npi(r["offsets"])
+    W13h, W2h = f64(W13), f64(W2)
+    dY, A, X, H, dHg = f64(dyp), f64(a), f64(xp), f64(H13), f64(dH13)
+    ref_dH = np.zeros((R, 2 * f))
+    ref_dX = np.zeros((R, d))
+    for e in range(E):
+        s = slice(off[e], off[e + 1])
+        if off[e + 1] == off[e]:
+            assert torch.all(dW13[e] == 0) and torch.all(dW2[e] == 0), e
+            continue
+        ref_dH[s] = oracle.swiglu_bwd(mxq(dY[s], 1) @ mxq(W2h[e], 0), H[s])
+        ref_dX[s] = mxq(dHg[s], 1) @ mxq(W13h[e], 0)
+        assert rel(dW2[e], mxq(dY[s], 0).T @ mxq(A[s], 0)) < TOL_MX, ("dW2", e)
+        assert rel(dW13[e], mxq(dHg[s], 0).T @ mxq(X[s], 0)) < TOL_MX, ("dW13", e)
+    assert rel(dH13, ref_dH) < TOL_MX
+    assert rel(dxp, ref_dX) < TOL_MX
+
+
+@pytest.mark.parametrize("T,d,E,k,f", [(700, 256, 8, 4, 128), (2000, 512, 128, 8, 256)])
+def test_mxfp8_layer_matches_mx_oracle(cuda_lib, T, d, E, k, f):
+    w = Workload("mx", T, d, E, k, f, "mxfp8", router=False, skew=False, seed=T)
+    inp = make_inputs(w)
+    desc, layer, dv, y, g, status = run_layer(w, inp)
+    assert status == 0
+    x, dy, L = f64(inp["x"]), f64(inp["dy"]), f64(inp["logits"])
+    W13, W2 = inp["W13"].float().numpy(), inp["W2"].float().numpy()
+    fwd = oracle.layer_fwd(x, W13, W2, logits=L, k=k, mx=True)
+    bwd = oracle.layer_bwd(fwd, dy, x, W13, W2, mx=True)
+    assert np.array_equal(npi(layer.views()["topk_idx"]), fwd["topk_idx"])
+    assert rel(y, fwd["y"]) < TOL_MX
+    for name in ("dx", "d_logits", "dW13", "dW2"):
+        assert rel(g[name], bwd[name]) < TOL_MX, name
+    # against the unquantised oracle the error is reported, not bounded
+    plain = oracle.layer_fwd(x, W13, W2, logits=L, k=k)
+    print("MXFP8 vs unquantised oracle: y rel err %.3e" % rel(y, plain["y"]))
+
+
+def test_full_size_mxfp8_sampled(cuda_lib):
+    """The MXFP8 workload at full size (T=32768, d=4096, E=128, top-8, d_ff=1536), one
+    layer fwd+bwd as the bench runs it.  Routing is checked in full; the grouped GEMMs on
+    sampled experts, each recomputed by the oracle over all of that expert's rows (a
+    grouped GEMM is one GEMM per expert, so one expert's rows are a complete case); the
+    combine on sampled tokens from the device's y_perm."""
+    from routing_grouped_gemm_route_b200.inputs import WORKLOADS
+    w = WORKLOADS["e128_mxfp8_large"]
+    inp = make_inputs(w, device="cuda")
+    desc, layer, dv, y, g, status = run_layer(w, inp)
+    assert status == 0
+    v = layer.views()
+    L = inp["logits"].cpu().numpy()
+    ref = oracle.route(L, w.k, w.E)
+    for key in ("topk_idx", "offsets", "slot", "row_token"):
+        assert np.array_equal(npi(v[key]), ref[key]), key
+    rng = np.random.default_rng(0)
+    # combine at full size: y on sampled tokens from the device's y_perm rows
+    toks = np.sort(rng.choice(w.T, size=256, replace=False))
+    yp = f64(v["y_perm"][torch.as_tensor(ref["slot"][toks].reshape(-1), device="cuda").long()])
+    yp = yp.reshape(len(toks), w.k, w.d)
+    want = np.einsum("tj,tjd->td", ref["gates"][toks], yp)
+    assert rel(y[toks], want) < 5e-3
+    # grouped GEMMs on sampled experts: every row of the expert
+    x, dy = inp["x"], inp["dy"]
+    counts = ref["counts"]
+    for e in dict.fromkeys([int(np.argmax(counts)), int(np.argmin(counts)), int(rng.integers(w.E))]):
+        r0, r1 = int(ref["offsets"][e]), int(ref["offsets"][e + 1])
+        if r1 == r0:
+            assert torch.all(g["dW13"][e] == 0) and torch.all(g["dW2"][e] == 0)
+            continue
+        rows = torch.as_tensor(ref["row_token"][r0:r1], device="cuda").long()
+        Xe = f64(x[rows])
+        gate = ref["gates"].reshape(-1)[np.argsort(ref["slot"].reshape(-1))][r0:r1]
+        dYe = gate[:, None] * f64(dy[rows])              # the expert's rows of dy_perm
+        W13e, W2e = f64(inp["W13"][e:e + 1]), f64(inp["W2"][e:e + 1])
+        off = np.array([0, r1 - r0])
+        H, A, Y = oracle.experts_fwd(Xe, off, W13e, W2e, mx=True)
+        assert rel(v["H13"][r0:r1], H) < TOL_MX, e
+        assert rel(v["a"][r0:r1], A) < TOL_MX, e
+        assert rel(v["y_perm"][r0:r1], Y) < TOL_MX, e
+        _, _, dW13, dW2 = oracle.experts_bwd(dYe, Xe, H, A, off, W13e, W2e, mx=True)
+        assert rel(g["dW2"][e], dW2[0]) < TOL_MX, e
+        assert rel(g["dW13"][e], dW13[0]) < TOL_MX, e

@@ -102,3 +102,45 @@ def test_partial_block_and_axis(n):
     assert np.all(dv[sat] == np.sign(v[sat]) * 448)
     assert np.all(np.abs(dv - v)[nrm] <= 2.0 ** -4 * np.abs(v)[nrm])
     assert np.all(np.abs(dv - v)[sub] <= 2.0 ** -10)
+
+
+# ---------------------------------------------------------------- bf16 rounding (BF16 I/O)
+
+def test_bf16_round_hand_cases():
+    r = oracle.bf16_round
+    # bf16 spacing at 1 is 2**-7: 1 + 2**-8 is a tie -> even (1.0); 1 + 3*2**-8 -> 1 + 2**-6
+    assert r(1.0 + 2.0 ** -8) == 1.0
+    assert r(1.0 + 3 * 2.0 ** -8) == 1.0 + 2.0 ** -6
+    assert r(-(1.0 + 3 * 2.0 ** -8)) == -(1.0 + 2.0 ** -6)
+    # just above the tie rounds up even where an fp32 intermediate would land on the tie
+    assert r(1.0 + 2.0 ** -8 + 2.0 ** -40) == 1.0 + 2.0 ** -7
+    assert r(3.0) == 3.0 and r(0.0) == 0.0 and np.signbit(r(-0.0))
+    # smallest subnormal 2**-133; half of it is a tie -> 0
+    assert r(2.0 ** -133) == 2.0 ** -133
+    assert r(2.0 ** -134) == 0.0
+    assert r(1.5 * 2.0 ** -133) == 2.0 ** -132
+    # largest finite 2**128 - 2**120; the tie above it overflows
+    assert r(2.0 ** 128 - 2.0 ** 120) == 2.0 ** 128 - 2.0 ** 120
+    assert np.isinf(r(2.0 ** 128 - 2.0 ** 119))
+
+
+def test_bf16_round_matches_torch_cast_of_fp32():
+    # values exact in fp32, so torch's fp32 -> bf16 cast is one rounding of the same number
+    g = np.random.default_rng(5)
+    v = (g.standard_normal(200000) * np.exp(g.uniform(-95, 85, 200000))).astype(np.float32)
+    v[:50] = np.float32(1.0) + np.float32(2.0 ** -8) * np.arange(50, dtype=np.float32)   # ties
+    want = torch.from_numpy(v).to(torch.bfloat16).double().numpy()
+    got = oracle.bf16_round(v.astype(np.float64))
+    assert np.array_equal(got, want)
+    # idempotent
+    assert np.array_equal(oracle.bf16_round(got), got)
+
+
+def test_mx_operand_of_layer_oracle_is_bf16_rounded():
+    # a layer whose activation "a" is not bf16-representable: the MX oracle quantises
+    # bf16(a), so its output equals the one computed from bf16-rounded a
+    from oracle.moe_oracle import _mx
+    g = np.random.default_rng(1)
+    a = g.standard_normal((64, 128))
+    assert np.array_equal(_mx(a, 1, True), mx.mx_quantize_dequantize(oracle.bf16_round(a), axis=1))
+    assert _mx(a, 1, False) is a
