@@ -50,6 +50,8 @@ def parse():
                     help="override T (a smaller case of the workload, for profiling)")
     ap.add_argument("--experts", type=int, default=None,
                     help="override E (a smaller case of the workload, for profiling)")
+    ap.add_argument("--dtype", default=None, choices=["fp32", "bf16", "mxfp8"],
+                    help="override the workload's GEMM precision (e.g. the MXFP8 shape in bf16)")
     return ap.parse_args()
 
 
@@ -315,6 +317,8 @@ def main():
         w = w.replace(T=args.tokens, name=w.name + f"[T={args.tokens}]")
     if args.experts is not None:
         w = w.replace(E=args.experts, name=w.name + f"[E={args.experts}]")
+    if args.dtype is not None and args.dtype != w.dtype:
+        w = w.replace(dtype=args.dtype, name=w.name + f"[{args.dtype}]")
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, w, world, rank)
@@ -355,9 +359,9 @@ def main():
         stages = ["router"] + stages + ["router_bwd"]
     mx = w.dtype == "mxfp8"
     # GEMM stages: bf16/fp32 fwd = 2 GEMMs, bwd = tensor-map builder + 4 GEMMs; MXFP8 adds
-    # the quantisers (segment prefix + quantise per operand) and two offset fills per stage
-    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 12 if mx else 2,
-                "combine": 1, "combine_bwd": 1, "gemm_bwd": 23 if mx else 5, "dispatch_bwd": 1,
+    # the quantisers (one segment prefix per stage, one launch per quantised operand)
+    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 7 if mx else 2,
+                "combine": 1, "combine_bwd": 1, "gemm_bwd": 12 if mx else 5, "dispatch_bwd": 1,
                 "router_bwd": 3}
 
     def run_stage(name):

@@ -100,11 +100,16 @@ struct Cfg {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = BNC * 128;
   static constexpr int STAGE = A_BYTES + B_BYTES;
-  // MXFP8: one 512-byte scale chunk for A's 128 rows and one per 128 rows of B, per stage
+  // MXFP8: per stage, one 512-byte scale chunk for this CTA's 128 rows of A and one per
+  // 128 rows of the whole BN of B (in a pair each CTA's MMA half reads all of B's scales
+  // from its own TMEM)
   static constexpr bool MX = ES == 1;
-  static constexpr int SF_CHUNKS_B = MX ? BNC / 128 : 0;
+  static constexpr int SF_CHUNKS_B = MX ? BN / 128 : 0;
   static constexpr int SF_STAGE = MX ? 512 * (1 + SF_CHUNKS_B) : 0;
   static constexpr int SFC = MX ? 4 * (1 + SF_CHUNKS_B) : 0;      // TMEM columns per stage
+  // accumulator buffers in TMEM: two (the epilogue drains one while the MMAs fill the
+  // other), except for MXFP8 256-column tiles, where the scale columns leave room for one
+  static constexpr int NACC = MX && BN == 256 ? 1 : 2;
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
   // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there);
   // elsewhere 4 warps keep up and leave more shared memory to the operand ring
@@ -130,8 +135,8 @@ struct Cfg {
   static constexpr int STAGES =
       BUDGET / (STAGE + SF_STAGE) > 8 ? 8 : BUDGET / (STAGE + SF_STAGE);
   static_assert(STAGES >= 2, "shared memory budget");
-  static_assert(!MX || 2 * BN + STAGES * SFC <= 512, "tensor memory budget");
-  static constexpr int SF_COL0 = 2 * BN;                          // first scale column
+  static_assert(!MX || NACC * BN + STAGES * SFC <= 512, "tensor memory budget");
+  static constexpr int SF_COL0 = NACC * BN;                       // first scale column
   static constexpr size_t smem_bytes(int E) {
     return 1024 + size_t(STAGES) * (STAGE + SF_STAGE) + EPI_BYTES + BAR_BYTES +
            size_t(2 * (E + 1) + 8) * 4;
@@ -253,14 +258,15 @@ template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int
 __global__ void __launch_bounds__(Cfg<T, OutT, BN, EPI, PAIR, MODE>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
-                    const __grid_constant__ CUtensorMap tmI, const Params p) {
+                    const __grid_constant__ CUtensorMap tmI, const __grid_constant__ CUtensorMap tmSA,
+                    const __grid_constant__ CUtensorMap tmSB, const Params p) {
   using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
   using ActT = typename std::conditional<sizeof(T) == 4, float, bf16>::type;  // epilogue inputs
   constexpr bool kTF32 = sizeof(T) == 4;
   constexpr bool kMX = C::MX;
   constexpr uint32_t IDESC = kMX ? idesc_mxf8(C::TM, BN, A_MN, B_MN)
                                  : idesc_f32acc(C::TM, BN, kTF32 ? 2u : 1u, A_MN, B_MN);
-  static_assert(!(kMX && PAIR), "MXFP8 tiles run one CTA per tile");
+  static_assert(!(kMX && EPI == EPI_SWIGLU_FWD && !PAIR), "MXFP8 SwiGLU forward: pair tiles");
   static_assert(!PAIR || !kTF32, "CTA pairs run the 16-bit kernels");
   static_assert(!B_MN || C::BNC % C::MNB == 0, "an M/N-major B half is whole 128-byte blocks");
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
@@ -388,16 +394,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           };
           const int k0 = kb * C::KB;
           if constexpr (kMX) {
-            // this stage's scale chunks: A's 128 rows, then B's rows 128 at a time
+            // this stage's scale chunks (one 512-byte row of a scale map each): my 128 rows
+            // of A, then all of B's rows 128 at a time
             uint8_t* sfs = sf_smem + stage * C::SF_STAGE;
-            const int a_mn = MODE == RAGGED_M ? tl.m0 + arow : tl.m0 + arow;
-            bulk_load(sfs, p.sfa.base + 512 * sf_chunk(p.sfa, p.tile_pref, tl.e, a_mn, kb), 512,
-                      &full[stage]);
+            load(sfs, &tmSA, 0, static_cast<int>(sf_chunk(p.sfa, p.tile_pref, tl.e, tl.m0 + arow, kb)));
 #pragma unroll
             for (int j = 0; j < C::SF_CHUNKS_B; ++j)
-              bulk_load(sfs + 512 * (1 + j),
-                        p.sfb.base + 512 * sf_chunk(p.sfb, p.tile_pref, tl.e, tl.n0 + bcol + 128 * j, kb),
-                        512, &full[stage]);
+              load(sfs + 512 * (1 + j), &tmSB, 0,
+                   static_cast<int>(sf_chunk(p.sfb, p.tile_pref, tl.e, tl.n0 + 128 * j, kb)));
           }
           if (MODE == RAGGED_M) {
             load(sA, &tmA, k0, tl.row0 + arow);
@@ -476,17 +480,20 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             sfa_t = tmem_base + col;
             sfb_t = tmem_base + col + 4;
 #pragma unroll
-            for (int j = 0; j <= C::SF_CHUNKS_B; ++j)
-              tmem_cp_scales(tmem_base + col + 4 * j, sdesc(src + 512 * j, 128, 128, 0));
+            for (int j = 0; j <= C::SF_CHUNKS_B; ++j) {
+              if (PAIR) tmem_cp_scales_pair(tmem_base + col + 4 * j, sdesc(src + 512 * j, 128, 128, 0));
+              else tmem_cp_scales(tmem_base + col + 4 * j, sdesc(src + 512 * j, 128, 128, 0));
+            }
           }
 #pragma unroll
           for (int kk = 0; kk < C::KB / C::UK; ++kk) {
             const uint64_t ad = a_desc0 + so + kk * A_STEP;
             const uint64_t bd = b_desc0 + so + kk * B_STEP;
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
-            if constexpr (kMX)
-              umma_mx(d_tmem, ad, bd, IDESC | idesc_sf_ids(kk, kk), sfa_t, sfb_t, accum);
-            else if (PAIR) umma_pair(d_tmem, ad, bd, IDESC, accum);
+            if constexpr (kMX) {
+              if (PAIR) umma_mx_pair(d_tmem, ad, bd, IDESC | idesc_sf_ids(kk, kk), sfa_t, sfb_t, accum);
+              else umma_mx(d_tmem, ad, bd, IDESC | idesc_sf_ids(kk, kk), sfa_t, sfb_t, accum);
+            } else if (PAIR) umma_pair(d_tmem, ad, bd, IDESC, accum);
             else umma<kTF32>(d_tmem, ad, bd, IDESC, accum);
           }
           if (PAIR) umma_commit_pair(&empty[stage], 3);   // frees the stage in both CTAs
@@ -495,7 +502,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         if (PAIR) umma_commit_pair(&tfull[acc], 3);
         else umma_commit(&tfull[acc]);
-        if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+        if (++acc == C::NACC) { acc = 0; acc_phase ^= 1u; }
       }
       // (a kernel's tcgen05 instructions all use one cta_group)
       if (PAIR) umma_commit_pair(fin, 1);
@@ -681,7 +688,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (PAIR) mbar_arrive_remote(tempty_leader + static_cast<uint32_t>(acc) * 8u);
         else mbar_arrive(&tempty[acc]);
       }
-      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (++acc == C::NACC) { acc = 0; acc_phase ^= 1u; }
     }
     if (lane == 0) {
       bulk_wait_all();
@@ -746,6 +753,21 @@ static EncodeTiledFn encode_fn() {
 
 enum class Box { KMajor, MNMajor, Chunk };
 
+// MXFP8 scale chunks as a 2-D map of `chunks` rows of 512 bytes (128 x uint32), one row
+// per box: a scale load is a TMA load of row `chunk` (x = 0), so it can complete on the
+// pair leader's barrier like the operand tiles.
+static bool make_sf_map(CUtensorMap* m, const void* base, int64_t chunks) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc || chunks < 1) return false;
+  cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(chunks)};
+  cuuint64_t strides[1] = {512};
+  cuuint32_t box[2] = {128, 1};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<void*>(base), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2-D row-major tensor [rows, cols] of bf16 or fp32 with box [box_rows, box_cols]:
 //   KMajor / MNMajor operand tiles: 128-byte rows, 128-byte swizzle (M/N-major fp32
 //   tiles: the 32-byte-atom variant, the layout the tensor core takes for M/N-major
@@ -776,8 +798,8 @@ static bool make_tmap(CUtensorMap* m, const void* base, int es_, uint64_t cols, 
 
 template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
 static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
-                         const CUtensorMap& to2, const CUtensorMap& ti, const Params& p,
-                         int max_tiles, cudaStream_t s) {
+                         const CUtensorMap& to2, const CUtensorMap& ti, const CUtensorMap& tsa,
+                         const CUtensorMap& tsb, const Params& p, int max_tiles, cudaStream_t s) {
   using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
   auto kern = grouped_gemm_kernel<T, OutT, BN, A_MN, B_MN, MODE, EPI, PAIR>;
   const size_t smem = C::smem_bytes(p.E);
@@ -812,7 +834,8 @@ static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   if (max_tiles < units) units = max_tiles;
   if (units < 1) return MOE_OK;
   cfg.gridDim = dim3(PAIR ? 2 * units : units, 1, 1);
-  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, ti, p) != cudaSuccess) return MOE_ECUDA;
+  if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, ti, tsa, tsb, p) != cudaSuccess)
+    return MOE_ECUDA;
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
@@ -830,8 +853,21 @@ static int ragged_m_tiles(const GemmShape& g, int n_tiles, int tm) {
 // forward also writes out_a [R, f]; SwiGLU backward reads aux [R, 2f].
 struct MxRefs {             // MXFP8 scale chunks of both operands (unused otherwise)
   Params::Sf a{}, b{};
+  int64_t a_chunks = 0, b_chunks = 0;   // sizes of the two scale buffers in chunks
   const int32_t* tile_pref = nullptr;
 };
+
+// Scale maps of an MXFP8 GEMM (copies of `dummy` for the other kernels, which never
+// read them).
+static bool sf_maps(const MxRefs& mx, bool is_mx, const CUtensorMap& dummy, CUtensorMap* tsa,
+                    CUtensorMap* tsb) {
+  if (!is_mx) {
+    *tsa = dummy;
+    *tsb = dummy;
+    return true;
+  }
+  return make_sf_map(tsa, mx.a.base, mx.a_chunks) && make_sf_map(tsb, mx.b.base, mx.b_chunks);
+}
 
 template <typename T, bool B_MN, int EPI, int BN, bool PAIR, typename OutT = T>
 static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B, int N,
@@ -876,8 +912,10 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.sfb = mx.b;
   p.tile_pref = mx.tile_pref;
   p.status = status;
+  CUtensorMap tsa, tsb;
+  if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
   return launch<T, OutT, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
-      ta, tb, to, to2, ti, p, ragged_m_tiles(g, N / BN, C::TM), s);
+      ta, tb, to, to2, ti, tsa, tsb, p, ragged_m_tiles(g, N / BN, C::TM), s);
 }
 
 // RAGGED_K GEMM: dW_e[M, N] = G_e^T . X_e with G [R, M] and X [R, N] (both act, M/N-major).
@@ -906,9 +944,11 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
   p.sfb = mx.b;
   p.tile_pref = mx.tile_pref;
   p.status = status;
+  CUtensorMap tsa, tsb;
+  if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
   const long long tiles = (long long)g.E * (M / C::TM) * (N / BN);
   return launch<T, OutT, BN, true, true, RAGGED_K, EPI_STORE, PAIR>(
-      ta, tb, to, to, to, p, tiles > (1 << 30) ? (1 << 30) : (int)tiles, s);
+      ta, tb, to, to, to, tsa, tsb, p, tiles > (1 << 30) ? (1 << 30) : (int)tiles, s);
 }
 
 #define MOE_DISPATCH_BN(bn, CALL)                             \
@@ -1030,33 +1070,76 @@ static Params::Sf sf_ref(const uint8_t* base, int seg_uniform, bool k_major, int
   return f;
 }
 
+// Segments of the experts' rows (their prefixes are computed once per direction).
+static MxSegs act_segs(const GemmShape& g, const int32_t* off, const MxWork& w) {
+  MxSegs a;
+  a.off = off;
+  a.tile_pref = w.act_pref;
+  a.blk_pref = w.act_pref + (g.E + 1);
+  a.E = g.E;
+  return a;
+}
+static MxSegs weight_segs(int E, int rows) {
+  MxSegs s;
+  s.E = E;
+  s.rows = rows;
+  return s;
+}
+
+// Scale references of an activation operand (ragged expert segments of the R rows, C
+// columns) and of a weight operand (E uniform segments of `rows` rows).
+static void act_sf(Params::Sf& f, int64_t& chunks, const GemmShape& g, const uint8_t* sf, int C,
+                   bool k_major) {
+  f = sf_ref(sf, 0, k_major, C / 128);
+  chunks = static_cast<int64_t>(mx_sf_bytes(g.R, C, g.E) / 512);
+}
+static void weight_sf(Params::Sf& f, int64_t& chunks, const GemmShape& g, const uint8_t* sf,
+                      int rows, int C, bool k_major) {
+  f = sf_ref(sf, rows / 128, k_major, C / 128);
+  chunks = static_cast<int64_t>(g.E) * (rows / 128) * (C / 128);
+}
+
+// MXFP8 GEMMs run 256 x 256 CTA-pair tiles where the output's N (and, for wgrad, M)
+// divides by 256, else 128 x 128 single-CTA tiles.  The fused SwiGLU forward always has
+// 2*d_ff % 256 == 0 (MXFP8 needs d_ff % 128 == 0).
 static moe_status mx_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
                          const int32_t* off, void* H13, void* a, void* y_perm, int* st,
                          cudaStream_t s, const MxWork& w) {
   const int E = g.E, d = g.d, f = g.f;
-  const int32_t* tp = w.act_pref;
-  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w13_off, E, 2 * f, s)));
-  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w2_off, E, d, s)));
+  const MxSegs act = act_segs(g, off, w);
+  MOE_MX_TRY(cuq(launch_mx_prefix(off, E, w.act_pref, w.act_pref + (E + 1), s)));
   // FC1: x_perm and W13 rowwise along d; W13's scales in the gate/up tile order
-  MOE_MX_TRY(cuq(launch_mx_quantize(x_perm, g.R, d, off, E, false, w.xr, w.xr_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(W13, (int64_t)E * 2 * f, d, w.w13_off, E, false, w.w13r,
-                                    w.w13r_sf, w.w_scratch, s, f)));
+  MOE_MX_TRY(cuq(launch_mx_quant(x_perm, g.R, d, act, 0, w.xr, w.xr_sf, nullptr, nullptr, st, s)));
+  MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), f, w.w13r,
+                                 w.w13r_sf, nullptr, nullptr, st, s)));
   MxRefs m1;
-  m1.a = sf_ref(w.xr_sf, 0, true, d / 128);
-  m1.b = sf_ref(w.w13r_sf, 2 * f / 128, true, d / 128);
-  m1.tile_pref = tp;
-  MOE_MX_TRY((run_m<fp8, false, EPI_SWIGLU_FWD, 128, false, bf16>(
+  act_sf(m1.a, m1.a_chunks, g, w.xr_sf, d, true);
+  weight_sf(m1.b, m1.b_chunks, g, w.w13r_sf, 2 * f, d, true);
+  m1.tile_pref = w.act_pref;
+  MOE_MX_TRY((run_m<fp8, false, EPI_SWIGLU_FWD, 256, true, bf16>(
       g, w.xr, d, w.w13r, 2 * f, 2 * f, d, H13, 2 * f, a, nullptr, off, st, s, m1)));
   // FC2: a and W2 rowwise along d_ff
-  MOE_MX_TRY(cuq(launch_mx_quantize(a, g.R, f, off, E, false, w.ar, w.ar_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(W2, (int64_t)E * d, f, w.w2_off, E, false, w.w2r, w.w2r_sf,
-                                    w.w_scratch, s)));
+  MOE_MX_TRY(cuq(launch_mx_quant(a, g.R, f, act, 0, w.ar, w.ar_sf, nullptr, nullptr, st, s)));
+  MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, w.w2r, w.w2r_sf,
+                                 nullptr, nullptr, st, s)));
   MxRefs m2;
-  m2.a = sf_ref(w.ar_sf, 0, true, f / 128);
-  m2.b = sf_ref(w.w2r_sf, d / 128, true, f / 128);
-  m2.tile_pref = tp;
+  act_sf(m2.a, m2.a_chunks, g, w.ar_sf, f, true);
+  weight_sf(m2.b, m2.b_chunks, g, w.w2r_sf, d, f, true);
+  m2.tile_pref = w.act_pref;
+  if (d % 256 == 0)
+    return run_m<fp8, false, EPI_STORE, 256, true, bf16>(g, w.ar, f, w.w2r, d, d, f, y_perm, d,
+                                                          nullptr, nullptr, off, st, s, m2);
   return run_m<fp8, false, EPI_STORE, 128, false, bf16>(g, w.ar, f, w.w2r, d, d, f, y_perm, d,
                                                          nullptr, nullptr, off, st, s, m2);
+}
+
+template <typename OutT>
+static moe_status mx_wgrad(const GemmShape& g, const uint8_t* G, int M, const uint8_t* X, int N,
+                           void* dW, bool accum, const int32_t* off, const CUtensorMap* maps,
+                           int* st, cudaStream_t s, const MxRefs& m) {
+  if (M % 256 == 0 && N % 256 == 0)
+    return run_k<fp8, OutT, 256, true>(g, G, M, X, N, dW, accum, off, maps, st, s, m);
+  return run_k<fp8, OutT, 128, false>(g, G, M, X, N, dW, accum, off, maps, st, s, m);
 }
 
 template <typename OutT>
@@ -1065,52 +1148,55 @@ static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_
                          const int32_t* off, void* dH13, void* dx_perm, void* dW13, void* dW2,
                          bool accum, CUtensorMap* maps, int* st, cudaStream_t s, const MxWork& w) {
   const int E = g.E, d = g.d, f = g.f;
-  const int32_t* tp = w.act_pref;
-  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w13_off, E, 2 * f, s)));
-  MOE_MX_TRY(cuq(launch_uniform_offsets(w.w2_off, E, d, s)));
-  // FC2 dgrad (dA = dY . W2_e, K = d): dY rowwise along d, W2 colwise along its d rows
-  MOE_MX_TRY(cuq(launch_mx_quantize(dy_perm, g.R, d, off, E, false, w.dyr, w.dyr_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(W2, (int64_t)E * d, f, w.w2_off, E, true, w.w2c, w.w2c_sf,
-                                    w.w_scratch, s)));
+  const MxSegs act = act_segs(g, off, w);
+  MOE_MX_TRY(cuq(launch_mx_prefix(off, E, w.act_pref, w.act_pref + (E + 1), s)));
+  // dY both ways in one pass: rowwise along d (FC2 dgrad), colwise along tokens (FC2 wgrad);
+  // W2 colwise along its d rows (FC2 dgrad)
+  MOE_MX_TRY(cuq(launch_mx_quant(dy_perm, g.R, d, act, 0, w.dyr, w.dyr_sf, w.dyc, w.dyc_sf, st, s)));
+  MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, nullptr, nullptr,
+                                 w.w2c, w.w2c_sf, st, s)));
   MxRefs m1;
-  m1.a = sf_ref(w.dyr_sf, 0, true, d / 128);
-  m1.b = sf_ref(w.w2c_sf, d / 128, false, f / 128);
-  m1.tile_pref = tp;
-  MOE_MX_TRY((run_m<fp8, true, EPI_SWIGLU_BWD, 128, false, bf16>(
-      g, w.dyr, d, w.w2c, f, d, f, dH13, 2 * f, nullptr, H13, off, st, s, m1)));
-  // FC2 wgrad (dW2_e = dY_e^T . a_e, K = the expert's tokens): both colwise along tokens
-  MOE_MX_TRY(cuq(launch_mx_quantize(dy_perm, g.R, d, off, E, true, w.dyc, w.dyc_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(a, g.R, f, off, E, true, w.ac, w.ac_sf, w.act_pref, s)));
-  // FC1 operands of the backward: dH13 both ways, W13 colwise along its 2*d_ff rows,
-  // x_perm colwise along tokens
-  // (dH13 is quantised after the FC2 dgrad that writes it)
+  act_sf(m1.a, m1.a_chunks, g, w.dyr_sf, d, true);
+  weight_sf(m1.b, m1.b_chunks, g, w.w2c_sf, d, f, false);
+  m1.tile_pref = w.act_pref;
+  if (f % 256 == 0)
+    MOE_MX_TRY((run_m<fp8, true, EPI_SWIGLU_BWD, 256, true, bf16>(
+        g, w.dyr, d, w.w2c, f, d, f, dH13, 2 * f, nullptr, H13, off, st, s, m1)));
+  else
+    MOE_MX_TRY((run_m<fp8, true, EPI_SWIGLU_BWD, 128, false, bf16>(
+        g, w.dyr, d, w.w2c, f, d, f, dH13, 2 * f, nullptr, H13, off, st, s, m1)));
+  // FC2 wgrad (dW2_e = dY_e^T . a_e, K = the expert's tokens): a colwise along tokens
+  MOE_MX_TRY(cuq(launch_mx_quant(a, g.R, f, act, 0, nullptr, nullptr, w.ac, w.ac_sf, st, s)));
   MOE_MX_TRY(build_wgrad_maps<fp8>(g, w.dyc, w.dhc, off, maps, s));
   MxRefs m2;
-  m2.a = sf_ref(w.dyc_sf, 0, false, d / 128);
-  m2.b = sf_ref(w.ac_sf, 0, false, f / 128);
-  m2.tile_pref = tp;
-  MOE_MX_TRY((run_k<fp8, OutT, 128, false>(g, w.dyc, d, w.ac, f, dW2, accum, off, maps, st, s,
-                                           m2)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(dH13, g.R, 2 * f, off, E, false, w.dhr, w.dhr_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(dH13, g.R, 2 * f, off, E, true, w.dhc, w.dhc_sf, w.act_pref, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(W13, (int64_t)E * 2 * f, d, w.w13_off, E, true, w.w13c,
-                                    w.w13c_sf, w.w_scratch, s)));
-  MOE_MX_TRY(cuq(launch_mx_quantize(x_perm, g.R, d, off, E, true, w.xc, w.xc_sf, w.act_pref, s)));
-  // FC1 dgrad (dX = dH13 . W13_e, K = 2*d_ff)
+  act_sf(m2.a, m2.a_chunks, g, w.dyc_sf, d, false);
+  act_sf(m2.b, m2.b_chunks, g, w.ac_sf, f, false);
+  m2.tile_pref = w.act_pref;
+  MOE_MX_TRY(mx_wgrad<OutT>(g, w.dyc, d, w.ac, f, dW2, accum, off, maps, st, s, m2));
+  // dH13 both ways (FC1 dgrad, FC1 wgrad), W13 colwise along its 2*d_ff rows, x_perm
+  // colwise along tokens
+  MOE_MX_TRY(cuq(launch_mx_quant(dH13, g.R, 2 * f, act, 0, w.dhr, w.dhr_sf, w.dhc, w.dhc_sf, st, s)));
+  MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), 0, nullptr,
+                                 nullptr, w.w13c, w.w13c_sf, st, s)));
   MxRefs m3;
-  m3.a = sf_ref(w.dhr_sf, 0, true, 2 * f / 128);
-  m3.b = sf_ref(w.w13c_sf, 2 * f / 128, false, d / 128);
-  m3.tile_pref = tp;
-  MOE_MX_TRY((run_m<fp8, true, EPI_STORE, 128, false, bf16>(g, w.dhr, 2 * f, w.w13c, d, 2 * f, d,
-                                                            dx_perm, d, nullptr, nullptr, off, st,
-                                                            s, m3)));
+  act_sf(m3.a, m3.a_chunks, g, w.dhr_sf, 2 * f, true);
+  weight_sf(m3.b, m3.b_chunks, g, w.w13c_sf, 2 * f, d, false);
+  m3.tile_pref = w.act_pref;
+  if (d % 256 == 0)
+    MOE_MX_TRY((run_m<fp8, true, EPI_STORE, 256, true, bf16>(g, w.dhr, 2 * f, w.w13c, d, 2 * f, d,
+                                                             dx_perm, d, nullptr, nullptr, off,
+                                                             st, s, m3)));
+  else
+    MOE_MX_TRY((run_m<fp8, true, EPI_STORE, 128, false, bf16>(g, w.dhr, 2 * f, w.w13c, d, 2 * f,
+                                                              d, dx_perm, d, nullptr, nullptr,
+                                                              off, st, s, m3)));
   // FC1 wgrad (dW13_e = dH13_e^T . X_e)
+  MOE_MX_TRY(cuq(launch_mx_quant(x_perm, g.R, d, act, 0, nullptr, nullptr, w.xc, w.xc_sf, st, s)));
   MxRefs m4;
-  m4.a = sf_ref(w.dhc_sf, 0, false, 2 * f / 128);
-  m4.b = sf_ref(w.xc_sf, 0, false, d / 128);
-  m4.tile_pref = tp;
-  return run_k<fp8, OutT, 128, false>(g, w.dhc, 2 * f, w.xc, d, dW13, accum, off, maps + E, st, s,
-                                      m4);
+  act_sf(m4.a, m4.a_chunks, g, w.dhc_sf, 2 * f, false);
+  act_sf(m4.b, m4.b_chunks, g, w.xc_sf, d, false);
+  m4.tile_pref = w.act_pref;
+  return mx_wgrad<OutT>(g, w.dhc, 2 * f, w.xc, d, dW13, accum, off, maps + E, st, s, m4);
 }
 
 }  // namespace gemm

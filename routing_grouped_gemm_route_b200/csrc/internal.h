@@ -44,20 +44,31 @@ cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void
 
 // ----------------------------------------------------------------------------- MXFP8
 size_t mx_sf_bytes(int64_t R, int C, int E);
-// `scratch`: 2*(E+1) int32 of device memory; receives tile_pref (prefix of
-// ceil(rows_e/128)) then the prefix of ceil(rows_e/32).  perm_f > 0: SwiGLU weight scale
-// order (see quant_rows_kernel).
+// Row segments of a quantised tensor: the experts' ragged rows (off [E+1] with tile_pref /
+// blk_pref their prefixes of ceil(rows_e/128) and ceil(rows_e/32), from launch_mx_prefix),
+// or, with rows > 0, E uniform segments of `rows` rows (a weight tensor [E*rows, C]).
+struct MxSegs {
+  const int32_t* off = nullptr;
+  const int32_t* tile_pref = nullptr;
+  const int32_t* blk_pref = nullptr;
+  int E = 0;
+  int rows = 0;
+};
+cudaError_t launch_mx_prefix(const int32_t* seg_off, int E, int32_t* tile_pref, int32_t* blk_pref,
+                             cudaStream_t s);
+// x [R, C] bf16 -> rowwise codes/scales (codes_r non-null) and/or colwise ones (codes_c
+// non-null), one read of x.  perm_f > 0: SwiGLU weight order of the rowwise scales.
+cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, int perm_f,
+                            uint8_t* codes_r, uint8_t* sf_r, uint8_t* codes_c, uint8_t* sf_c,
+                            int* status, cudaStream_t s);
+// The C-ABI quantiser: prefix into `scratch` (2*(E+1) int32), then one direction.
 cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
                                bool colwise, uint8_t* codes, uint8_t* sf, int32_t* scratch,
-                               cudaStream_t s, int perm_f = 0);
-cudaError_t launch_uniform_offsets(int32_t* seg_off, int E, int rows, cudaStream_t s);
+                               int* status, cudaStream_t s);
 
 // Device buffers of the MXFP8 grouped GEMMs (codes + 512-byte scale chunks).
 struct MxWork {
   int32_t* act_pref;      // [2(E+1)]: tile prefix (then 32-row prefix) of the experts' rows
-  int32_t* w13_off;       // [E+1] uniform segments of 2*d_ff rows
-  int32_t* w2_off;        // [E+1] uniform segments of d rows
-  int32_t* w_scratch;     // [2(E+1)]
   uint8_t *xr, *xr_sf, *xc, *xc_sf;       // x_perm rowwise / colwise
   uint8_t *ar, *ar_sf, *ac, *ac_sf;       // a
   uint8_t *dyr, *dyr_sf, *dyc, *dyc_sf;   // dy_perm

@@ -56,7 +56,7 @@ WsLayout ws_layout(const moe_desc& d) {
   w.mx_ints = o;
   if (d.dtype == MOE_MXFP8) {
     const size_t E = d.E, f = d.d_ff, dm = d.d;
-    o = up(o + 6 * (E + 1) * 4);
+    o = up(o + 2 * (E + 1) * 4);
     // (rows, cols, segments) of x_perm r/c, a r/c, dy r/c, dH13 r/c, W13 r/c, W2 r/c
     const size_t rows[12] = {R, R, R, R, R, R, R, R, E * 2 * f, E * 2 * f, E * dm, E * dm};
     const size_t cols[12] = {dm, dm, f, f, dm, dm, 2 * f, 2 * f, dm, dm, f, f};
@@ -150,11 +150,7 @@ MxWork mx_work(const moe_desc& d, void* ws) {
   const WsLayout w = ws_layout(d);
   MxWork m;
   int32_t* ints = at<int32_t>(ws, w.mx_ints);
-  const int E1 = d.E + 1;
   m.act_pref = ints;
-  m.w_scratch = ints + 2 * E1;
-  m.w13_off = ints + 4 * E1;
-  m.w2_off = ints + 5 * E1;
   uint8_t* b[24];
   for (int i = 0; i < 24; ++i) b[i] = at<uint8_t>(ws, w.mx_bytes[i]);
   m.xr = b[0]; m.xr_sf = b[1]; m.xc = b[2]; m.xc_sf = b[3];
@@ -385,7 +381,7 @@ moe_status moe_mx_quantize(const void* x, int64_t rows, int32_t cols, const int3
   if (ws_bytes < 256 + 8 * (size_t)(num_segments + 1)) return MOE_EWORKSPACE;
   int32_t* scratch = at<int32_t>(ws, 256);
   return cu(launch_mx_quantize(x, rows, cols, seg_offsets, num_segments, colwise != 0, codes,
-                               scales, scratch, S(stream)));
+                               scales, scratch, status_ptr(ws), S(stream)));
 }
 
 moe_status moe_grouped_gemm_bwd(const moe_desc* desc, const void* dy_perm, const void* x_perm,

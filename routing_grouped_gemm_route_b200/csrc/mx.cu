@@ -27,11 +27,16 @@
 #include <cuda_fp8.h>
 #include <math.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 #include "internal.h"
+#include "sm100.cuh"
 
 namespace moe {
 namespace {
+
+using namespace sm100;
 
 // Shared exponent of a block with max magnitude `amax` (>= 0).
 __device__ __forceinline__ int mx_exponent(float amax) {
@@ -39,21 +44,18 @@ __device__ __forceinline__ int mx_exponent(float amax) {
   int s = ilogbf(amax) - 8;          // floor(log2(amax)) for finite non-zero amax
   return s < -127 ? -127 : (s > 127 ? 127 : s);
 }
-__device__ __forceinline__ uint8_t e4m3(float v) {
-  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+// 2^-s as a float, exactly (2^-127 is the subnormal 0x00400000).  Multiplying by it is
+// the same IEEE operation as scaling the exponent: exact, or one round to nearest even.
+__device__ __forceinline__ float exp2_neg(int s) {
+  return s <= 126 ? __int_as_float((127 - s) << 23) : __int_as_float(0x00400000);
+}
+// Two E4M3 codes (round to nearest even, saturating to +-448) of a and b; a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return static_cast<uint32_t>(
+      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
 __device__ __forceinline__ size_t sf_byte(int64_t chunk, int i, int block) {
   return (size_t)chunk * 512 + 16 * (i & 31) + 4 * ((i & 127) >> 5) + block;
-}
-
-// Segment of row r: the e with seg_off[e] <= r < seg_off[e+1] (skipping empty ones).
-__device__ __forceinline__ int segment_of(const int32_t* seg_off, int E, int r) {
-  int lo = 0, hi = E;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (seg_off[mid] <= r) lo = mid; else hi = mid;
-  }
-  return lo;
 }
 
 // tile_pref[e] = sum_{e'<e} ceil(rows_e'/128); blk_pref[e] = sum_{e'<e} ceil(rows_e'/32).
@@ -72,126 +74,235 @@ __global__ void seg_prefix_kernel(const int32_t* __restrict__ seg_off, int E,
   blk_pref[E] = b;
 }
 
-// Rowwise: one warp per row, lane l handles blocks l, l+32, ... (64 contiguous bytes each).
-// perm_f > 0 (SwiGLU weights [W1; W3], d_ff = perm_f rows each): the scale of row p is
-// filed under the row order gate[0:64], up[0:64], gate[64:128], up[64:128], ..., the order
-// in which a 128-row B tile of the fused SwiGLU GEMM takes 64 gate and 64 up rows.
-__global__ void __launch_bounds__(256) quant_rows_kernel(
-    const __nv_bfloat16* __restrict__ x, int R, int C, const int32_t* __restrict__ seg_off, int E,
-    const int32_t* __restrict__ tile_pref, int perm_f, uint8_t* __restrict__ codes,
-    uint8_t* __restrict__ sf) {
-  const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (r >= R) return;
-  const int e = segment_of(seg_off, E, r);
-  int p = r - seg_off[e];
-  if (perm_f > 0) p = p < perm_f ? (p / 64) * 128 + (p % 64) : ((p - perm_f) / 64) * 128 + 64 + (p - perm_f) % 64;
-  const int64_t group = (int64_t)tile_pref[e] + p / 128;
-  const int nb = C / 32;
-  const __nv_bfloat16* row = x + (int64_t)r * C;
-  for (int b = lane; b < nb; b += 32) {
-    float v[32];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      Vec16<__nv_bfloat16> pk;
-      pk.raw = *reinterpret_cast<const uint4*>(row + b * 32 + j * 8);
-      pk.to_float(v + j * 8);
-    }
-    float amax = 0.f;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
-    const int s = mx_exponent(amax);
-    uint32_t w[8];
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      w[j] = (uint32_t)e4m3(scalbnf(v[4 * j], -s)) | ((uint32_t)e4m3(scalbnf(v[4 * j + 1], -s)) << 8) |
-             ((uint32_t)e4m3(scalbnf(v[4 * j + 2], -s)) << 16) |
-             ((uint32_t)e4m3(scalbnf(v[4 * j + 3], -s)) << 24);
-    }
-    uint4* dst = reinterpret_cast<uint4*>(codes + (int64_t)r * C + b * 32);   // codes stay in x's row order
-    dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-    dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-    const int64_t chunk = group * (C / 128) + (b * 32) / 128;
-    sf[sf_byte(chunk, p, b & 3)] = static_cast<uint8_t>(s + 127);
+// One tile = one 32-row block of a segment (its rows p0 .. p0+nrows-1, starting at row r0
+// of the tensor) x 256 columns.
+struct TilePos {
+  int e, p0, r0, nrows;
+};
+__device__ __forceinline__ bool tile_pos(const MxSegs& g, int blk, TilePos& o) {
+  if (g.rows > 0) {
+    const int per = (g.rows + 31) / 32;
+    const int e = blk / per;
+    if (e >= g.E) return false;
+    o.e = e;
+    o.p0 = (blk - e * per) * 32;
+    o.r0 = e * g.rows + o.p0;
+    o.nrows = min(32, g.rows - o.p0);
+    return true;
   }
-}
-
-// Colwise: one CTA per (32-row block of a segment, 256 columns); thread = column.
-__global__ void __launch_bounds__(256) quant_cols_kernel(
-    const __nv_bfloat16* __restrict__ x, int R, int C, const int32_t* __restrict__ seg_off, int E,
-    const int32_t* __restrict__ tile_pref, const int32_t* __restrict__ blk_pref,
-    uint8_t* __restrict__ codes, uint8_t* __restrict__ sf) {
-  const int blk = blockIdx.y;                 // global 32-row block index over all segments
-  if (blk >= blk_pref[E]) return;
-  int lo = 0, hi = E;                         // segment: blk_pref[lo] <= blk < blk_pref[lo+1]
+  if (blk >= g.blk_pref[g.E]) return false;
+  int lo = 0, hi = g.E;                       // largest e with blk_pref[e] <= blk
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
-    if (blk_pref[mid] <= blk) lo = mid; else hi = mid;
+    if (g.blk_pref[mid] <= blk) lo = mid; else hi = mid;
   }
-  const int e = lo;
-  const int p0 = (blk - blk_pref[e]) * 32;    // first row of the block inside the segment
-  const int r0 = seg_off[e] + p0;
-  const int nrows = min(32, seg_off[e + 1] - r0);
-  const int c = blockIdx.x * 256 + threadIdx.x;
-  if (c >= C) return;
-  float v[32];
-  float amax = 0.f;
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    v[j] = j < nrows ? __bfloat162float(x[(int64_t)(r0 + j) * C + c]) : 0.f;
-    amax = fmaxf(amax, fabsf(v[j]));
-  }
-  const int s = mx_exponent(amax);
-#pragma unroll
-  for (int j = 0; j < 32; ++j)
-    if (j < nrows) codes[(int64_t)(r0 + j) * C + c] = e4m3(scalbnf(v[j], -s));
-  const int64_t chunk = ((int64_t)tile_pref[e] + p0 / 128) * (C / 128) + c / 128;
-  sf[sf_byte(chunk, c, (p0 & 127) >> 5)] = static_cast<uint8_t>(s + 127);
-  // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad GEMM
-  // still reads all four scales (its rows past the segment are zero codes), so the absent
-  // blocks get the finite scale 2^-127 rather than whatever the buffer held (0xFF = NaN).
-  if (p0 + 32 >= seg_off[e + 1] - seg_off[e])
-    for (int b = ((p0 & 127) >> 5) + 1; b < 4; ++b) sf[sf_byte(chunk, c, b)] = 0;
+  o.e = lo;
+  o.p0 = (blk - g.blk_pref[lo]) * 32;
+  o.r0 = g.off[lo] + o.p0;
+  o.nrows = min(32, g.off[lo + 1] - o.r0);
+  return true;
+}
+__device__ __forceinline__ int seg_rows(const MxSegs& g, int e) {
+  return g.rows > 0 ? g.rows : g.off[e + 1] - g.off[e];
+}
+__device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
+  return g.rows > 0 ? (int64_t)e * ((g.rows + 127) / 128) : (int64_t)g.tile_pref[e];
 }
 
-// seg_off[e] = e * rows (uniform segments: one per expert's weight matrix)
-__global__ void uniform_offsets_kernel(int32_t* seg_off, int E, int rows) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
-  if (e <= E) seg_off[e] = e * rows;
+constexpr int kQRows = 32, kQCols = 256;
+constexpr int kQPitch = kQCols * 2 + 16;     // bytes per staged row (16-byte skew: no bank conflicts)
+
+// 32 bf16 of a staged row (64 contiguous bytes) as floats.
+__device__ __forceinline__ void staged32(const uint8_t* p, float* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    Vec16<__nv_bfloat16> pk;
+    pk.raw = *reinterpret_cast<const uint4*>(p + 16 * j);
+    pk.to_float(v + 8 * j);
+  }
+}
+// 32 codes of v[j] * m[j] (PER_ELEM) or v[j] * m[0] -> two 16-byte stores
+template <bool PER_ELEM>
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const float* v, const float* m) {
+  uint32_t w[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int i = 4 * j;
+    const float m0 = m[PER_ELEM ? i : 0], m1 = m[PER_ELEM ? i + 1 : 0];
+    const float m2 = m[PER_ELEM ? i + 2 : 0], m3 = m[PER_ELEM ? i + 3 : 0];
+    w[j] = e4m3x2(v[i] * m0, v[i + 1] * m1) | (e4m3x2(v[i + 2] * m2, v[i + 3] * m3) << 16);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
+
+// Persistent quantiser.  A tile is one 32-row block of a segment x 256 columns; each CTA
+// walks tiles blockIdx.x, +gridDim.x, ... with two shared-memory buffers: while it
+// quantises one tile, the next one's rows stream in by 1-D bulk copies (so the bytes in
+// flight do not depend on registers).  Per tile it writes the rowwise codes/scales (ROW:
+// blocks of 32 along columns) and/or the colwise ones (COL: blocks of 32 along the
+// segment's rows; the tile is exactly one such block per column).
+// perm_f > 0 (SwiGLU weights [W1; W3], d_ff = perm_f rows each): the rowwise scale of
+// row p is filed under the row order gate[0:128], up[0:128], gate[128:256], ..., the
+// order in which a 256-column tile of the fused SwiGLU GEMM takes 128 gate and 128 up
+// rows of B.
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(256, 4) quant_tile_kernel(
+    const __nv_bfloat16* __restrict__ x, int C, const MxSegs g, int perm_f,
+    uint8_t* __restrict__ codes_r, uint8_t* __restrict__ sf_r, uint8_t* __restrict__ codes_c,
+    uint8_t* __restrict__ sf_c, int* status) {
+  __shared__ __align__(128) uint8_t buf[2][kQRows * kQPitch];
+  __shared__ float col_m[kQCols];
+  __shared__ uint64_t bar[2];
+  __shared__ TilePos pos[2];
+  __shared__ int abort_flag;
+  const int t = threadIdx.x;
+  const int ctiles = (C + kQCols - 1) / kQCols;
+  const int nblk = g.rows > 0 ? g.E * ((g.rows + 31) / 32) : g.blk_pref[g.E];
+  const int ntiles = nblk * ctiles;
+  if ((int)blockIdx.x >= ntiles) return;      // uniform over the CTA
+  if (t == 0) {
+    mbar_init(&bar[0], 1);
+    mbar_init(&bar[1], 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // warp 0 loads tile `tile` into buffer `b`: lane 0 arms the barrier with the byte count,
+  // lane r copies row r (the phase cannot complete before lane 0's arrival)
+  auto issue = [&](int tile, int b) {
+    TilePos tp;
+    tile_pos(g, tile / ctiles, tp);
+    const int c0 = (tile % ctiles) * kQCols;
+    const int ncols = min(kQCols, C - c0);
+    if (t == 0) {
+      pos[b] = tp;
+      fence_proxy_async_smem();               // earlier generic reads of buf[b] before the copies
+      mbar_arrive_expect_tx(&bar[b], static_cast<uint32_t>(tp.nrows * ncols * 2));
+    }
+    __syncwarp();
+    if (t < tp.nrows)
+      bulk_load(buf[b] + t * kQPitch, x + (int64_t)(tp.r0 + t) * C + c0,
+                static_cast<uint32_t>(ncols * 2), &bar[b]);
+  };
+  if (t < 32) issue(blockIdx.x, 0);
+  const int W = C / 128;
+  const int row = t & 31, q = t >> 5;         // this thread's row and 32-column block
+  int it = 0;
+  bool next_issued = false;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
+    const int b = it & 1;
+    const int next = tile + gridDim.x;
+    next_issued = next < ntiles;
+    if (t < 32 && next_issued) issue(next, b ^ 1);   // buf[b^1] was released by the last barrier
+    const bool ok = mbar_wait(&bar[b], (it >> 1) & 1u, reinterpret_cast<volatile int*>(&abort_flag), status);
+    if (__syncthreads_or(!ok)) break;
+    const TilePos tp = pos[b];
+    const int c0 = (tile % ctiles) * kQCols;
+    const int ncols = min(kQCols, C - c0);
+    const int64_t tile0 = seg_tile0(g, tp.e);
+    const uint8_t* tb = buf[b];
+    const bool active = row < tp.nrows && q * 32 < ncols;
+    float v[32];
+    if (active) staged32(tb + row * kQPitch + q * 64, v);
+    if (ROW && active) {
+      float amax = 0.f;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+      const int s = mx_exponent(amax);
+      const float m = exp2_neg(s);
+      store_codes32<false>(codes_r + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, &m);
+      int p = tp.p0 + row;
+      if (perm_f > 0)
+        p = p < perm_f ? (p / 128) * 256 + (p % 128)
+                       : ((p - perm_f) / 128) * 256 + 128 + (p - perm_f) % 128;
+      const int col = c0 + q * 32;
+      sf_r[sf_byte((tile0 + p / 128) * W + col / 128, p, (col & 127) >> 5)] =
+          static_cast<uint8_t>(s + 127);
+    }
+    if (COL) {
+      if (t < ncols) {
+        float amax = 0.f;
+        for (int r = 0; r < tp.nrows; ++r) {  // rows past the segment's end take no part
+          const __nv_bfloat16 h = *reinterpret_cast<const __nv_bfloat16*>(tb + r * kQPitch + 2 * t);
+          amax = fmaxf(amax, fabsf(__bfloat162float(h)));
+        }
+        const int s = mx_exponent(amax);
+        col_m[t] = exp2_neg(s);
+        const int col = c0 + t;
+        const int64_t chunk = (tile0 + tp.p0 / 128) * W + col / 128;
+        const int blk = (tp.p0 & 127) >> 5;
+        sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
+        // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad
+        // GEMM still reads all four scales (its rows past the segment are zero codes), so
+        // the absent blocks get the finite scale 2^-127 rather than whatever the buffer
+        // held (0xFF = NaN).
+        if (tp.p0 + 32 >= seg_rows(g, tp.e))
+          for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
+      }
+      __syncthreads();
+      if (active)
+        store_codes32<true>(codes_c + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, col_m + q * 32);
+    }
+    __syncthreads();   // buf[b] and col_m free for reuse
+  }
+  // After an abort, the copies still in flight must land before the CTA exits.
+  if (t == 0 && abort_flag) {
+    mbar_wait_teardown(&bar[it & 1], (it >> 1) & 1u);
+    if (next_issued) mbar_wait_teardown(&bar[(it + 1) & 1], ((it + 1) >> 1) & 1u);
+  }
 }
 
 }  // namespace
-
-cudaError_t launch_uniform_offsets(int32_t* seg_off, int E, int rows, cudaStream_t s) {
-  uniform_offsets_kernel<<<(E + 1 + 255) / 256, 256, 0, s>>>(seg_off, E, rows);
-  return cudaGetLastError();
-}
 
 size_t mx_sf_bytes(int64_t R, int C, int E) {
   // chunks: (sum_e ceil(rows_e/128)) * (C/128) <= (R/128 + E) * (C/128)
   return (size_t)((R + 127) / 128 + E) * (size_t)(C / 128) * 512;
 }
 
+cudaError_t launch_mx_prefix(const int32_t* seg_off, int E, int32_t* tile_pref, int32_t* blk_pref,
+                             cudaStream_t s) {
+  seg_prefix_kernel<<<1, 32, 0, s>>>(seg_off, E, tile_pref, blk_pref);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, int perm_f,
+                            uint8_t* codes_r, uint8_t* sf_r, uint8_t* codes_c, uint8_t* sf_c,
+                            int* status, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  // tiles: sum_e ceil(rows_e/32) <= R/32 + E row blocks, times the column tiles
+  const int64_t blocks = g.rows > 0 ? (int64_t)g.E * ((g.rows + 31) / 32) : (R + 31) / 32 + g.E;
+  const int64_t tiles = blocks * ((C + kQCols - 1) / kQCols);
+  if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const int64_t grid = std::min<int64_t>(tiles, (int64_t)num_sms() * 4);
+  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
+  const bool row = codes_r != nullptr, col = codes_c != nullptr;
+  if (row && col)
+    quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, perm_f, codes_r, sf_r,
+                                                                 codes_c, sf_c, status);
+  else if (row)
+    quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, perm_f, codes_r, sf_r,
+                                                                  nullptr, nullptr, status);
+  else if (col)
+    quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, 0, nullptr, nullptr,
+                                                                  codes_c, sf_c, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
                                bool colwise, uint8_t* codes, uint8_t* sf, int32_t* scratch,
-                               cudaStream_t s, int perm_f) {
+                               int* status, cudaStream_t s) {
   if (R == 0) return cudaSuccess;
-  int32_t* tile_pref = scratch;               // [E+1]
-  int32_t* blk_pref = scratch + (E + 1);      // [E+1]
-  seg_prefix_kernel<<<1, 32, 0, s>>>(seg_off, E, tile_pref, blk_pref);
-  cudaError_t err = cudaGetLastError();
+  MxSegs g;
+  g.off = seg_off;
+  g.tile_pref = scratch;               // [E+1]
+  g.blk_pref = scratch + (E + 1);      // [E+1]
+  g.E = E;
+  cudaError_t err = launch_mx_prefix(seg_off, E, scratch, scratch + (E + 1), s);
   if (err != cudaSuccess) return err;
-  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  if (!colwise) {
-    quant_rows_kernel<<<(unsigned)((R + 7) / 8), 256, 0, s>>>(xb, (int)R, C, seg_off, E, tile_pref,
-                                                            perm_f, codes, sf);
-  } else {
-    // one CTA row per possible 32-row block: sum_e ceil(rows_e/32) <= R/32 + E
-    dim3 grid((C + 255) / 256, (unsigned)((R + 31) / 32 + E));
-    quant_cols_kernel<<<grid, 256, 0, s>>>(xb, (int)R, C, seg_off, E, tile_pref, blk_pref, codes,
-                                           sf);
-  }
-  return cudaGetLastError();
+  return colwise ? launch_mx_quant(x, R, C, g, 0, nullptr, nullptr, codes, sf, status, s)
+                 : launch_mx_quant(x, R, C, g, 0, codes, sf, nullptr, nullptr, status, s);
 }
 
 }  // namespace moe
