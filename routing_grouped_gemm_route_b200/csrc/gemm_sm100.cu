@@ -111,9 +111,11 @@ struct Cfg {
   // other), except for MXFP8 256-column tiles, where the scale columns leave room for one
   static constexpr int NACC = MX && BN == 256 ? 1 : 2;
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
-  // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there);
-  // elsewhere 4 warps keep up and leave more shared memory to the operand ring
-  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD ? 8 : 4;
+  // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there)
+  // and for single-accumulator tiles (the MMAs wait for the whole epilogue, so it is
+  // split over two warps per lane quadrant); elsewhere 4 warps keep up and leave more
+  // shared memory to the operand ring
+  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD || NACC == 1 ? 8 : 4;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int COLGRP = EPI_WARPS / 4;          // warps sharing one lane quadrant
   static constexpr int NCH = BN / 32;                   // 32-column chunks per tile
@@ -564,7 +566,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         if (nvalid > 0) {
           if (EPI == EPI_STORE) {
 #pragma unroll 1
-            for (int c = 0; c < BN; c += 32) {
+            for (int c = cfirst * 32; c < (cfirst + C::WCH) * 32; c += 32) {
               tmem_ld32(tb + c, v);
               tmem_ld_wait();
               reg_fence32(v);
@@ -581,8 +583,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             const int h0 = tl.n0 / 2;
             uint32_t v3[32];
             float h3[32], av[32];
+            constexpr int HW = BN / 2 / C::COLGRP;   // gate (and up) columns of this warp
 #pragma unroll 1
-            for (int c = 0; c < BN / 2; c += 32) {
+            for (int c = cg * HW; c < (cg + 1) * HW; c += 32) {
               tmem_ld32(tb + c, v);
               tmem_ld32(tb + BN / 2 + c, v3);
               tmem_ld_wait();

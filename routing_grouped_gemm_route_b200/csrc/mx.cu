@@ -111,35 +111,55 @@ __device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
 
 constexpr int kQRows = 32, kQCols = 256;
 constexpr int kQPitch = kQCols * 2 + 16;     // bytes per staged row (16-byte skew: no bank conflicts)
+constexpr int kQBufs = 2;                    // tiles in flight per CTA (one being quantised)
+constexpr int kQBufBytes = kQRows * kQPitch;
+constexpr size_t kQSmem = 128 + (size_t)kQBufs * kQBufBytes;
 
-// 32 bf16 of a staged row (64 contiguous bytes) as floats.
-__device__ __forceinline__ void staged32(const uint8_t* p, float* v) {
+// 32 bf16 of a staged row (64 contiguous bytes), kept packed: w[i] holds elements
+// 2i (low half) and 2i+1 (high half).
+__device__ __forceinline__ void staged32(const uint8_t* p, uint32_t* w) {
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    Vec16<__nv_bfloat16> pk;
-    pk.raw = *reinterpret_cast<const uint4*>(p + 16 * j);
-    pk.to_float(v + 8 * j);
+    const uint4 u = *reinterpret_cast<const uint4*>(p + 16 * j);
+    w[4 * j] = u.x;
+    w[4 * j + 1] = u.y;
+    w[4 * j + 2] = u.z;
+    w[4 * j + 3] = u.w;
   }
 }
-// 32 codes of v[j] * m[j] (PER_ELEM) or v[j] * m[0] -> two 16-byte stores
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+// max |x| over packed bf16 pairs, pairwise (exact: the result is one of the inputs)
+__device__ __forceinline__ __nv_bfloat162 absmax2(__nv_bfloat162 m, uint32_t w) {
+  return __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
+}
+__device__ __forceinline__ float amax32(const uint32_t* w) {
+  __nv_bfloat162 m = __float2bfloat162_rn(0.f);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) m = absmax2(m, w[i]);
+  return fmaxf(__low2float(m), __high2float(m));
+}
+
+// 32 codes of the packed bf16 w[] times m[j] (PER_ELEM) or m[0] -> two 16-byte stores
 template <bool PER_ELEM>
-__device__ __forceinline__ void store_codes32(uint8_t* dst, const float* v, const float* m) {
-  uint32_t w[8];
+__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* w, const float* m) {
+  uint32_t o[8];
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int i = 4 * j;
     const float m0 = m[PER_ELEM ? i : 0], m1 = m[PER_ELEM ? i + 1 : 0];
     const float m2 = m[PER_ELEM ? i + 2 : 0], m3 = m[PER_ELEM ? i + 3 : 0];
-    w[j] = e4m3x2(v[i] * m0, v[i + 1] * m1) | (e4m3x2(v[i + 2] * m2, v[i + 3] * m3) << 16);
+    o[j] = e4m3x2(bf_lo(w[2 * j]) * m0, bf_hi(w[2 * j]) * m1) |
+           (e4m3x2(bf_lo(w[2 * j + 1]) * m2, bf_hi(w[2 * j + 1]) * m3) << 16);
   }
   uint4* d = reinterpret_cast<uint4*>(dst);
-  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
-  d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+  d[0] = make_uint4(o[0], o[1], o[2], o[3]);
+  d[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
 // Persistent quantiser.  A tile is one 32-row block of a segment x 256 columns; each CTA
-// walks tiles blockIdx.x, +gridDim.x, ... with two shared-memory buffers: while it
-// quantises one tile, the next one's rows stream in by 1-D bulk copies (so the bytes in
+// walks tiles blockIdx.x, +gridDim.x, ... with kQBufs shared-memory buffers: while it
+// quantises one tile, the next ones' rows stream in by 1-D bulk copies (so the bytes in
 // flight do not depend on registers).  Per tile it writes the rowwise codes/scales (ROW:
 // blocks of 32 along columns) and/or the colwise ones (COL: blocks of 32 along the
 // segment's rows; the tile is exactly one such block per column).
@@ -152,10 +172,12 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
     const __nv_bfloat16* __restrict__ x, int C, const MxSegs g, int perm_f,
     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ sf_r, uint8_t* __restrict__ codes_c,
     uint8_t* __restrict__ sf_c, int* status) {
-  __shared__ __align__(128) uint8_t buf[2][kQRows * kQPitch];
+  extern __shared__ uint8_t q_smem_raw[];
+  uint8_t* bufs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q_smem_raw) + 127) &
+                                             ~uintptr_t(127));
   __shared__ float col_m[kQCols];
-  __shared__ uint64_t bar[2];
-  __shared__ TilePos pos[2];
+  __shared__ uint64_t bar[kQBufs];
+  __shared__ TilePos pos[kQBufs];
   __shared__ int abort_flag;
   const int t = threadIdx.x;
   const int ctiles = (C + kQCols - 1) / kQCols;
@@ -163,8 +185,7 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
   const int ntiles = nblk * ctiles;
   if ((int)blockIdx.x >= ntiles) return;      // uniform over the CTA
   if (t == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int i = 0; i < kQBufs; ++i) mbar_init(&bar[i], 1);
     abort_flag = 0;
     fence_mbar_init();
   }
@@ -183,34 +204,35 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
     }
     __syncwarp();
     if (t < tp.nrows)
-      bulk_load(buf[b] + t * kQPitch, x + (int64_t)(tp.r0 + t) * C + c0,
+      bulk_load(bufs + b * kQBufBytes + t * kQPitch, x + (int64_t)(tp.r0 + t) * C + c0,
                 static_cast<uint32_t>(ncols * 2), &bar[b]);
   };
-  if (t < 32) issue(blockIdx.x, 0);
+  // prologue: the first kQBufs-1 tiles
+  for (int i = 0; i < kQBufs - 1; ++i) {
+    const int tile = blockIdx.x + i * gridDim.x;
+    if (t < 32 && tile < ntiles) issue(tile, i);
+  }
   const int W = C / 128;
   const int row = t & 31, q = t >> 5;         // this thread's row and 32-column block
   int it = 0;
-  bool next_issued = false;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int b = it & 1;
-    const int next = tile + gridDim.x;
-    next_issued = next < ntiles;
-    if (t < 32 && next_issued) issue(next, b ^ 1);   // buf[b^1] was released by the last barrier
-    const bool ok = mbar_wait(&bar[b], (it >> 1) & 1u, reinterpret_cast<volatile int*>(&abort_flag), status);
+    const int b = it % kQBufs;
+    // the buffer of iteration it-1 was released by the barrier that ended it
+    const int ahead = tile + (kQBufs - 1) * gridDim.x;
+    if (t < 32 && ahead < ntiles) issue(ahead, (it + kQBufs - 1) % kQBufs);
+    const bool ok = mbar_wait(&bar[b], (it / kQBufs) & 1u,
+                              reinterpret_cast<volatile int*>(&abort_flag), status);
     if (__syncthreads_or(!ok)) break;
     const TilePos tp = pos[b];
     const int c0 = (tile % ctiles) * kQCols;
     const int ncols = min(kQCols, C - c0);
     const int64_t tile0 = seg_tile0(g, tp.e);
-    const uint8_t* tb = buf[b];
+    const uint8_t* tb = bufs + b * kQBufBytes;
     const bool active = row < tp.nrows && q * 32 < ncols;
-    float v[32];
+    uint32_t v[16];
     if (active) staged32(tb + row * kQPitch + q * 64, v);
     if (ROW && active) {
-      float amax = 0.f;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      const int s = mx_exponent(amax);
+      const int s = mx_exponent(amax32(v));
       const float m = exp2_neg(s);
       store_codes32<false>(codes_r + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, &m);
       int p = tp.p0 + row;
@@ -222,35 +244,44 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
           static_cast<uint8_t>(s + 127);
     }
     if (COL) {
-      if (t < ncols) {
-        float amax = 0.f;
-        for (int r = 0; r < tp.nrows; ++r) {  // rows past the segment's end take no part
-          const __nv_bfloat16 h = *reinterpret_cast<const __nv_bfloat16*>(tb + r * kQPitch + 2 * t);
-          amax = fmaxf(amax, fabsf(__bfloat162float(h)));
+      if (2 * t < ncols) {
+        // columns 2t and 2t+1; rows past the segment's end take no part (they hold
+        // whatever the buffer had: masked out)
+        __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
+#pragma unroll
+        for (int r = 0; r < kQRows; ++r) {
+          const uint32_t w = *reinterpret_cast<const uint32_t*>(tb + r * kQPitch + 4 * t);
+          m2 = absmax2(m2, r < tp.nrows ? w : 0u);
         }
-        const int s = mx_exponent(amax);
-        col_m[t] = exp2_neg(s);
-        const int col = c0 + t;
-        const int64_t chunk = (tile0 + tp.p0 / 128) * W + col / 128;
+        const int64_t chunk = (tile0 + tp.p0 / 128) * W + (c0 + 2 * t) / 128;
         const int blk = (tp.p0 & 127) >> 5;
-        sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
-        // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad
-        // GEMM still reads all four scales (its rows past the segment are zero codes), so
-        // the absent blocks get the finite scale 2^-127 rather than whatever the buffer
-        // held (0xFF = NaN).
-        if (tp.p0 + 32 >= seg_rows(g, tp.e))
-          for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
+        const bool last = tp.p0 + 32 >= seg_rows(g, tp.e);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int s = mx_exponent(h ? __high2float(m2) : __low2float(m2));
+          const int col = c0 + 2 * t + h;
+          col_m[2 * t + h] = exp2_neg(s);
+          sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
+          // The segment's last chunk may hold fewer than four blocks.  A K-stage of a
+          // wgrad GEMM still reads all four scales (its rows past the segment are zero
+          // codes), so the absent blocks get the finite scale 2^-127 rather than whatever
+          // the buffer held (0xFF = NaN).
+          if (last)
+            for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
+        }
       }
       __syncthreads();
       if (active)
         store_codes32<true>(codes_c + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, col_m + q * 32);
     }
-    __syncthreads();   // buf[b] and col_m free for reuse
+    __syncthreads();   // this buffer and col_m free for reuse
   }
-  // After an abort, the copies still in flight must land before the CTA exits.
+  // After an abort, the copies still in flight (iterations it .. it+kQBufs-1 that have a
+  // tile) must land before the CTA exits.
   if (t == 0 && abort_flag) {
-    mbar_wait_teardown(&bar[it & 1], (it >> 1) & 1u);
-    if (next_issued) mbar_wait_teardown(&bar[(it + 1) & 1], ((it + 1) >> 1) & 1u);
+    for (int j = it; j < it + kQBufs; ++j)
+      if (blockIdx.x + j * gridDim.x < ntiles)
+        mbar_wait_teardown(&bar[j % kQBufs], (j / kQBufs) & 1u);
   }
 }
 
@@ -278,15 +309,15 @@ cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, in
   const int64_t grid = std::min<int64_t>(tiles, (int64_t)num_sms() * 4);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   const bool row = codes_r != nullptr, col = codes_c != nullptr;
-  if (row && col)
-    quant_tile_kernel<true, true><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, perm_f, codes_r, sf_r,
-                                                                 codes_c, sf_c, status);
-  else if (row)
-    quant_tile_kernel<true, false><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, perm_f, codes_r, sf_r,
-                                                                  nullptr, nullptr, status);
-  else if (col)
-    quant_tile_kernel<false, true><<<(unsigned)grid, 256, 0, s>>>(xb, C, g, 0, nullptr, nullptr,
-                                                                  codes_c, sf_c, status);
+  auto kern = row && col ? quant_tile_kernel<true, true>
+              : row      ? quant_tile_kernel<true, false>
+                         : quant_tile_kernel<false, true>;
+  if (!row && !col) return cudaSuccess;
+  cudaError_t err =
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQSmem);
+  if (err != cudaSuccess) return err;
+  kern<<<(unsigned)grid, 256, kQSmem, s>>>(xb, C, g, row ? perm_f : 0, codes_r, sf_r, codes_c,
+                                           sf_c, status);
   return cudaGetLastError();
 }
 
