@@ -43,6 +43,8 @@ def parse():
     ap.add_argument("--workload", default="e128_bf16")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--router", action="store_true", help="compute logits = x.Wr on the device")
+    ap.add_argument("--recompute", action="store_true",
+                    help="activation recompute: the backward redoes dispatch, FC1 and FC2")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-steps", type=int, default=30, help="0 skips the end-to-end leg")
@@ -331,7 +333,8 @@ def main():
     lib.load()
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_inputs(w, device=dev, seed=w.seed + rank)
-    flags = lib.MOE_FLAG_ROUTER if w.router else 0
+    flags = (lib.MOE_FLAG_ROUTER if w.router else 0) | \
+        (lib.MOE_FLAG_RECOMPUTE if args.recompute else 0)
     desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
     act = lib.act_dtype(desc)
     T, d, f, E, k = w.T, w.d, w.d_ff, w.E, w.k
@@ -355,6 +358,9 @@ def main():
 
     stages = ["route", "dispatch", "gemm_fwd", "combine", "combine_bwd", "gemm_bwd",
               "dispatch_bwd"]
+    if args.recompute:
+        # the backward first recomputes the forward's activations (same buffers here)
+        stages = stages[:4] + ["re_dispatch", "re_gemm_fwd"] + stages[4:]
     if w.router:
         stages = ["router"] + stages + ["router_bwd"]
     mx = w.dtype == "mxfp8"
@@ -363,15 +369,16 @@ def main():
     launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 7 if mx else 2,
                 "combine": 1, "combine_bwd": 1, "gemm_bwd": 12 if mx else 5, "dispatch_bwd": 1,
                 "router_bwd": 3}
+    launches["re_dispatch"], launches["re_gemm_fwd"] = launches["dispatch"], launches["gemm_fwd"]
 
     def run_stage(name):
         if name == "router":
             lib.moe_router_logits(desc, x, Wr, logits)
         elif name == "route":
             lib.moe_route(desc, logits, idx, gates, counts, offsets, slot, row_token, row_gate, ws)
-        elif name == "dispatch":
+        elif name in ("dispatch", "re_dispatch"):
             lib.moe_dispatch(desc, x, slot, x_perm, ws)
-        elif name == "gemm_fwd":
+        elif name in ("gemm_fwd", "re_gemm_fwd"):
             lib.moe_grouped_gemm_fwd(desc, x_perm, W13, W2, offsets, H13, a, y_perm, ws)
         elif name == "combine":
             lib.moe_combine(desc, y_perm, gates, slot, y, ws)
@@ -415,6 +422,13 @@ def main():
     ms_total = max_over_ranks(ms_local, world)
     if lib.moe_read_device_status(ws) != 0:
         raise RuntimeError("device status set during the timed region")
+    # expert load of this routing (device statistics kernel, outside the timed region)
+    st_buf = torch.zeros(64, dtype=torch.uint8, device=dev)
+    lib.moe_load_stats(counts, st_buf)
+    load = lib.decode_load_stats(st_buf)
+    load = {"max_over_mean": round(load["max_over_mean"], 3), "cv": round(load["cv"], 4),
+            "empty_experts": load["num_empty"], "max_rows": load["max_count"],
+            "min_rows": load["min_count"]}
 
     stage_ms = {s: sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(K)) / K
                 for j, s in enumerate(stages)}
@@ -422,7 +436,8 @@ def main():
     pk = peaks()
 
     # algorithmic work per stage
-    gemm_flops = {"gemm_fwd": 6.0 * R * d * f, "gemm_bwd": 12.0 * R * d * f}
+    gemm_flops = {"gemm_fwd": 6.0 * R * d * f, "gemm_bwd": 12.0 * R * d * f,
+                  "re_gemm_fwd": 6.0 * R * d * f}
     hbm_bytes = {
         "route": T * E * 4 + T * k * 12 + R * 8 + 2 * 4 * ((T + 255) // 256) * E,
         "dispatch": T * d * es + T * k * 4 + R * d * es,
@@ -430,6 +445,7 @@ def main():
         "combine_bwd": T * d * es + 2 * R * d * es + T * k * 12 + T * E * 4,
         "dispatch_bwd": R * d * es + T * k * 4 + T * d * es,
     }
+    hbm_bytes["re_dispatch"] = hbm_bytes["dispatch"]
     stage_rep = {}
     for s, ms in stage_ms.items():
         r = {"ms": round(ms, 4)}
@@ -489,7 +505,8 @@ def main():
             "vs_baseline": None, "dtype": ("mxfp8-e4m3" if mx else "bf16") if act == torch.bfloat16 else "f32",
             "data": "synthetic (seeded N(0,1) activations/logits, N(0,0.02) weights)",
             "config": {"workload": workload_desc(w), "T": T, "d_model": d, "E": E, "top_k": k,
-                       "d_ff": f, "router_on_device": w.router,
+                       "d_ff": f, "router_on_device": w.router, "recompute": args.recompute,
+                       "expert_load": load,
                        "parallelism": f"replicas x{world} (data parallel, no data-path collective)",
                        "l2": "no flush: each step's working set (~5 GB of weights, activations "
                              "and grads) exceeds the 126 MB L2"},

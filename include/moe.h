@@ -70,6 +70,12 @@ typedef enum moe_dtype {
 #define MOE_FLAG_ROUTER   1  /* logits = x . Wr computed on the device (else injected) */
 #define MOE_FLAG_DW_FP32  2  /* dW13 / dW2 are float (else act type) */
 #define MOE_FLAG_ACCUM_DW 4  /* add into existing float dW (requires MOE_FLAG_DW_FP32) */
+/* Activation recompute (deniz.in, "Açık ödünleşimler": recompute drops most activation
+ * memory for part of the throughput).  moe_layer_fwd keeps only the routing metadata
+ * in `saved` (x_perm, H13, a, y_perm become workspace scratch), and moe_layer_bwd
+ * recomputes dispatch, FC1 + SwiGLU and FC2 from x (then required) before the backward.
+ * The results are bit-identical to the run without the flag. */
+#define MOE_FLAG_RECOMPUTE 8
 
 /* device status bits */
 #define MOE_DEV_BAD_INDEX   1  /* an expert index or slot was out of range; the row was skipped */
@@ -93,6 +99,8 @@ typedef struct moe_saved_layout {
   size_t row_token;  /* int32 [R] */
   size_t row_gate;   /* float [R] */
   size_t logits;     /* float [T,E] (router on only; else equal to `x_perm`, unused) */
+  /* the four activations below are absent (zero bytes, offsets equal to `total`) with
+   * MOE_FLAG_RECOMPUTE */
   size_t x_perm;     /* act [R,d] */
   size_t H13;        /* act [R,2*d_ff] */
   size_t a;          /* act [R,d_ff] */
@@ -255,6 +263,25 @@ moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
                           const float* d_logits, void* dx, void* dWr, void* ws,
                           size_t ws_bytes, void* stream);
 
+/* Expert load statistics of one routing (deniz.in, "Ekibin reddettiği yaklaşımlar": the
+ * experts' imbalance can grow while a balancing loss improves, "Token Gerrymandering";
+ * this is its measurable side -- the pages give no loss formula and none is computed).
+ * From counts [E] (device, e.g. the `counts` of moe_route or of `saved`):
+ *   total = sum_e counts[e], mean = total / E, max_count, min_count,
+ *   num_empty = #{e : counts[e] == 0}, max_over_mean = max_count / mean (0 if total = 0),
+ *   cv = sqrt(sum_e (counts[e] - mean)^2 / E) / mean (0 if total = 0),
+ * written to *out, a device pointer (16-byte aligned), by one small kernel on `stream`
+ * -- no host synchronisation; copy it back when needed.  Counts must be >= 0 (a
+ * negative count sets MOE_DEV_BAD_OFFSETS in the status word `status`, if non-null, and
+ * is read as 0).  E in [1, 1024]. */
+typedef struct moe_load_stats_t {
+  int64_t total;
+  int32_t max_count, min_count, num_empty, num_experts;
+  double mean, max_over_mean, cv;
+} moe_load_stats_t;
+moe_status moe_load_stats(const int32_t* counts, int32_t E, moe_load_stats_t* out,
+                          int32_t* status, void* stream);
+
 /* Whole layer forward: [router] -> route -> dispatch -> grouped GEMM fwd -> combine.
  * logits: injected routing logits [T,E] float, or NULL with MOE_FLAG_ROUTER and Wr.
  * y [T,d] act.  `saved` (moe_saved_layout.total bytes) receives the tensors listed in
@@ -266,7 +293,8 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
 
 /* Whole layer backward for upstream gradient dy [T,d] act.  Out: dx [T,d] act,
  * d_logits [T,E] float, dW13, dW2 (see moe_grouped_gemm_bwd), and dWr [d,E] act when
- * MOE_FLAG_ROUTER (x and Wr required then; x may be NULL otherwise). */
+ * MOE_FLAG_ROUTER.  x (the forward's input) is required with MOE_FLAG_ROUTER or
+ * MOE_FLAG_RECOMPUTE and may be NULL otherwise. */
 moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x,
                          const void* saved, size_t saved_bytes, const void* W13,
                          const void* W2, const void* Wr, void* dx, float* d_logits,

@@ -308,6 +308,23 @@ def layer_bwd(fwd: dict, dy, x, W13, W2, Wr=None, mx: bool = False) -> dict:
     return out
 
 
+def load_stats(counts) -> dict:
+    """Expert load statistics of one routing: the measurable side of the imbalance the
+    write-ups call "Token Gerrymandering" (deniz.in, "Ekibin reddettiği yaklaşımlar"; they
+    give no formula, so these are the plain definitions).  counts [E] >= 0."""
+    c = np.asarray(counts, dtype=np.int64)
+    E = len(c)
+    total = int(c.sum())
+    mean = total / E
+    out = dict(total=total, max_count=int(c.max()), min_count=int(c.min()),
+               num_empty=int((c == 0).sum()), num_experts=E, mean=mean,
+               max_over_mean=0.0, cv=0.0)
+    if total > 0:
+        out["max_over_mean"] = float(c.max()) / mean
+        out["cv"] = float(np.sqrt(np.mean((c.astype(np.float64) - mean) ** 2))) / mean
+    return out
+
+
 def rel_fro(a, b) -> float:
     """Relative Frobenius error ||a - b|| / ||b||  (0 when both are zero)."""
     a = _f64(a)

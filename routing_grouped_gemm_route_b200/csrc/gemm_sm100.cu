@@ -302,7 +302,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   const int unit = PAIR ? static_cast<int>(blockIdx.x >> 1) : static_cast<int>(blockIdx.x);
   const int n_units = PAIR ? static_cast<int>(gridDim.x >> 1) : static_cast<int>(gridDim.x);
 
-  for (int i = threadIdx.x; i <= E; i += C::THREADS) s_off[i] = p.offsets[i];
+  // no offsets: one segment of all R rows (the router GEMMs)
+  for (int i = threadIdx.x; i <= E; i += C::THREADS)
+    s_off[i] = p.offsets ? p.offsets[i] : (i == 0 ? 0 : p.R);
   __syncthreads();
 
   if (warp == 0) {
@@ -719,7 +721,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
 // needs at least one row; an expert with no rows never loads through its map.)
 __global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
                                    const __grid_constant__ CUtensorMap tmpl1,
-                                   const int32_t* __restrict__ offsets, int E,
+                                   const int32_t* __restrict__ offsets, int E, int R,
                                    CUtensorMap* maps) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 2 * E) return;
@@ -728,7 +730,7 @@ __global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
   uint4* dst = reinterpret_cast<uint4*>(maps + i);
 #pragma unroll
   for (int j = 0; j < 8; ++j) dst[j] = src[j];
-  const int rows = offsets[e + 1];
+  const int rows = offsets ? offsets[e + 1] : R;   // no offsets: one segment of R rows
   tmap_replace_outer_dim(maps + i, static_cast<uint32_t>(rows > 0 ? rows : 1));
   fence_tmap_release();
 }
@@ -1049,7 +1051,7 @@ static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, cons
   if (!make_tmap(&t1, dH13, ES, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
     return MOE_ECUDA;
   const int threads = 2 * g.E;
-  expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, maps);
+  expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, g.R, maps);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
@@ -1202,6 +1204,57 @@ static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_
   return mx_wgrad<OutT>(g, w.dhc, 2 * f, w.xc, d, dW13, accum, off, maps + E, st, s, m4);
 }
 
+// ------------------------------------------------------------------------ router GEMMs
+// The router projection and its two backward products as one-segment GEMMs (no offsets:
+// all T rows form the single segment), bf16 operands, fp32 accumulation.  E % 64 == 0.
+static int bn_of(int n) { return n % 256 == 0 ? 256 : n % 128 == 0 ? 128 : 64; }
+
+static moe_status router_logits_tc(int T, int d, int E, const void* x, const void* Wr,
+                                   float* logits, int* st, cudaStream_t s) {
+  const GemmShape g{1, T, d, 0, false, false};
+  // logits[T,E] = x[T,d] . Wr[d,E]: B = Wr read M/N-major ([K=d rows, N=E cols])
+  switch (bn_of(E)) {
+    case 256:
+      return run_m<bf16, true, EPI_STORE, 256, true, float>(g, x, d, Wr, E, d, E, logits, E,
+                                                           nullptr, nullptr, nullptr, st, s);
+    case 128:
+      return run_m<bf16, true, EPI_STORE, 128, true, float>(g, x, d, Wr, E, d, E, logits, E,
+                                                           nullptr, nullptr, nullptr, st, s);
+    default:
+      return run_m<bf16, true, EPI_STORE, 64, false, float>(g, x, d, Wr, E, d, E, logits, E,
+                                                           nullptr, nullptr, nullptr, st, s);
+  }
+}
+
+static moe_status router_dx_tc(int T, int d, int E, const void* dl16, const void* Wr,
+                               float* dx_extra, int* st, cudaStream_t s) {
+  const GemmShape g{1, T, d, 0, false, false};
+  // dx_extra[T,d] = d_logits[T,E] . Wr^T: B = Wr read K-major ([N=d rows, K=E cols])
+  if (d % 256 == 0)
+    return run_m<bf16, false, EPI_STORE, 256, true, float>(g, dl16, E, Wr, d, d, E, dx_extra, d,
+                                                          nullptr, nullptr, nullptr, st, s);
+  return run_m<bf16, false, EPI_STORE, 128, true, float>(g, dl16, E, Wr, d, d, E, dx_extra, d,
+                                                        nullptr, nullptr, nullptr, st, s);
+}
+
+static moe_status router_dwr_tc(int T, int d, int E, const void* x, const void* dl16, void* dWr,
+                                CUtensorMap* maps, int* st, cudaStream_t s) {
+  const GemmShape g{1, T, d, 0, false, false};
+  // dWr[d,E] = x^T . d_logits: a ragged-K GEMM over the one segment (K = T)
+  using C = Cfg<bf16, bf16, 128, EPI_STORE>;
+  CUtensorMap t0;
+  if (!make_tmap(&t0, x, 2, d, T, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  expert_maps_kernel<<<1, 128, 0, s>>>(t0, t0, nullptr, 1, T, maps);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ECUDA;
+  const int bn = bn_of(E);
+  if (d % 256 == 0 && bn >= 128) {
+    if (bn == 256) return run_k<bf16, bf16, 256, true>(g, x, d, dl16, E, dWr, false, nullptr, maps, st, s);
+    return run_k<bf16, bf16, 128, true>(g, x, d, dl16, E, dWr, false, nullptr, maps, st, s);
+  }
+  MOE_DISPATCH_BN(bn, (run_k<bf16, bf16, BN, false>(g, x, d, dl16, E, dWr, false, nullptr, maps,
+                                                     st, s)));
+}
+
 }  // namespace gemm
 
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
@@ -1260,6 +1313,18 @@ moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm,
                              dW2, dw_fp32, dw_accum, maps_ws, status, s);
   return gemm_bwd_t<__nv_bfloat16>(g, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm,
                                    dW13, dW2, dw_fp32, dw_accum, maps_ws, status, s);
+}
+
+moe_status router_logits_tc(int T, int d, int E, const void* x, const void* Wr, float* logits,
+                            int* status, cudaStream_t s) {
+  return gemm::router_logits_tc(T, d, E, x, Wr, logits, status, s);
+}
+moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, const void* dl16,
+                         float* dx_extra, void* dWr, void* maps_ws, int* status, cudaStream_t s) {
+  moe_status r = gemm::router_dx_tc(T, d, E, dl16, Wr, dx_extra, status, s);
+  if (r != MOE_OK) return r;
+  return gemm::router_dwr_tc(T, d, E, x, dl16, dWr, reinterpret_cast<CUtensorMap*>(maps_ws),
+                             status, s);
 }
 
 }  // namespace moe

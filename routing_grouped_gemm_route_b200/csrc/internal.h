@@ -23,6 +23,8 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
 
 // C[M,N] (fp32 out, or act out) = A . B with arbitrary element strides; a plain
 // CUDA-core kernel for the small router projections.
+cudaError_t launch_load_stats(const int32_t* counts, int E, moe_load_stats_t* out, int32_t* status,
+                              cudaStream_t s);
 cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A, int64_t sam,
                                int64_t sak, bool a_is_act, const void* B, int64_t sbk,
                                int64_t sbn, bool b_is_act, void* C, bool c_is_act,
@@ -95,5 +97,14 @@ moe_status gemm_bwd(const GemmShape& g, const void* dy_perm, const void* x_perm,
                     void* dH13, void* dx_perm, void* dW13, void* dW2, bool dw_fp32,
                     bool dw_accum, void* maps_ws, int* status, cudaStream_t s,
                     const MxWork* mx = nullptr);
+
+// Router GEMMs on the tensor cores (bf16 operands, fp32 accumulation; E % 64 == 0):
+// logits[T,E] = x . Wr; dx_extra[T,d] = dl16 . Wr^T (float); dWr[d,E] = x^T . dl16 (bf16),
+// with dl16 the bf16 copy of d_logits and maps_ws 2 tensor maps of device scratch.
+moe_status router_logits_tc(int T, int d, int E, const void* x, const void* Wr, float* logits,
+                            int* status, cudaStream_t s);
+moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, const void* dl16,
+                         float* dx_extra, void* dWr, void* maps_ws, int* status, cudaStream_t s);
+cudaError_t launch_f32_to_bf16(int64_t n, const float* src, void* dst, cudaStream_t s);
 
 }  // namespace moe

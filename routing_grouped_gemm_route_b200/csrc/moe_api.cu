@@ -34,6 +34,8 @@ inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 struct WsLayout {
   size_t status, hist, cta_base, maps, dy_perm, dH13, dx_perm, dx_router;
+  size_t rc_x_perm, rc_H13, rc_a, rc_y_perm;   // MOE_FLAG_RECOMPUTE: the activations
+  size_t dl16;                                  // bf16 copy of d_logits (router, bf16)
   size_t mx_ints, mx_bytes[24];   // MXFP8 operands (codes and scale chunks), see MxWork
   size_t total;
 };
@@ -53,6 +55,13 @@ WsLayout ws_layout(const moe_desc& d) {
   w.dx_perm = o; o = up(o + R * d.d * es);
   w.dx_router = o;
   if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.d * 4);
+  w.dl16 = o;
+  if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.E * 2);
+  const bool rc = d.flags & MOE_FLAG_RECOMPUTE;
+  w.rc_x_perm = o; if (rc) o = up(o + R * d.d * es);
+  w.rc_H13 = o; if (rc) o = up(o + R * 2 * (size_t)d.d_ff * es);
+  w.rc_a = o; if (rc) o = up(o + R * (size_t)d.d_ff * es);
+  w.rc_y_perm = o; if (rc) o = up(o + R * d.d * es);
   w.mx_ints = o;
   if (d.dtype == MOE_MXFP8) {
     const size_t E = d.E, f = d.d_ff, dm = d.d;
@@ -87,10 +96,11 @@ moe_saved_layout saved_layout(const moe_desc& d) {
   s.row_gate = o; o = up(o + R * 4);
   s.logits = o;
   if (d.flags & MOE_FLAG_ROUTER) o = up(o + T * E * 4);
-  s.x_perm = o; o = up(o + R * d.d * es);
-  s.H13 = o; o = up(o + R * 2 * (size_t)d.d_ff * es);
-  s.a = o; o = up(o + R * (size_t)d.d_ff * es);
-  s.y_perm = o; o = up(o + R * d.d * es);
+  const bool keep = !(d.flags & MOE_FLAG_RECOMPUTE);   // else recomputed in the backward
+  s.x_perm = o; if (keep) o = up(o + R * d.d * es);
+  s.H13 = o; if (keep) o = up(o + R * 2 * (size_t)d.d_ff * es);
+  s.a = o; if (keep) o = up(o + R * (size_t)d.d_ff * es);
+  s.y_perm = o; if (keep) o = up(o + R * d.d * es);
   s.total = o;
   return s;
 }
@@ -105,7 +115,8 @@ moe_status check(const moe_desc* d) {
   if ((int64_t)d->E * 2 * d->d_ff >= (int64_t(1) << 31) || (int64_t)d->E * d->d >= (int64_t(1) << 31))
     return MOE_EINVAL;
   if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
-  if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW)) return MOE_EINVAL;
+  if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE))
+    return MOE_EINVAL;
   if ((d->flags & MOE_FLAG_ACCUM_DW) && !(d->flags & MOE_FLAG_DW_FP32)) return MOE_EINVAL;
   if (d->dtype == MOE_MXFP8 && d->d_ff % 128 != 0) return MOE_EUNSUPPORTED;
   return MOE_OK;
@@ -209,9 +220,14 @@ moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_p
                   fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s, &mx);
 }
 
+// bf16 router GEMMs run on the tensor cores when E is a multiple of 64; fp32 (and other
+// E) use the CUDA-core kernel.
+inline bool router_tc(const moe_desc& d) { return d.dtype != MOE_FP32 && d.E % 64 == 0; }
+
 moe_status router_fwd_body(const moe_desc& d, const void* x, const void* Wr, float* logits,
-                           cudaStream_t s) {
+                           int* status, cudaStream_t s) {
   if (d.T == 0) return MOE_OK;
+  if (router_tc(d)) return router_logits_tc(d.T, d.d, d.E, x, Wr, logits, status, s);
   const bool f32 = d.dtype == MOE_FP32;
   // logits[T,E] = x[T,d] . Wr[d,E]
   return cu(launch_router_gemm(f32, d.T, d.E, d.d, x, d.d, 1, true, Wr, d.E, 1, true, logits,
@@ -220,8 +236,16 @@ moe_status router_fwd_body(const moe_desc& d, const void* x, const void* Wr, flo
 
 moe_status router_bwd_body(const moe_desc& d, const void* x, const void* Wr,
                            const float* d_logits, float* dx_extra, void* dx_act, void* dWr,
-                           cudaStream_t s) {
+                           void* ws, cudaStream_t s) {
   const bool f32 = d.dtype == MOE_FP32;
+  if (d.T > 0 && dx_extra && router_tc(d)) {
+    // d_logits rounded once to bf16 feeds both tensor-core products
+    const WsLayout w = ws_layout(d);
+    void* dl16 = at<char>(ws, w.dl16);
+    MOE_TRY(cu(launch_f32_to_bf16((int64_t)d.T * d.E, d_logits, dl16, s)));
+    return router_bwd_tc(d.T, d.d, d.E, x, Wr, dl16, dx_extra, dWr, at<char>(ws, w.maps),
+                         status_ptr(ws), s);
+  }
   if (d.T > 0) {
     if (dx_extra) {
       // dx_extra[T,d] (float) = d_logits[T,E] . Wr^T
@@ -300,7 +324,7 @@ moe_status moe_router_logits(const moe_desc* desc, const void* x, const void* Wr
   MOE_TRY(check(desc));
   MOE_TRY(tptrs(*desc, {x, logits}));
   MOE_TRY(ptrs({Wr}));
-  return router_fwd_body(*desc, x, Wr, logits, S(stream));
+  return router_fwd_body(*desc, x, Wr, logits, nullptr, S(stream));
 }
 
 moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_idx, float* gates,
@@ -414,13 +438,42 @@ moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
   MOE_TRY(ptrs({Wr, dWr}));
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
-  if (d.dtype == MOE_FP32) return router_bwd_body(d, x, Wr, d_logits, nullptr, dx, dWr, S(stream));
+  if (d.dtype == MOE_FP32)
+    return router_bwd_body(d, x, Wr, d_logits, nullptr, dx, dWr, ws, S(stream));
   // bf16: accumulate the router term in fp32, then add it to dx with one rounding
   const WsLayout w = ws_layout(d);
   if (!(d.flags & MOE_FLAG_ROUTER)) return MOE_EINVAL;
   float* extra = at<float>(ws, w.dx_router);
-  MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, S(stream)));
+  MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, ws, S(stream)));
   return cu(launch_add_f32(false, (int64_t)d.T * d.d, dx, extra, S(stream)));
+}
+
+struct Acts {
+  void *x_perm, *H13, *a, *y_perm;
+};
+Acts acts(const moe_desc& d, const void* saved, const moe_saved_layout& L, void* ws) {
+  Acts r;
+  if (d.flags & MOE_FLAG_RECOMPUTE) {
+    const WsLayout w = ws_layout(d);
+    r.x_perm = at<char>(ws, w.rc_x_perm);
+    r.H13 = at<char>(ws, w.rc_H13);
+    r.a = at<char>(ws, w.rc_a);
+    r.y_perm = at<char>(ws, w.rc_y_perm);
+  } else {
+    void* sv = const_cast<void*>(saved);
+    r.x_perm = at<char>(sv, L.x_perm);
+    r.H13 = at<char>(sv, L.H13);
+    r.a = at<char>(sv, L.a);
+    r.y_perm = at<char>(sv, L.y_perm);
+  }
+  return r;
+}
+
+moe_status moe_load_stats(const int32_t* counts, int32_t E, moe_load_stats_t* out,
+                          int32_t* status, void* stream) {
+  if (E < 1 || E > 1024) return MOE_EINVAL;
+  MOE_TRY(ptrs({counts, out}));
+  return cu(launch_load_stats(counts, E, out, status, S(stream)));
 }
 
 moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logits, const void* Wr,
@@ -442,7 +495,7 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   const float* lg = logits;
   if (router) {
     float* out = at<float>(saved, L.logits);
-    MOE_TRY(router_fwd_body(d, x, Wr, out, s));
+    MOE_TRY(router_fwd_body(d, x, Wr, out, st, s));
     lg = out;
   }
   int32_t* idx = at<int32_t>(saved, L.topk_idx);
@@ -453,13 +506,13 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
                      at<int32_t>(saved, L.row_token), at<float>(saved, L.row_gate), ws, s));
   if (d.T == 0) return MOE_OK;
   const bool f32 = d.dtype == MOE_FP32;
-  void* x_perm = at<char>(saved, L.x_perm);
-  void* y_perm = at<char>(saved, L.y_perm);
-  MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, x_perm, st, s)));
+  // the activations the backward reads: in `saved`, or workspace scratch when the
+  // backward recomputes them
+  const Acts A = acts(d, saved, L, ws);
+  MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
   MxWork mx = mx_work(d, ws);
-  MOE_TRY(gemm_fwd(gshape(d), x_perm, W13, W2, offsets, at<char>(saved, L.H13),
-                   at<char>(saved, L.a), y_perm, st, s, &mx));
-  return cu(launch_gather_sum(f32, d.T, d.d, d.k, y_perm, gates, slot, nullptr, y, st, s));
+  MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, A.y_perm, gates, slot, nullptr, y, st, s));
 }
 
 moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, const void* saved,
@@ -469,12 +522,11 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
   MOE_TRY(check(desc));
   const moe_desc& d = *desc;
   const bool router = d.flags & MOE_FLAG_ROUTER;
+  const bool recompute = d.flags & MOE_FLAG_RECOMPUTE;
   MOE_TRY(tptrs(d, {dy, dx, d_logits}));
   MOE_TRY(ptrs({saved, W13, W2, dW13, dW2}));
-  if (router) {
-    MOE_TRY(tptrs(d, {x}));
-    MOE_TRY(ptrs({Wr, dWr}));
-  }
+  if (router || recompute) MOE_TRY(tptrs(d, {x}));
+  if (router) MOE_TRY(ptrs({Wr, dWr}));
   MOE_TRY(ws_ok(d, ws, ws_bytes));
   const moe_saved_layout L = saved_layout(d);
   if (saved_bytes < L.total) return MOE_EWORKSPACE;
@@ -490,15 +542,23 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
   void* dy_perm = at<char>(ws, w.dy_perm);
   void* dH13 = at<char>(ws, w.dH13);
   void* dx_perm = at<char>(ws, w.dx_perm);
+  const Acts A = acts(d, saved, L, ws);
+  if (recompute && d.T > 0) {
+    // the forward's activations again, from x and the saved routing (same kernels,
+    // same inputs: bit-identical to the ones the forward used)
+    MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
+    MxWork mx = mx_work(d, ws);
+    MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+  }
 
-  MOE_TRY(cu(launch_combine_bwd(f32, d.T, d.d, d.k, d.E, dy, at<char>(saved, L.y_perm), gates,
-                                idx, slot, dy_perm, d_logits, st, s)));
-  MOE_TRY(gemm_bwd_body(d, dy_perm, at<char>(saved, L.x_perm), at<char>(saved, L.H13),
-                        at<char>(saved, L.a), W13, W2, offsets, dH13, dx_perm, dW13, dW2, ws, s));
+  MOE_TRY(cu(launch_combine_bwd(f32, d.T, d.d, d.k, d.E, dy, A.y_perm, gates, idx, slot, dy_perm,
+                                d_logits, st, s)));
+  MOE_TRY(gemm_bwd_body(d, dy_perm, A.x_perm, A.H13, A.a, W13, W2, offsets, dH13, dx_perm, dW13,
+                        dW2, ws, s));
   float* extra = nullptr;
   if (router) {
     extra = at<float>(ws, w.dx_router);
-    MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, s));
+    MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, ws, s));
   }
   return cu(launch_gather_sum(f32, d.T, d.d, d.k, dx_perm, nullptr, slot, extra, dx, st, s));
 }

@@ -8,6 +8,8 @@
 // token, 16-byte vector loads and stores, each x row read once and written k times
 // (dispatch), each routed row read once (combine, unpermute-reduce).  Combine and
 // unpermute are gathers summed in fp32 in a fixed order: no atomics, deterministic.
+#include <algorithm>
+
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
 
@@ -223,6 +225,29 @@ cudaError_t launch_add_f32(bool fp32, int64_t n, void* y, const float* extra, cu
   const int blocks = 4 * num_sms();
   if (fp32) add_f32_kernel<float><<<blocks, 256, 0, s>>>((float*)y, extra, n);
   else add_f32_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((__nv_bfloat16*)y, extra, n);
+  return cudaGetLastError();
+}
+
+// bf16 copy (round to nearest even) of a float array; n a multiple of 8.
+__global__ void f32_to_bf16_kernel(const float* __restrict__ src, __nv_bfloat16* dst, int64_t n) {
+  const int64_t nv = n / 8;
+  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nv;
+       v += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = reinterpret_cast<const float4*>(src)[2 * v];
+    const float4 b = reinterpret_cast<const float4*>(src)[2 * v + 1];
+    const float f[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    Vec16<__nv_bfloat16> o;
+    o.from_float(f);
+    stg16(dst + v * 8, o.raw);
+  }
+}
+
+cudaError_t launch_f32_to_bf16(int64_t n, const float* src, void* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 8 != 0) return cudaErrorInvalidValue;
+  const int64_t nv = n / 8;
+  const int blocks = (int)std::min<int64_t>((nv + 255) / 256, (int64_t)num_sms() * 8);
+  f32_to_bf16_kernel<<<blocks, 256, 0, s>>>(src, reinterpret_cast<__nv_bfloat16*>(dst), n);
   return cudaGetLastError();
 }
 

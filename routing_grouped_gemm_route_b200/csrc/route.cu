@@ -247,6 +247,61 @@ __global__ void __launch_bounds__(256) router_gemm_kernel(int M, int N, int K, c
   }
 }
 
+// Expert load statistics: one CTA, thread e reads counts[e] (e < E <= 1024).  Sums in
+// int64 (exact); the spread about the mean in double, reduced in a fixed order.
+template <typename V, typename Op>
+__device__ __forceinline__ V block_reduce(V v, Op op, V identity, V* scratch) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) scratch[warp] = v;
+  __syncthreads();
+  const int nw = (blockDim.x + 31) >> 5;
+  v = lane < nw ? scratch[lane] : identity;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = op(v, __shfl_xor_sync(0xffffffffu, v, o));
+  __syncthreads();   // scratch free for the next reduction
+  return v;
+}
+
+__global__ void __launch_bounds__(1024) load_stats_kernel(const int32_t* __restrict__ counts, int E,
+                                                          moe_load_stats_t* out, int32_t* status) {
+  __shared__ long long s_ll[32];
+  __shared__ double s_d[32];
+  const int e = threadIdx.x;
+  long long c = 0;
+  if (e < E) {
+    c = counts[e];
+    if (c < 0) {
+      set_status(reinterpret_cast<int*>(status), MOE_DEV_BAD_OFFSETS);
+      c = 0;
+    }
+  }
+  auto add = [](long long a, long long b) { return a + b; };
+  const long long lo = INT32_MIN, hi = INT32_MAX;
+  const long long total = block_reduce(c, add, 0LL, s_ll);
+  const long long mx = block_reduce(e < E ? c : lo,
+                                    [](long long a, long long b) { return a > b ? a : b; }, lo, s_ll);
+  const long long mn = block_reduce(e < E ? c : hi,
+                                    [](long long a, long long b) { return a < b ? a : b; }, hi, s_ll);
+  const long long empty = block_reduce((long long)(e < E && c == 0), add, 0LL, s_ll);
+  const double mean = (double)total / (double)E;
+  const double dev = e < E ? ((double)c - mean) * ((double)c - mean) : 0.0;
+  const double ss = block_reduce(dev, [](double a, double b) { return a + b; }, 0.0, s_d);
+  if (e == 0) {
+    moe_load_stats_t r;
+    r.total = total;
+    r.max_count = (int32_t)mx;
+    r.min_count = (int32_t)mn;
+    r.num_empty = (int32_t)empty;
+    r.num_experts = E;
+    r.mean = mean;
+    r.max_over_mean = total > 0 ? (double)mx / mean : 0.0;
+    r.cv = total > 0 ? sqrt(ss / (double)E) / mean : 0.0;
+    *out = r;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
@@ -274,6 +329,13 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   }
   slot_kernel<<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, T, E, k, slot,
                                               row_token, row_gate, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_load_stats(const int32_t* counts, int E, moe_load_stats_t* out, int32_t* status,
+                              cudaStream_t s) {
+  const int threads = (E + 31) / 32 * 32;
+  load_stats_kernel<<<1, threads, 0, s>>>(counts, E, out, status);
   return cudaGetLastError();
 }
 

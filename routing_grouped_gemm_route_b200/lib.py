@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(_PKG, "libmoe.so")
 MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE_EDEVICE = \
     0, -1, -2, -3, -4, -5, -6
 MOE_FP32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
-MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW = 1, 2, 4
+MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW, MOE_FLAG_RECOMPUTE = 1, 2, 4, 8
 MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
@@ -30,8 +30,8 @@ EXPORTS = ["moe_status_string", "moe_check_desc", "moe_workspace_size", "moe_sav
            "moe_workspace_init", "moe_read_device_status", "moe_router_logits", "moe_route",
            "moe_route_noalloc", "moe_mx_scale_bytes", "moe_mx_quantize",
            "moe_dispatch", "moe_grouped_gemm_fwd", "moe_combine", "moe_combine_bwd",
-           "moe_grouped_gemm_bwd", "moe_dispatch_bwd", "moe_router_bwd", "moe_layer_fwd",
-           "moe_layer_bwd"]
+           "moe_grouped_gemm_bwd", "moe_dispatch_bwd", "moe_router_bwd", "moe_load_stats",
+           "moe_layer_fwd", "moe_layer_bwd"]
 
 
 class MoEError(RuntimeError):
@@ -50,6 +50,13 @@ class moe_saved_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_idx", "gates", "counts", "offsets", "slot", "row_token", "row_gate",
                  "logits", "x_perm", "H13", "a", "y_perm", "total")]
+
+
+class moe_load_stats_t(ctypes.Structure):
+    _fields_ = [("total", ctypes.c_int64), ("max_count", ctypes.c_int32),
+                ("min_count", ctypes.c_int32), ("num_empty", ctypes.c_int32),
+                ("num_experts", ctypes.c_int32), ("mean", ctypes.c_double),
+                ("max_over_mean", ctypes.c_double), ("cv", ctypes.c_double)]
 
 
 _lib = None
@@ -87,6 +94,7 @@ def load():
         "moe_grouped_gemm_bwd": [_P] + [_P] * 11 + [_P, _S, _P],
         "moe_dispatch_bwd": [_P, _P, _P, _P, _P, _S, _P],
         "moe_router_bwd": [_P, _P, _P, _P, _P, _P, _P, _S, _P],
+        "moe_load_stats": [_P, _I, _P, _P, _P],
         "moe_layer_fwd": [_P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _S, _P],
         "moe_layer_bwd": [_P, _P, _P, _P, _S, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P],
     }
@@ -259,6 +267,26 @@ def moe_router_bwd(desc, x, Wr, d_logits, dx, dWr, ws, stream=None):
            "moe_router_bwd")
 
 
+LOAD_STATS_BYTES = ctypes.sizeof(moe_load_stats_t)
+
+
+def moe_load_stats(counts, out, status=None, stream=None):
+    """counts: int32 [E] device tensor; out: a device tensor of at least LOAD_STATS_BYTES
+    bytes (16-byte aligned) that receives a moe_load_stats_t; status: optional int32
+    device word for MOE_DEV_BAD_OFFSETS."""
+    if out.numel() * out.element_size() < LOAD_STATS_BYTES:
+        raise MoEError(MOE_EWORKSPACE, "moe_load_stats")
+    _check(load().moe_load_stats(_ptr(counts), int(counts.numel()), _ptr(out), _ptr(status),
+                                 _stream(stream)), "moe_load_stats")
+
+
+def decode_load_stats(out) -> dict:
+    """The moe_load_stats_t in `out` (copied to the host) as a dict."""
+    raw = bytes(out.detach().cpu().view(torch.uint8)[:LOAD_STATS_BYTES].numpy().tobytes())
+    st = moe_load_stats_t.from_buffer_copy(raw)
+    return {name: getattr(st, name) for name, _ in moe_load_stats_t._fields_}
+
+
 def moe_layer_fwd(desc, x, logits, Wr, W13, W2, y, saved, ws, stream=None):
     _check(load().moe_layer_fwd(ctypes.byref(desc), _ptr(x), _ptr(logits), _ptr(Wr), _ptr(W13),
                                 _ptr(W2), _ptr(y), _ptr(saved), _nbytes(saved), _ptr(ws),
@@ -290,11 +318,12 @@ def saved_views(desc, saved: torch.Tensor) -> dict:
                offsets=view(L.offsets, E + 1, torch.int32, (E + 1,)),
                slot=view(L.slot, T * k, torch.int32, (T, k)),
                row_token=view(L.row_token, R, torch.int32, (R,)),
-               row_gate=view(L.row_gate, R, torch.float32, (R,)),
-               x_perm=view(L.x_perm, R * d, act, (R, d)),
-               H13=view(L.H13, R * 2 * f, act, (R, 2 * f)),
-               a=view(L.a, R * f, act, (R, f)),
-               y_perm=view(L.y_perm, R * d, act, (R, d)))
+               row_gate=view(L.row_gate, R, torch.float32, (R,)))
+    if not desc.flags & MOE_FLAG_RECOMPUTE:     # else the backward recomputes them
+        out.update(x_perm=view(L.x_perm, R * d, act, (R, d)),
+                   H13=view(L.H13, R * 2 * f, act, (R, 2 * f)),
+                   a=view(L.a, R * f, act, (R, f)),
+                   y_perm=view(L.y_perm, R * d, act, (R, d)))
     if desc.flags & MOE_FLAG_ROUTER:
         out["logits"] = view(L.logits, T * E, torch.float32, (T, E))
     return out

@@ -53,7 +53,9 @@ def test_descriptor_checks(L, args, code):
 
 
 def test_flag_checks(L):
-    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 8)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 16)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
+                                            lib.MOE_FLAG_RECOMPUTE)) == 0
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
                                             lib.MOE_FLAG_ACCUM_DW)) == lib.MOE_EINVAL
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
@@ -73,6 +75,24 @@ def test_sizes_grow_with_the_problem(L):
     assert all(o % 256 == 0 for o in offs) and offs == sorted(offs)
     assert s.y_perm + R * 2048 * 2 <= s.total
     assert s.H13 - s.x_perm >= R * 2048 * 2 and s.a - s.H13 >= R * 2048 * 2
+
+
+def test_recompute_moves_activations_from_saved_to_workspace(L):
+    d = lib.make_desc(16384, 2048, 1024, 128, 4, "bf16")
+    r = lib.make_desc(16384, 2048, 1024, 128, 4, "bf16", lib.MOE_FLAG_RECOMPUTE)
+    R = 16384 * 4
+    acts = R * 2048 * 2 * 2 + R * 1024 * 2 * 3          # x_perm, y_perm, H13, a
+    s_d, s_r = lib.moe_saved_layout_get(d), lib.moe_saved_layout_get(r)
+    assert s_d.total - s_r.total >= acts
+    assert s_r.x_perm == s_r.H13 == s_r.a == s_r.y_perm == s_r.total
+    assert s_r.total < 3 * 1024 * 1024                    # routing metadata only
+    assert lib.moe_workspace_size(r) - lib.moe_workspace_size(d) >= acts
+
+
+def test_load_stats_struct_layout(L):
+    # the C struct: int64 total, four int32, three doubles
+    assert lib.LOAD_STATS_BYTES == 48
+    assert lib.moe_load_stats_t.mean.offset == 24
 
 
 def _p(v):

@@ -58,6 +58,9 @@ def test_tiny_fp32_workload(cuda_lib):
 @pytest.mark.parametrize("T,d,E,k,f,dt,router,skew", [
     (1000, 256, 8, 4, 128, "bf16", False, False),
     (777, 128, 8, 2, 256, "bf16", True, False),
+    (1500, 256, 128, 4, 128, "bf16", True, False),     # router on the tensor cores
+    (333, 384, 64, 2, 128, "bf16", True, True),
+    (700, 512, 256, 8, 128, "bf16", True, False),
     (2000, 256, 128, 4, 128, "bf16", False, False),
     (2000, 256, 128, 4, 128, "bf16", False, True),
     (333, 384, 12, 3, 192, "fp32", False, False),

@@ -1,0 +1,86 @@
+"""Device load statistics (moe_load_stats) against the oracle's definitions, and the
+layer with activation recompute (MOE_FLAG_RECOMPUTE) against the layer without it."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from routing_grouped_gemm_route_b200 import lib
+from routing_grouped_gemm_route_b200.inputs import Workload, make_inputs, random_logits
+
+from helpers import TOL, f64, npi, rel, run_layer, run_route
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_stats(counts_dev, status=None):
+    out = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    lib.moe_load_stats(counts_dev, out, status)
+    torch.cuda.synchronize()
+    return lib.decode_load_stats(out)
+
+
+def assert_stats_equal(got, want):
+    for key in ("total", "max_count", "min_count", "num_empty", "num_experts"):
+        assert got[key] == want[key], key
+    for key in ("mean", "max_over_mean", "cv"):
+        assert abs(got[key] - want[key]) <= 1e-12 * max(1.0, abs(want[key])), key
+
+
+@pytest.mark.parametrize("T,E,k,skew", [(16384, 128, 4, False), (16384, 128, 4, True),
+                                        (4096, 8, 2, False), (1000, 1024, 8, True),
+                                        (300, 1, 1, False)])
+def test_load_stats_of_routing(cuda_lib, T, E, k, skew):
+    L = random_logits(T, E, seed=T + E)
+    if skew:
+        # Zipf-like bias over a seeded permutation of the experts
+        g = np.random.default_rng(E)
+        rank = g.permutation(E) + 1
+        L = L + torch.tensor(-1.8 * np.log(rank), dtype=torch.float32)[None, :]
+    desc = lib.make_desc(T, 128, 64, E, k, "bf16")
+    r = run_route(desc, L.cuda())
+    want = oracle.load_stats(npi(r["counts"]))
+    assert_stats_equal(gpu_stats(r["counts"]), want)
+
+
+def test_load_stats_edge_cases(cuda_lib):
+    for counts in ([0, 0, 0, 0], [5], [0] * 1023 + [77], list(range(1024))):
+        c = torch.tensor(counts, dtype=torch.int32, device="cuda")
+        assert_stats_equal(gpu_stats(c), oracle.load_stats(counts))
+    # a negative count is reported and read as 0
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    c = torch.tensor([3, -2, 5], dtype=torch.int32, device="cuda")
+    st = gpu_stats(c, status)
+    assert int(status.item()) & lib.MOE_DEV_BAD_OFFSETS
+    assert_stats_equal(st, oracle.load_stats([3, 0, 5]))
+
+
+@pytest.mark.parametrize("T,d,E,k,f,dt,router", [
+    (3000, 256, 16, 4, 128, "bf16", False),
+    (2000, 256, 8, 2, 256, "bf16", True),
+    (1500, 256, 8, 4, 128, "mxfp8", False),
+    (512, 128, 8, 2, 256, "fp32", True),
+    (0, 256, 8, 2, 128, "bf16", False),
+])
+def test_recompute_is_bit_identical(cuda_lib, T, d, E, k, f, dt, router):
+    w = Workload("rc", T, d, E, k, f, dt, router=router, skew=False, seed=T + 3)
+    inp = make_inputs(w)
+    _, lay0, _, y0, g0, st0 = run_layer(w, inp)
+    _, lay1, _, y1, g1, st1 = run_layer(w, inp, flags=lib.MOE_FLAG_RECOMPUTE)
+    assert st0 == 0 and st1 == 0
+    assert lay1.saved.numel() < lay0.saved.numel() or T == 0
+    assert torch.equal(y0, y1)
+    for name in ("dx", "d_logits", "dW13", "dW2") + (("dWr",) if router else ()):
+        assert torch.equal(g0[name], g1[name]), name
+    if T and dt == "bf16":
+        # and against the oracle, as the plain layer is
+        x, dy = f64(inp["x"]), f64(inp["dy"])
+        W13, W2 = inp["W13"].float().numpy(), inp["W2"].float().numpy()
+        L = None if router else f64(inp["logits"])
+        Wr = inp["Wr"].float().numpy() if router else None
+        if router:
+            L = f64(lay1.views()["logits"])
+        fwd = oracle.layer_fwd(x, W13, W2, logits=L, k=k)
+        bwd = oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr)
+        assert rel(y1, fwd["y"]) < TOL
+        assert rel(g1["dW13"], bwd["dW13"]) < TOL

@@ -123,3 +123,28 @@ def test_skewed_routing_is_imbalanced():
     c = oracle.route(L, 4, 128)["counts"]
     assert (c == 0).sum() >= 40
     assert c.max() > 10 * c.mean()
+
+
+# ------------------------------------------------------------------- load statistics
+
+def test_load_stats_hand_example():
+    # mean 3; deviations -3, -1, 1, 3 -> mean square 5
+    st = oracle.load_stats([0, 2, 4, 6])
+    assert (st["total"], st["max_count"], st["min_count"], st["num_empty"]) == (12, 6, 0, 1)
+    assert st["mean"] == 3.0 and st["max_over_mean"] == 2.0
+    assert abs(st["cv"] - np.sqrt(5.0) / 3.0) < 1e-15
+
+
+def test_load_stats_balanced_and_one_hot():
+    st = oracle.load_stats([7] * 8)
+    assert st["max_over_mean"] == 1.0 and st["cv"] == 0.0 and st["num_empty"] == 0
+    # everything on one of E experts: max/mean = E, E-1 empty, cv = sqrt(E-1)
+    st = oracle.load_stats([0] * 7 + [40])
+    assert st["max_over_mean"] == 8.0 and st["num_empty"] == 7
+    assert abs(st["cv"] - np.sqrt(7.0)) < 1e-14
+
+
+def test_load_stats_no_tokens():
+    st = oracle.load_stats([0, 0, 0])
+    assert st["total"] == 0 and st["num_empty"] == 3
+    assert st["max_over_mean"] == 0.0 and st["cv"] == 0.0
