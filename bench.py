@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--router", action="store_true", help="compute logits = x.Wr on the device")
     ap.add_argument("--recompute", action="store_true",
                     help="activation recompute: the backward redoes dispatch, FC1 and FC2")
+    ap.add_argument("--shared-expert", action="store_true",
+                    help="one shared expert (dense SwiGLU FFN on every token); the step is then "
+                         "timed through the whole-layer calls")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-steps", type=int, default=30, help="0 skips the end-to-end leg")
@@ -321,6 +324,8 @@ def main():
         w = w.replace(E=args.experts, name=w.name + f"[E={args.experts}]")
     if args.dtype is not None and args.dtype != w.dtype:
         w = w.replace(dtype=args.dtype, name=w.name + f"[{args.dtype}]")
+    if args.shared_expert:
+        w = w.replace(shared=True, name=w.name + "[shared expert]")
     world, rank, local = dist_setup()
     if args.impl == "reference":
         run_reference(args, w, world, rank)
@@ -334,7 +339,8 @@ def main():
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_inputs(w, device=dev, seed=w.seed + rank)
     flags = (lib.MOE_FLAG_ROUTER if w.router else 0) | \
-        (lib.MOE_FLAG_RECOMPUTE if args.recompute else 0)
+        (lib.MOE_FLAG_RECOMPUTE if args.recompute else 0) | \
+        (lib.MOE_FLAG_SHARED_EXPERT if w.shared else 0)
     desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
     act = lib.act_dtype(desc)
     T, d, f, E, k = w.T, w.d, w.d_ff, w.E, w.k
@@ -353,7 +359,8 @@ def main():
     x_perm, H13, a, y_perm, y = z(R, d), z(R, 2 * f), z(R, f), z(R, d), z(T, d)
     dy_perm, dH13, dx_perm, dx = z(R, d), z(R, 2 * f), z(R, d), z(T, d)
     d_logits = z(T, E, dt=torch.float32)
-    dW13, dW2 = z(E, 2 * f, d), z(E, d, f)
+    nw = E + (1 if w.shared else 0)                 # weight slices (shared expert last)
+    dW13, dW2 = z(nw, 2 * f, d), z(nw, d, f)
     dWr = z(d, E) if w.router else None
 
     stages = ["route", "dispatch", "gemm_fwd", "combine", "combine_bwd", "gemm_bwd",
@@ -361,6 +368,12 @@ def main():
     if args.recompute:
         # the backward first recomputes the forward's activations (same buffers here)
         stages = stages[:4] + ["re_dispatch", "re_gemm_fwd"] + stages[4:]
+    layer = None
+    if w.shared:
+        # the shared expert lives in the whole-layer calls: time those
+        layer = lib.Layer(desc, device=dev)
+        stages = ["layer_fwd", "layer_bwd"]
+        layer_out = dict(dx=dx, d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
     if w.router:
         stages = ["router"] + stages + ["router_bwd"]
     mx = w.dtype == "mxfp8"
@@ -370,6 +383,10 @@ def main():
                 "combine": 1, "combine_bwd": 1, "gemm_bwd": 12 if mx else 5, "dispatch_bwd": 1,
                 "router_bwd": 3}
     launches["re_dispatch"], launches["re_gemm_fwd"] = launches["dispatch"], launches["gemm_fwd"]
+    # whole-layer calls: route 3, dispatch 1, GEMMs 2, shared 2, combine 1 (+ router 1);
+    # combine-bwd 1, GEMMs 5, shared 5, unpermute 1 (+ router: bf16 copy, maps, 2 GEMMs)
+    launches["layer_fwd"] = 9 + (1 if w.router else 0)
+    launches["layer_bwd"] = 12 + (4 if w.router else 0)
 
     def run_stage(name):
         if name == "router":
@@ -391,13 +408,17 @@ def main():
             lib.moe_dispatch_bwd(desc, dx_perm, slot, dx, ws)
         elif name == "router_bwd":
             lib.moe_router_bwd(desc, x, Wr, d_logits, dx, dWr, ws)
+        elif name == "layer_fwd":
+            layer.fwd(x, W13, W2, logits=None if w.router else logits, Wr=Wr, y=y)
+        elif name == "layer_bwd":
+            layer.bwd(dy, W13, W2, x=x, Wr=Wr, out=layer_out)
 
     K, W = args.steps, args.warmup
     for _ in range(W):
         for s in stages:
             run_stage(s)
     torch.cuda.synchronize()
-    if lib.moe_read_device_status(ws) != 0:
+    if lib.moe_read_device_status(layer.ws if layer else ws) != 0:
         raise RuntimeError("device status set during warm-up")
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(len(stages) + 1)] for _ in range(K)]
@@ -420,8 +441,10 @@ def main():
     clk = clocks.stop()
     ms_local = start.elapsed_time(stop)
     ms_total = max_over_ranks(ms_local, world)
-    if lib.moe_read_device_status(ws) != 0:
+    if lib.moe_read_device_status(layer.ws if layer else ws) != 0:
         raise RuntimeError("device status set during the timed region")
+    if layer is not None:
+        counts = layer.views()["counts"]
     # expert load of this routing (device statistics kernel, outside the timed region)
     st_buf = torch.zeros(64, dtype=torch.uint8, device=dev)
     lib.moe_load_stats(counts, st_buf)
@@ -457,8 +480,15 @@ def main():
             r.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm"], 3)})
         stage_rep[s] = r
 
-    gemm_ms = stage_ms["gemm_fwd"] + stage_ms["gemm_bwd"]
-    gemm_tflops = (gemm_flops["gemm_fwd"] + gemm_flops["gemm_bwd"]) / (gemm_ms * 1e-3) / 1e12
+    if layer is None:
+        gemm_ms = stage_ms["gemm_fwd"] + stage_ms["gemm_bwd"]
+        gemm_work = gemm_flops["gemm_fwd"] + gemm_flops["gemm_bwd"]
+    else:
+        # whole-layer timing: all GEMM flops (routed + shared expert) over the whole step,
+        # a lower bound of the GEMM kernels' rate
+        gemm_ms = stage_ms["layer_fwd"] + stage_ms["layer_bwd"]
+        gemm_work = 18.0 * (R + T) * d * f
+    gemm_tflops = gemm_work / (gemm_ms * 1e-3) / 1e12
     peak_tf = pk["bf16_sustained"]
     peak_kind = "sustained dense bf16"
     if act == torch.float32:
@@ -486,6 +516,9 @@ def main():
                 if pk["source"] == "measured" else f"fallback 1.4 PFLOP/s, {peak_kind}"}
     if mx:
         roofline["kernel"] += "; the GEMM stages include the MXFP8 quantisers of their operands"
+    if layer is not None:
+        roofline["kernel"] = ("grouped GEMM incl. the shared expert (18*(T*k + T)*d*d_ff flops) "
+                              "over the whole moe_layer_fwd + moe_layer_bwd time (lower bound)")
 
     # ---------------------------------------------------------------- end to end (host buffers)
     e2e = None
@@ -505,7 +538,7 @@ def main():
             "vs_baseline": None, "dtype": ("mxfp8-e4m3" if mx else "bf16") if act == torch.bfloat16 else "f32",
             "data": "synthetic (seeded N(0,1) activations/logits, N(0,0.02) weights)",
             "config": {"workload": workload_desc(w), "T": T, "d_model": d, "E": E, "top_k": k,
-                       "d_ff": f, "router_on_device": w.router, "recompute": args.recompute,
+                       "d_ff": f, "router_on_device": w.router, "recompute": args.recompute, "shared_expert": w.shared,
                        "expert_load": load,
                        "parallelism": f"replicas x{world} (data parallel, no data-path collective)",
                        "l2": "no flush: each step's working set (~5 GB of weights, activations "

@@ -76,6 +76,13 @@ typedef enum moe_dtype {
  * recomputes dispatch, FC1 + SwiGLU and FC2 from x (then required) before the backward.
  * The results are bit-identical to the run without the flag. */
 #define MOE_FLAG_RECOMPUTE 8
+/* One shared expert (bigchange.ai pt-BR, last section: the production rows use top-4
+ * routing and one shared expert): a SwiGLU FFN of the routed experts' shape applied to
+ * every token with weight 1 and added to y.  W13, W2 (and dW13, dW2) then hold E+1
+ * experts, the last being the shared one; the router still chooses among the first E.
+ * It runs as the grouped GEMM with one segment of all T tokens; x is required in
+ * moe_layer_bwd.  Not with MOE_MXFP8 (MOE_EUNSUPPORTED). */
+#define MOE_FLAG_SHARED_EXPERT 16
 
 /* device status bits */
 #define MOE_DEV_BAD_INDEX   1  /* an expert index or slot was out of range; the row was skipped */
@@ -105,6 +112,9 @@ typedef struct moe_saved_layout {
   size_t H13;        /* act [R,2*d_ff] */
   size_t a;          /* act [R,d_ff] */
   size_t y_perm;     /* act [R,d] */
+  /* shared expert (MOE_FLAG_SHARED_EXPERT without MOE_FLAG_RECOMPUTE; else absent) */
+  size_t H13_shared; /* act [T,2*d_ff] */
+  size_t a_shared;   /* act [T,d_ff] */
   size_t total;      /* bytes needed */
 } moe_saved_layout;
 
@@ -293,8 +303,8 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
 
 /* Whole layer backward for upstream gradient dy [T,d] act.  Out: dx [T,d] act,
  * d_logits [T,E] float, dW13, dW2 (see moe_grouped_gemm_bwd), and dWr [d,E] act when
- * MOE_FLAG_ROUTER.  x (the forward's input) is required with MOE_FLAG_ROUTER or
- * MOE_FLAG_RECOMPUTE and may be NULL otherwise. */
+ * MOE_FLAG_ROUTER.  x (the forward's input) is required with MOE_FLAG_ROUTER,
+ * MOE_FLAG_RECOMPUTE or MOE_FLAG_SHARED_EXPERT and may be NULL otherwise. */
 moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x,
                          const void* saved, size_t saved_bytes, const void* W13,
                          const void* W2, const void* Wr, void* dx, float* d_logits,

@@ -270,9 +270,16 @@ def experts_bwd(dy_perm, x_perm, H13, a, offsets, W13, W2, mx: bool = False):
 
 # --------------------------------------------------------------------------- whole layer
 
-def layer_fwd(x, W13, W2, logits=None, Wr=None, k: int = 2, mx: bool = False) -> dict:
-    """Forward of the routed MoE layer; returns every intermediate by name."""
-    E = W13.shape[0]
+def layer_fwd(x, W13, W2, logits=None, Wr=None, k: int = 2, mx: bool = False,
+              shared: bool = False) -> dict:
+    """Forward of the routed MoE layer; returns every intermediate by name.
+
+    ``shared``: W13 / W2 hold one more expert than the router chooses from; that last
+    one is the shared expert (the write-ups' production rows use one: bigchange.ai
+    pt-BR, last section), a SwiGLU FFN applied to every token with weight 1 and added
+    to y: y_t = sum_j g_tj FFN_{e_tj}(x_t) + FFN_shared(x_t).
+    """
+    E = W13.shape[0] - (1 if shared else 0)
     if logits is None:
         if Wr is None:
             raise ValueError("need logits or Wr")
@@ -281,9 +288,16 @@ def layer_fwd(x, W13, W2, logits=None, Wr=None, k: int = 2, mx: bool = False) ->
         L = _f64(logits)
     r = route(L, k, E)
     x_perm = dispatch(x, r["slot"])
-    H13, A, Yp = experts_fwd(x_perm, r["offsets"], W13, W2, mx=mx)
+    H13, A, Yp = experts_fwd(x_perm, r["offsets"], W13[:E], W2[:E], mx=mx)
     y = combine(Yp, r["gates"], r["slot"])
-    r.update(logits=L, x_perm=x_perm, H13=H13, a=A, y_perm=Yp, y=y)
+    r.update(logits=L, x_perm=x_perm, H13=H13, a=A, y_perm=Yp)
+    if shared:
+        # one expert over all T tokens in token order: a dense SwiGLU FFN
+        T = _f64(x).shape[0]
+        Hs, As, Ys = experts_fwd(_f64(x), [0, T], W13[E:], W2[E:], mx=mx)
+        y = y + Ys
+        r.update(H13_shared=Hs, a_shared=As, y_shared=Ys)
+    r["y"] = y
     return r
 
 
@@ -291,14 +305,24 @@ def layer_bwd(fwd: dict, dy, x, W13, W2, Wr=None, mx: bool = False) -> dict:
     """Backward of ``layer_fwd`` for upstream gradient ``dy``.
 
     Returns dx, d_logits, dW13, dW2 and, when the router ran (``Wr`` given), dWr.
-    With the router, dx includes d_logits . Wr^T and dWr = x^T . d_logits.
+    With the router, dx includes d_logits . Wr^T and dWr = x^T . d_logits.  With a
+    shared expert (the forward ran with ``shared``), dW13 / dW2 have its gradient as
+    their last expert and dx includes its input gradient.
     """
-    E = W13.shape[0]
+    shared = "y_shared" in fwd
+    E = W13.shape[0] - (1 if shared else 0)
     dy_perm, d_logits = combine_bwd(dy, fwd["y_perm"], fwd["gates"], fwd["topk_idx"],
                                     fwd["slot"], E)
     dH13, dx_perm, dW13, dW2 = experts_bwd(dy_perm, fwd["x_perm"], fwd["H13"], fwd["a"],
-                                           fwd["offsets"], W13, W2, mx=mx)
+                                           fwd["offsets"], W13[:E], W2[:E], mx=mx)
     dx = dispatch_bwd(dx_perm, fwd["slot"])
+    if shared:
+        T = _f64(dy).shape[0]
+        _, dXs, dW13s, dW2s = experts_bwd(_f64(dy), _f64(x), fwd["H13_shared"], fwd["a_shared"],
+                                          [0, T], W13[E:], W2[E:], mx=mx)
+        dx = dx + dXs
+        dW13 = np.concatenate([dW13, dW13s])
+        dW2 = np.concatenate([dW2, dW2s])
     out = dict(dy_perm=dy_perm, dH13=dH13, dx_perm=dx_perm, dW13=dW13, dW2=dW2,
                d_logits=d_logits)
     if Wr is not None:

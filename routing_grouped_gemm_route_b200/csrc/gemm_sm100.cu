@@ -979,14 +979,14 @@ static moe_status fc1_fwd(const GemmShape& g, const void* x_perm, const void* W1
                                                          H13, 2 * g.f, a, nullptr, off, st, s);
 }
 
-template <typename T>
+template <typename T, typename OutT = T>
 static moe_status fc2_fwd(const GemmShape& g, const void* a, const void* W2, const int32_t* off,
                           void* y_perm, int* st, cudaStream_t s) {
   if (g.d % 256 == 0)
-    return run_m<T, false, EPI_STORE, 256, kPair<T>>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d,
-                                                      nullptr, nullptr, off, st, s);
-  return run_m<T, false, EPI_STORE, 128, kPair<T>>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d,
-                                                    nullptr, nullptr, off, st, s);
+    return run_m<T, false, EPI_STORE, 256, kPair<T>, OutT>(g, a, g.f, W2, g.d, g.d, g.f, y_perm,
+                                                            g.d, nullptr, nullptr, off, st, s);
+  return run_m<T, false, EPI_STORE, 128, kPair<T>, OutT>(g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d,
+                                                          nullptr, nullptr, off, st, s);
 }
 
 template <typename T>
@@ -1006,15 +1006,16 @@ static moe_status fc2_dgrad(const GemmShape& g, const void* dy_perm, const void*
                                                     2 * g.f, nullptr, H13, off, st, s);
 }
 
-template <typename T>
+template <typename T, typename OutT = T>
 static moe_status fc1_dgrad(const GemmShape& g, const void* dH13, const void* W13,
                             const int32_t* off, void* dx_perm, int* st, cudaStream_t s) {
   // dX = dH13 . W13_e: K = 2f, N = d; B[n, k] = W13[e*2f + k, n] (M/N-major)
   if (g.d % 256 == 0)
-    return run_m<T, true, EPI_STORE, 256, kPair<T>>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
-                                                     dx_perm, g.d, nullptr, nullptr, off, st, s);
-  return run_m<T, true, EPI_STORE, 128, kPair<T>>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
-                                                   dx_perm, g.d, nullptr, nullptr, off, st, s);
+    return run_m<T, true, EPI_STORE, 256, kPair<T>, OutT>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
+                                                           dx_perm, g.d, nullptr, nullptr, off, st,
+                                                           s);
+  return run_m<T, true, EPI_STORE, 128, kPair<T>, OutT>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
+                                                         dx_perm, g.d, nullptr, nullptr, off, st, s);
 }
 
 template <typename T, typename OutT>
@@ -1255,6 +1256,35 @@ static moe_status router_dwr_tc(int T, int d, int E, const void* x, const void* 
                                                      st, s)));
 }
 
+// ------------------------------------------------------------------------ shared expert
+// A dense SwiGLU FFN over all T tokens: the grouped GEMMs with one segment (no offsets),
+// the FC2 output and the FC1 input gradient in fp32 (added into the combine / unpermute).
+template <typename T>
+static moe_status shared_fwd_t(const GemmShape& g1, const void* x, const void* W13s,
+                               const void* W2s, void* H13s, void* as, float* ys, int* st,
+                               cudaStream_t s) {
+  moe_status r = fc1_fwd<T>(g1, x, W13s, nullptr, H13s, as, st, s);
+  if (r != MOE_OK) return r;
+  return fc2_fwd<T, float>(g1, as, W2s, nullptr, ys, st, s);
+}
+
+template <typename T>
+static moe_status shared_bwd_t(const GemmShape& g1, const void* dy, const void* x,
+                               const void* H13s, const void* as, const void* W13s,
+                               const void* W2s, void* dH13s, float* dxs, void* dW13s, void* dW2s,
+                               bool dw_fp32, bool dw_accum, CUtensorMap* maps, int* st,
+                               cudaStream_t s) {
+  moe_status r = build_wgrad_maps<T>(g1, dy, dH13s, nullptr, maps, s);
+  if (r != MOE_OK) return r;
+  r = fc2_dgrad<T>(g1, dy, W2s, H13s, nullptr, dH13s, st, s);
+  if (r != MOE_OK) return r;
+  r = wgrad<T>(g1, dy, g1.d, as, g1.f, dW2s, dw_fp32, dw_accum, nullptr, maps, st, s);
+  if (r != MOE_OK) return r;
+  r = fc1_dgrad<T, float>(g1, dH13s, W13s, nullptr, dxs, st, s);
+  if (r != MOE_OK) return r;
+  return wgrad<T>(g1, dH13s, 2 * g1.f, x, g1.d, dW13s, dw_fp32, dw_accum, nullptr, maps + 1, st, s);
+}
+
 }  // namespace gemm
 
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,
@@ -1325,6 +1355,25 @@ moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, con
   if (r != MOE_OK) return r;
   return gemm::router_dwr_tc(T, d, E, x, dl16, dWr, reinterpret_cast<CUtensorMap*>(maps_ws),
                              status, s);
+}
+
+moe_status shared_fwd(const GemmShape& g, const void* x, const void* W13s, const void* W2s,
+                      void* H13s, void* as, float* ys, int* status, cudaStream_t s) {
+  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false};
+  if (g.fp32) return gemm::shared_fwd_t<float>(g1, x, W13s, W2s, H13s, as, ys, status, s);
+  return gemm::shared_fwd_t<__nv_bfloat16>(g1, x, W13s, W2s, H13s, as, ys, status, s);
+}
+moe_status shared_bwd(const GemmShape& g, const void* dy, const void* x, const void* H13s,
+                      const void* as, const void* W13s, const void* W2s, void* dH13s, float* dxs,
+                      void* dW13s, void* dW2s, bool dw_fp32, bool dw_accum, void* maps_ws,
+                      int* status, cudaStream_t s) {
+  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false};
+  CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_ws);
+  if (g.fp32)
+    return gemm::shared_bwd_t<float>(g1, dy, x, H13s, as, W13s, W2s, dH13s, dxs, dW13s, dW2s,
+                                     dw_fp32, dw_accum, maps, status, s);
+  return gemm::shared_bwd_t<__nv_bfloat16>(g1, dy, x, H13s, as, W13s, W2s, dH13s, dxs, dW13s, dW2s,
+                                           dw_fp32, dw_accum, maps, status, s);
 }
 
 }  // namespace moe

@@ -34,9 +34,11 @@ cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A
 cudaError_t launch_dispatch(bool fp32, int T, int d, int k, const void* x, const int32_t* slot,
                             void* x_perm, int* status, cudaStream_t s);
 // y[t] = sum_j w_tj * src[slot[t,j]] (+ extra[t] fp32 when given); w = gates or all ones.
+// y[t] = extra[t] + extra2[t] + sum_j gates[t,j] * src[slot[t,j]] (fp32 sum; null extras
+// and gates = 1 when gates is null)
 cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, const void* src,
                               const float* gates, const int32_t* slot, const float* extra,
-                              void* y, int* status, cudaStream_t s);
+                              void* y, int* status, cudaStream_t s, const float* extra2 = nullptr);
 // y[i] += extra[i] for n elements (fp32 add, one rounding to the act type)
 cudaError_t launch_add_f32(bool fp32, int64_t n, void* y, const float* extra, cudaStream_t s);
 cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void* dy,
@@ -106,5 +108,15 @@ moe_status router_logits_tc(int T, int d, int E, const void* x, const void* Wr, 
 moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, const void* dl16,
                          float* dx_extra, void* dWr, void* maps_ws, int* status, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(int64_t n, const float* src, void* dst, cudaStream_t s);
+
+// Shared expert (a dense SwiGLU FFN over all g.R = T rows, one segment): forward writes
+// H13s, as (act) and ys [T,d] (float); backward writes dH13s (act scratch), dxs [T,d]
+// (float) and dW13s / dW2s (one expert's slice).  maps_ws: 2 tensor maps of scratch.
+moe_status shared_fwd(const GemmShape& g, const void* x, const void* W13s, const void* W2s,
+                      void* H13s, void* as, float* ys, int* status, cudaStream_t s);
+moe_status shared_bwd(const GemmShape& g, const void* dy, const void* x, const void* H13s,
+                      const void* as, const void* W13s, const void* W2s, void* dH13s, float* dxs,
+                      void* dW13s, void* dW2s, bool dw_fp32, bool dw_accum, void* maps_ws,
+                      int* status, cudaStream_t s);
 
 }  // namespace moe

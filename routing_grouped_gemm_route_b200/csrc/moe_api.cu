@@ -36,6 +36,7 @@ struct WsLayout {
   size_t status, hist, cta_base, maps, dy_perm, dH13, dx_perm, dx_router;
   size_t rc_x_perm, rc_H13, rc_a, rc_y_perm;   // MOE_FLAG_RECOMPUTE: the activations
   size_t dl16;                                  // bf16 copy of d_logits (router, bf16)
+  size_t sh_f32, sh_dH13, rc_sh_H13, rc_sh_a;   // shared expert: y / dx (float), dH13, recompute
   size_t mx_ints, mx_bytes[24];   // MXFP8 operands (codes and scale chunks), see MxWork
   size_t total;
 };
@@ -57,7 +58,13 @@ WsLayout ws_layout(const moe_desc& d) {
   if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.d * 4);
   w.dl16 = o;
   if (d.flags & MOE_FLAG_ROUTER) o = up(o + (size_t)d.T * d.E * 2);
+  const bool sh = d.flags & MOE_FLAG_SHARED_EXPERT;
   const bool rc = d.flags & MOE_FLAG_RECOMPUTE;
+  const size_t T = d.T;
+  w.sh_f32 = o; if (sh) o = up(o + T * d.d * 4);
+  w.sh_dH13 = o; if (sh) o = up(o + T * 2 * (size_t)d.d_ff * es);
+  w.rc_sh_H13 = o; if (sh && rc) o = up(o + T * 2 * (size_t)d.d_ff * es);
+  w.rc_sh_a = o; if (sh && rc) o = up(o + T * (size_t)d.d_ff * es);
   w.rc_x_perm = o; if (rc) o = up(o + R * d.d * es);
   w.rc_H13 = o; if (rc) o = up(o + R * 2 * (size_t)d.d_ff * es);
   w.rc_a = o; if (rc) o = up(o + R * (size_t)d.d_ff * es);
@@ -101,6 +108,10 @@ moe_saved_layout saved_layout(const moe_desc& d) {
   s.H13 = o; if (keep) o = up(o + R * 2 * (size_t)d.d_ff * es);
   s.a = o; if (keep) o = up(o + R * (size_t)d.d_ff * es);
   s.y_perm = o; if (keep) o = up(o + R * d.d * es);
+  // shared expert: its H13 [T,2f] and a [T,f] for the backward
+  const bool sh = keep && (d.flags & MOE_FLAG_SHARED_EXPERT);
+  s.H13_shared = o; if (sh) o = up(o + T * 2 * (size_t)d.d_ff * es);
+  s.a_shared = o; if (sh) o = up(o + T * (size_t)d.d_ff * es);
   s.total = o;
   return s;
 }
@@ -115,8 +126,15 @@ moe_status check(const moe_desc* d) {
   if ((int64_t)d->E * 2 * d->d_ff >= (int64_t(1) << 31) || (int64_t)d->E * d->d >= (int64_t(1) << 31))
     return MOE_EINVAL;
   if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
-  if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE))
+  if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE |
+                   MOE_FLAG_SHARED_EXPERT))
     return MOE_EINVAL;
+  if (d->flags & MOE_FLAG_SHARED_EXPERT) {
+    if (d->dtype == MOE_MXFP8) return MOE_EUNSUPPORTED;
+    if ((int64_t)(d->E + 1) * 2 * d->d_ff >= (int64_t(1) << 31) ||
+        (int64_t)(d->E + 1) * d->d >= (int64_t(1) << 31))
+      return MOE_EINVAL;
+  }
   if ((d->flags & MOE_FLAG_ACCUM_DW) && !(d->flags & MOE_FLAG_DW_FP32)) return MOE_EINVAL;
   if (d->dtype == MOE_MXFP8 && d->d_ff % 128 != 0) return MOE_EUNSUPPORTED;
   return MOE_OK;
@@ -179,10 +197,11 @@ MxWork mx_work(const moe_desc& d, void* ws) {
     if (_st != MOE_OK) return _st;     \
   } while (0)
 
-GemmShape gshape(const moe_desc& d) {
+// rows < 0: the routed rows T*k; else that many rows (the shared expert's T)
+GemmShape gshape(const moe_desc& d, int rows = -1) {
   GemmShape g;
   g.E = d.E;
-  g.R = (int)R_of(d);
+  g.R = rows < 0 ? (int)R_of(d) : rows;
   g.d = d.d;
   g.f = d.d_ff;
   g.fp32 = d.dtype == MOE_FP32;
@@ -450,6 +469,7 @@ moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
 
 struct Acts {
   void *x_perm, *H13, *a, *y_perm;
+  void *H13s, *as;   // shared expert
 };
 Acts acts(const moe_desc& d, const void* saved, const moe_saved_layout& L, void* ws) {
   Acts r;
@@ -459,14 +479,25 @@ Acts acts(const moe_desc& d, const void* saved, const moe_saved_layout& L, void*
     r.H13 = at<char>(ws, w.rc_H13);
     r.a = at<char>(ws, w.rc_a);
     r.y_perm = at<char>(ws, w.rc_y_perm);
+    r.H13s = at<char>(ws, w.rc_sh_H13);
+    r.as = at<char>(ws, w.rc_sh_a);
   } else {
     void* sv = const_cast<void*>(saved);
     r.x_perm = at<char>(sv, L.x_perm);
     r.H13 = at<char>(sv, L.H13);
     r.a = at<char>(sv, L.a);
     r.y_perm = at<char>(sv, L.y_perm);
+    r.H13s = at<char>(sv, L.H13_shared);
+    r.as = at<char>(sv, L.a_shared);
   }
   return r;
+}
+// The shared expert's slice (index E) of W13 / W2 or of their gradients.
+inline const void* w13_slice(const moe_desc& d, const void* W13, size_t es) {
+  return static_cast<const char*>(W13) + (size_t)d.E * 2 * d.d_ff * d.d * es;
+}
+inline const void* w2_slice(const moe_desc& d, const void* W2, size_t es) {
+  return static_cast<const char*>(W2) + (size_t)d.E * d.d * d.d_ff * es;
 }
 
 moe_status moe_load_stats(const int32_t* counts, int32_t E, moe_load_stats_t* out,
@@ -512,7 +543,15 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
   MxWork mx = mx_work(d, ws);
   MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
-  return cu(launch_gather_sum(f32, d.T, d.d, d.k, A.y_perm, gates, slot, nullptr, y, st, s));
+  float* ys = nullptr;
+  if (d.flags & MOE_FLAG_SHARED_EXPERT) {
+    // the shared expert over every token, its output in fp32 for the combine to add
+    const size_t es = act_bytes(d);
+    ys = at<float>(ws, ws_layout(d).sh_f32);
+    MOE_TRY(shared_fwd(gshape(d, d.T), x, w13_slice(d, W13, es), w2_slice(d, W2, es), A.H13s, A.as,
+                       ys, st, s));
+  }
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, A.y_perm, gates, slot, ys, y, st, s));
 }
 
 moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, const void* saved,
@@ -523,9 +562,11 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
   const moe_desc& d = *desc;
   const bool router = d.flags & MOE_FLAG_ROUTER;
   const bool recompute = d.flags & MOE_FLAG_RECOMPUTE;
+  const bool shared = d.flags & MOE_FLAG_SHARED_EXPERT;
+  const size_t es = act_bytes(d);
   MOE_TRY(tptrs(d, {dy, dx, d_logits}));
   MOE_TRY(ptrs({saved, W13, W2, dW13, dW2}));
-  if (router || recompute) MOE_TRY(tptrs(d, {x}));
+  if (router || recompute || shared) MOE_TRY(tptrs(d, {x}));
   if (router) MOE_TRY(ptrs({Wr, dWr}));
   MOE_TRY(ws_ok(d, ws, ws_bytes));
   const moe_saved_layout L = saved_layout(d);
@@ -549,18 +590,39 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
     MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
     MxWork mx = mx_work(d, ws);
     MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+    if (shared)
+      MOE_TRY(shared_fwd(gshape(d, d.T), x, w13_slice(d, W13, es), w2_slice(d, W2, es), A.H13s,
+                         A.as, at<float>(ws, w.sh_f32), st, s));
   }
 
   MOE_TRY(cu(launch_combine_bwd(f32, d.T, d.d, d.k, d.E, dy, A.y_perm, gates, idx, slot, dy_perm,
                                 d_logits, st, s)));
   MOE_TRY(gemm_bwd_body(d, dy_perm, A.x_perm, A.H13, A.a, W13, W2, offsets, dH13, dx_perm, dW13,
                         dW2, ws, s));
+  float* dxs = nullptr;
+  if (shared && d.T > 0) {
+    // the shared expert's backward: dy is its (unpermuted, ungated) output gradient
+    const size_t dw_es = (d.flags & MOE_FLAG_DW_FP32) ? 4 : es;
+    dxs = at<float>(ws, w.sh_f32);
+    MOE_TRY(shared_bwd(gshape(d, d.T), dy, x, A.H13s, A.as, w13_slice(d, W13, es),
+                       w2_slice(d, W2, es), at<char>(ws, w.sh_dH13), dxs,
+                       const_cast<void*>(w13_slice(d, dW13, dw_es)),
+                       const_cast<void*>(w2_slice(d, dW2, dw_es)), d.flags & MOE_FLAG_DW_FP32,
+                       d.flags & MOE_FLAG_ACCUM_DW, at<char>(ws, w.maps), st, s));
+  } else if (shared && !(d.flags & MOE_FLAG_ACCUM_DW)) {
+    // no tokens: the shared expert's weight gradients are zero
+    const size_t dw_es = (d.flags & MOE_FLAG_DW_FP32) ? 4 : es;
+    MOE_TRY(cu(cudaMemsetAsync(const_cast<void*>(w13_slice(d, dW13, dw_es)), 0,
+                               (size_t)2 * d.d_ff * d.d * dw_es, s)));
+    MOE_TRY(cu(cudaMemsetAsync(const_cast<void*>(w2_slice(d, dW2, dw_es)), 0,
+                               (size_t)d.d * d.d_ff * dw_es, s)));
+  }
   float* extra = nullptr;
   if (router) {
     extra = at<float>(ws, w.dx_router);
     MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, ws, s));
   }
-  return cu(launch_gather_sum(f32, d.T, d.d, d.k, dx_perm, nullptr, slot, extra, dx, st, s));
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, dx_perm, nullptr, slot, extra, dx, st, s, dxs));
 }
 
 }  // extern "C"

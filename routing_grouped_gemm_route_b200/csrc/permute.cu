@@ -73,7 +73,8 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(const T* __restri
 template <typename T, int KMAX>
 __global__ void __launch_bounds__(kWarps * 32) gather_sum_kernel(
     const T* __restrict__ src, const float* __restrict__ gates, const int32_t* __restrict__ slot,
-    const float* __restrict__ extra, T* __restrict__ y, int T_, int d, int k, int R, int* status) {
+    const float* __restrict__ extra, const float* __restrict__ extra2, T* __restrict__ y, int T_,
+    int d, int k, int R, int* status) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
   if (t >= T_) return;
@@ -106,6 +107,14 @@ __global__ void __launch_bounds__(kWarps * 32) gather_sum_kernel(
       for (int i = 0; i < V; i += 4) {
         const float4 e4 = *reinterpret_cast<const float4*>(ex + i);
         acc[i] = e4.x; acc[i + 1] = e4.y; acc[i + 2] = e4.z; acc[i + 3] = e4.w;
+      }
+    }
+    if (extra2) {
+      const float* ex = extra2 + (int64_t)t * d + (int64_t)v * V;
+#pragma unroll
+      for (int i = 0; i < V; i += 4) {
+        const float4 e4 = *reinterpret_cast<const float4*>(ex + i);
+        acc[i] += e4.x; acc[i + 1] += e4.y; acc[i + 2] += e4.z; acc[i + 3] += e4.w;
       }
     }
     Vec16<T> in[KMAX];
@@ -267,11 +276,11 @@ cudaError_t launch_dispatch(bool fp32, int T, int d, int k, const void* x, const
 
 template <typename T>
 static void gather_sum_t(int km, int blocks, cudaStream_t s, const void* src, const float* gates,
-                         const int32_t* slot, const float* extra, void* y, int T_, int d, int k,
-                         int R, int* status) {
+                         const int32_t* slot, const float* extra, const float* extra2, void* y,
+                         int T_, int d, int k, int R, int* status) {
 #define MOE_GS(KM)                                                                            \
   gather_sum_kernel<T, KM><<<blocks, kWarps * 32, 0, s>>>((const T*)src, gates, slot, extra, \
-                                                          (T*)y, T_, d, k, R, status)
+                                                          extra2, (T*)y, T_, d, k, R, status)
   switch (km) {
     case 1: MOE_GS(1); break;
     case 2: MOE_GS(2); break;
@@ -285,12 +294,15 @@ static void gather_sum_t(int km, int blocks, cudaStream_t s, const void* src, co
 
 cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, const void* src,
                               const float* gates, const int32_t* slot, const float* extra,
-                              void* y, int* status, cudaStream_t s) {
+                              void* y, int* status, cudaStream_t s, const float* extra2) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kWarps - 1) / kWarps;
   const int km = kmax_of(k);
-  if (fp32) gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, y, T, d, k, T * k, status);
-  else gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, y, T, d, k, T * k, status);
+  if (fp32)
+    gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, T * k, status);
+  else
+    gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, T * k,
+                                status);
   return cudaGetLastError();
 }
 

@@ -44,6 +44,7 @@ class Workload:
     router: bool        # True: logits = x . Wr on the device; False: logits are injected
     skew: bool          # Zipf-skewed expert bias added to the injected logits
     seed: int = 0
+    shared: bool = False  # one shared expert (an extra W13/W2 slice, applied to every token)
 
     @property
     def R(self) -> int:
@@ -88,7 +89,8 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu", seed: int | Non
     Returns a dict of tensors: x [T,d], W13 [E,2*d_ff,d] (rows 0..d_ff-1 gate W1, then up W3),
     W2 [E,d,d_ff], dy [T,d] (upstream gradient), and either Wr [d,E] (router on) or
     logits [T,E] fp32 (injected random routing).  Activations and weights are in the
-    workload's storage dtype; logits are always fp32.
+    workload's storage dtype; logits are always fp32.  With a shared expert W13 and W2
+    have E+1 slices, the last drawn after everything else (so the rest is unchanged).
     """
     device = torch.device(device)
     s = w.seed if seed is None else seed
@@ -118,6 +120,9 @@ def make_inputs(w: Workload, device: str | torch.device = "cpu", seed: int | Non
             logits += zipf_bias(w.E, gb).to(device)
         out["logits"] = logits
     out["dy"] = normal((w.T, w.d))
+    if w.shared:
+        out["W13"] = torch.cat([out["W13"], normal((1, 2 * w.d_ff, w.d), 0.02)])
+        out["W2"] = torch.cat([out["W2"], normal((1, w.d, w.d_ff), 0.02)])
     return out
 
 

@@ -20,6 +20,7 @@ MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE
     0, -1, -2, -3, -4, -5, -6
 MOE_FP32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
 MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW, MOE_FLAG_RECOMPUTE = 1, 2, 4, 8
+MOE_FLAG_SHARED_EXPERT = 16
 MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
@@ -49,7 +50,8 @@ class moe_desc(ctypes.Structure):
 class moe_saved_layout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("topk_idx", "gates", "counts", "offsets", "slot", "row_token", "row_gate",
-                 "logits", "x_perm", "H13", "a", "y_perm", "total")]
+                 "logits", "x_perm", "H13", "a", "y_perm", "H13_shared", "a_shared",
+                 "total")]
 
 
 class moe_load_stats_t(ctypes.Structure):
@@ -324,6 +326,9 @@ def saved_views(desc, saved: torch.Tensor) -> dict:
                    H13=view(L.H13, R * 2 * f, act, (R, 2 * f)),
                    a=view(L.a, R * f, act, (R, f)),
                    y_perm=view(L.y_perm, R * d, act, (R, d)))
+        if desc.flags & MOE_FLAG_SHARED_EXPERT:
+            out.update(H13_shared=view(L.H13_shared, T * 2 * f, act, (T, 2 * f)),
+                       a_shared=view(L.a_shared, T * f, act, (T, f)))
     if desc.flags & MOE_FLAG_ROUTER:
         out["logits"] = view(L.logits, T * E, torch.float32, (T, E))
     return out
@@ -349,11 +354,12 @@ class Layer:
         d = self.desc
         act = act_dtype(d)
         dw_dt = torch.float32 if d.flags & MOE_FLAG_DW_FP32 else act
+        nw = d.E + (1 if d.flags & MOE_FLAG_SHARED_EXPERT else 0)   # weight slices
         if out is None:
             out = dict(dx=torch.empty(d.T, d.d, dtype=act, device=self.device),
                        d_logits=torch.empty(d.T, d.E, dtype=torch.float32, device=self.device),
-                       dW13=torch.empty(d.E, 2 * d.d_ff, d.d, dtype=dw_dt, device=self.device),
-                       dW2=torch.empty(d.E, d.d, d.d_ff, dtype=dw_dt, device=self.device),
+                       dW13=torch.empty(nw, 2 * d.d_ff, d.d, dtype=dw_dt, device=self.device),
+                       dW2=torch.empty(nw, d.d, d.d_ff, dtype=dw_dt, device=self.device),
                        dWr=(torch.empty(d.d, d.E, dtype=act, device=self.device)
                             if d.flags & MOE_FLAG_ROUTER else None))
         moe_layer_bwd(d, dy, x, self.saved, W13, W2, Wr, out["dx"], out["d_logits"], out["dW13"],

@@ -37,6 +37,8 @@ def workload(T, d, E, k, f, dtype="bf16", router=False, skew=False, seed=0):
 def desc_of(w: Workload, flags=0):
     if w.router:
         flags |= lib.MOE_FLAG_ROUTER
+    if w.shared:
+        flags |= lib.MOE_FLAG_SHARED_EXPERT
     return lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
 
 

@@ -53,7 +53,7 @@ def test_descriptor_checks(L, args, code):
 
 
 def test_flag_checks(L):
-    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 16)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 32)) == lib.MOE_EINVAL
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
                                             lib.MOE_FLAG_RECOMPUTE)) == 0
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
@@ -87,6 +87,17 @@ def test_recompute_moves_activations_from_saved_to_workspace(L):
     assert s_r.x_perm == s_r.H13 == s_r.a == s_r.y_perm == s_r.total
     assert s_r.total < 3 * 1024 * 1024                    # routing metadata only
     assert lib.moe_workspace_size(r) - lib.moe_workspace_size(d) >= acts
+
+
+def test_shared_expert_layout_and_checks(L):
+    sh = lib.make_desc(4096, 256, 128, 16, 4, "bf16", lib.MOE_FLAG_SHARED_EXPERT)
+    assert lib.moe_check_desc(sh) == 0
+    s = lib.moe_saved_layout_get(sh)
+    assert s.a_shared - s.H13_shared >= 4096 * 256 * 2 and s.total - s.a_shared >= 4096 * 128 * 2
+    plain = lib.moe_saved_layout_get(lib.make_desc(4096, 256, 128, 16, 4, "bf16"))
+    assert plain.H13_shared == plain.a_shared == plain.total
+    mx = lib.make_desc(4096, 256, 128, 16, 4, "mxfp8", lib.MOE_FLAG_SHARED_EXPERT)
+    assert lib.moe_check_desc(mx) == lib.MOE_EUNSUPPORTED
 
 
 def test_load_stats_struct_layout(L):

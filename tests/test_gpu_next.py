@@ -84,3 +84,56 @@ def test_recompute_is_bit_identical(cuda_lib, T, d, E, k, f, dt, router):
         bwd = oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr)
         assert rel(y1, fwd["y"]) < TOL
         assert rel(g1["dW13"], bwd["dW13"]) < TOL
+
+
+# ------------------------------------------------------------------- shared expert
+
+@pytest.mark.parametrize("T,d,E,k,f,dt,router,flags", [
+    (3000, 256, 16, 4, 128, "bf16", False, 0),
+    (1000, 512, 64, 4, 256, "bf16", True, 0),
+    (700, 256, 8, 2, 128, "bf16", False, lib.MOE_FLAG_RECOMPUTE),
+    (333, 384, 12, 3, 192, "fp32", True, 0),
+    (1200, 256, 8, 2, 128, "bf16", False, lib.MOE_FLAG_DW_FP32),
+])
+def test_shared_expert_layer_matches_oracle(cuda_lib, T, d, E, k, f, dt, router, flags):
+    w = Workload("sh", T, d, E, k, f, dt, router=router, skew=False, seed=T + 5, shared=True)
+    inp = make_inputs(w)
+    desc, layer, dv, y, g, status = run_layer(w, inp, flags=flags)
+    assert status == 0
+    assert g["dW13"].shape[0] == E + 1
+    v = layer.views()
+    x, dy = f64(inp["x"]), f64(inp["dy"])
+    W13, W2 = inp["W13"].float().numpy(), inp["W2"].float().numpy()
+    L = f64(v["logits"]) if router else f64(inp["logits"])
+    Wr = inp["Wr"].float().numpy() if router else None
+    fwd = oracle.layer_fwd(x, W13, W2, logits=L, k=k, shared=True)
+    bwd = oracle.layer_bwd(fwd, dy, x, W13, W2, Wr=Wr)
+    assert np.array_equal(npi(v["topk_idx"]), fwd["topk_idx"])
+    assert rel(y, fwd["y"]) < TOL
+    for name in ("dx", "d_logits", "dW13", "dW2") + (("dWr",) if router else ()):
+        assert rel(g[name], bwd[name]) < TOL, name
+    # the shared expert's own slices, on their own
+    assert rel(g["dW13"][E], bwd["dW13"][E]) < TOL
+    assert rel(g["dW2"][E], bwd["dW2"][E]) < TOL
+    if not flags & lib.MOE_FLAG_RECOMPUTE:
+        assert rel(v["a_shared"], fwd["a_shared"]) < TOL
+
+
+def test_shared_expert_recompute_is_bit_identical(cuda_lib):
+    w = Workload("shrc", 2000, 256, 16, 4, 128, "bf16", router=True, skew=False, seed=77,
+                 shared=True)
+    inp = make_inputs(w)
+    _, lay0, _, y0, g0, st0 = run_layer(w, inp)
+    _, lay1, _, y1, g1, st1 = run_layer(w, inp, flags=lib.MOE_FLAG_RECOMPUTE)
+    assert st0 == 0 and st1 == 0
+    assert torch.equal(y0, y1)
+    for name in ("dx", "d_logits", "dW13", "dW2", "dWr"):
+        assert torch.equal(g0[name], g1[name]), name
+
+
+def test_shared_expert_no_tokens(cuda_lib):
+    w = Workload("sh0", 0, 256, 8, 2, 128, "bf16", router=False, skew=False, seed=1, shared=True)
+    inp = make_inputs(w)
+    _, layer, _, y, g, status = run_layer(w, inp)
+    assert status == 0
+    assert torch.all(g["dW13"] == 0) and torch.all(g["dW2"] == 0)

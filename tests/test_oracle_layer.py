@@ -185,3 +185,53 @@ def test_combine_bwd_softmax_jacobian_rows_sum_to_zero():
     # softmax is invariant to adding a constant to all logits, so each row of dL sums to 0
     assert np.allclose(dL.sum(axis=1), 0.0, atol=1e-13)
     assert np.allclose(dyp[r["slot"][:, 0]], r["gates"][:, :1] * dy, rtol=1e-15, atol=0)
+
+
+# --------------------------------------------------------------- shared expert
+
+def tiny_shared(T=12, d=16, E=4, k=2, f=8, router=False, seed=0):
+    w = Workload("ts", T, d, E, k, f, "fp32", router=router, skew=False, seed=seed, shared=True)
+    inp = make_inputs(w)
+    return w, {n: (None if v is None else v.double().numpy()) for n, v in inp.items()}
+
+
+def test_shared_expert_identical_weights_double_the_dense_ffn():
+    # all routed experts and the shared one equal: gates sum to 1, so y = 2 * FFN(x)
+    w, t = tiny_shared(T=20, d=16, E=5, k=3, f=8, seed=4)
+    W13 = np.repeat(t["W13"][:1], 6, axis=0)
+    W2 = np.repeat(t["W2"][:1], 6, axis=0)
+    fwd = oracle.layer_fwd(t["x"], W13, W2, logits=t["logits"], k=3, shared=True)
+    x = torch.tensor(t["x"])
+    h = x @ torch.tensor(W13[0]).T
+    dense = ((F.silu(h[:, :8]) * h[:, 8:]) @ torch.tensor(W2[0]).T).numpy()
+    assert np.allclose(fwd["y"], 2 * dense, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("router", [False, True])
+def test_shared_expert_bwd_matches_torch_autograd(router):
+    w, t = tiny_shared(T=14, d=16, E=4, k=2, f=8, router=router, seed=9)
+    E = 4
+    fwd = oracle.layer_fwd(t["x"], t["W13"], t["W2"], logits=t["logits"], Wr=t["Wr"], k=2,
+                           shared=True)
+    bwd = oracle.layer_bwd(fwd, t["dy"], t["x"], t["W13"], t["W2"], Wr=t["Wr"])
+    # torch: the routed layer on the first E experts plus a dense SwiGLU FFN on the last
+    x = torch.tensor(t["x"], requires_grad=True)
+    W13 = torch.tensor(t["W13"], requires_grad=True)
+    W2 = torch.tensor(t["W2"], requires_grad=True)
+    Wr = torch.tensor(t["Wr"], requires_grad=True) if router else None
+    Lt = x @ Wr if router else torch.tensor(t["logits"], requires_grad=True)
+    idx = torch.tensor(fwd["topk_idx"], dtype=torch.long)
+    g = torch.softmax(Lt.gather(1, idx), dim=1)
+    h = torch.einsum("tkfd,td->tkf", W13[:E][idx], x)
+    yk = torch.einsum("tkdf,tkf->tkd", W2[:E][idx], F.silu(h[..., :8]) * h[..., 8:])
+    hs = x @ W13[E].T
+    y = (g[..., None] * yk).sum(1) + (F.silu(hs[:, :8]) * hs[:, 8:]) @ W2[E].T
+    (y * torch.tensor(t["dy"])).sum().backward()
+    assert np.allclose(fwd["y"], y.detach().numpy(), rtol=1e-12, atol=1e-14)
+    assert np.allclose(bwd["dx"], x.grad.numpy(), rtol=1e-10, atol=1e-13)
+    assert np.allclose(bwd["dW13"], W13.grad.numpy(), rtol=1e-10, atol=1e-13)
+    assert np.allclose(bwd["dW2"], W2.grad.numpy(), rtol=1e-10, atol=1e-13)
+    if router:
+        assert np.allclose(bwd["dWr"], Wr.grad.numpy(), rtol=1e-10, atol=1e-13)
+    else:
+        assert np.allclose(bwd["d_logits"], Lt.grad.numpy(), rtol=1e-10, atol=1e-13)
