@@ -45,6 +45,9 @@ def parse():
     ap.add_argument("--router", action="store_true", help="compute logits = x.Wr on the device")
     ap.add_argument("--recompute", action="store_true",
                     help="activation recompute: the backward redoes dispatch, FC1 and FC2")
+    ap.add_argument("--capacity", default=None,
+                    help="capacity-padded layout (the comparator of the device-scheduled grouped "
+                         "GEMM): 'auto' = the largest expert count of this routing, or a number")
     ap.add_argument("--shared-expert", action="store_true",
                     help="one shared expert (dense SwiGLU FFN on every token); the step is then "
                          "timed through the whole-layer calls")
@@ -342,9 +345,30 @@ def main():
         (lib.MOE_FLAG_RECOMPUTE if args.recompute else 0) | \
         (lib.MOE_FLAG_SHARED_EXPERT if w.shared else 0)
     desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
+    capacity = 0
+    if args.capacity is not None:
+        if args.capacity == "auto":
+            # the largest count of this routing (read once on the host, before any timing;
+            # the injected logits do not change between steps)
+            probe = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype)
+            lg = inp["logits"]
+            if w.router:
+                lg = torch.empty(w.T, w.E, dtype=torch.float32, device=dev)
+                lib.moe_router_logits(probe, inp["x"], inp["Wr"], lg)
+            pws = lib.alloc_workspace(probe)
+            z32 = lambda *sh, dt=torch.int32: torch.empty(*sh, dtype=dt, device=dev)
+            pc = z32(w.E)
+            lib.moe_route(probe, lg, z32(w.T, w.k), z32(w.T, w.k, dt=torch.float32), pc,
+                          z32(w.E + 1), z32(w.T, w.k), z32(w.T * w.k),
+                          z32(w.T * w.k, dt=torch.float32), pws)
+            capacity = int(pc.max().item())
+            del pws
+        else:
+            capacity = int(args.capacity)
+        desc.capacity = capacity
     act = lib.act_dtype(desc)
     T, d, f, E, k = w.T, w.d, w.d_ff, w.E, w.k
-    R = T * k
+    R = lib.rows_of(desc)
     es = 4 if act == torch.float32 else 2
     ws = lib.alloc_workspace(desc)
 
@@ -459,14 +483,16 @@ def main():
     pk = peaks()
 
     # algorithmic work per stage
-    gemm_flops = {"gemm_fwd": 6.0 * R * d * f, "gemm_bwd": 12.0 * R * d * f,
-                  "re_gemm_fwd": 6.0 * R * d * f}
+    # algorithmic work counts routed rows only (the padded layout's extra rows are waste)
+    Ra = T * k
+    gemm_flops = {"gemm_fwd": 6.0 * Ra * d * f, "gemm_bwd": 12.0 * Ra * d * f,
+                  "re_gemm_fwd": 6.0 * Ra * d * f}
     hbm_bytes = {
-        "route": T * E * 4 + T * k * 12 + R * 8 + 2 * 4 * ((T + 255) // 256) * E,
-        "dispatch": T * d * es + T * k * 4 + R * d * es,
-        "combine": R * d * es + T * k * 8 + T * d * es,
-        "combine_bwd": T * d * es + 2 * R * d * es + T * k * 12 + T * E * 4,
-        "dispatch_bwd": R * d * es + T * k * 4 + T * d * es,
+        "route": T * E * 4 + T * k * 12 + Ra * 8 + 2 * 4 * ((T + 255) // 256) * E,
+        "dispatch": T * d * es + T * k * 4 + Ra * d * es,
+        "combine": Ra * d * es + T * k * 8 + T * d * es,
+        "combine_bwd": T * d * es + 2 * Ra * d * es + T * k * 12 + T * E * 4,
+        "dispatch_bwd": Ra * d * es + T * k * 4 + T * d * es,
     }
     hbm_bytes["re_dispatch"] = hbm_bytes["dispatch"]
     stage_rep = {}
@@ -487,7 +513,7 @@ def main():
         # whole-layer timing: all GEMM flops (routed + shared expert) over the whole step,
         # a lower bound of the GEMM kernels' rate
         gemm_ms = stage_ms["layer_fwd"] + stage_ms["layer_bwd"]
-        gemm_work = 18.0 * (R + T) * d * f
+        gemm_work = 18.0 * (Ra + T) * d * f
     gemm_tflops = gemm_work / (gemm_ms * 1e-3) / 1e12
     peak_tf = pk["bf16_sustained"]
     peak_kind = "sustained dense bf16"
@@ -539,6 +565,9 @@ def main():
             "data": "synthetic (seeded N(0,1) activations/logits, N(0,0.02) weights)",
             "config": {"workload": workload_desc(w), "T": T, "d_model": d, "E": E, "top_k": k,
                        "d_ff": f, "router_on_device": w.router, "recompute": args.recompute, "shared_expert": w.shared,
+                       "layout": (f"capacity-padded: every expert {capacity} rows, "
+                                  f"{E * capacity} rows in all vs {T * k} routed"
+                                  if capacity else "ragged (device-scheduled grouped GEMM)"),
                        "expert_load": load,
                        "parallelism": f"replicas x{world} (data parallel, no data-path collective)",
                        "l2": "no flush: each step's working set (~5 GB of weights, activations "

@@ -28,7 +28,8 @@
  *     for MOE_BF16 and MOE_MXFP8 (MXFP8 quantises inside the grouped GEMM calls).
  *     Logits, gates and d_logits are always float; indices are int32.
  *   - Shapes: T >= 0 tokens, d = d_model (multiple of 128), d_ff (multiple of 64),
- *     1 <= E <= 1024 experts, 1 <= k <= min(E, 32), T*k < 2^31.  R = T*k routed rows.
+ *     1 <= E <= 1024 experts, 1 <= k <= min(E, 32), T*k < 2^31.  R = T*k routed rows
+ *     (E*capacity in the capacity-padded layout, see moe_desc.capacity).
  *   - Argument checks run on the host before any launch and return MOE_EINVAL,
  *     MOE_EALIGN, MOE_EWORKSPACE or MOE_EUNSUPPORTED with nothing launched.  A failed
  *     launch returns MOE_ECUDA.  Data-dependent faults found on the device (an index
@@ -93,6 +94,16 @@ typedef struct moe_desc {
   int32_t T, d, d_ff, E, k;
   int32_t dtype;   /* moe_dtype */
   int32_t flags;   /* MOE_FLAG_* */
+  /* 0: the ragged layout (expert e owns rows [offsets[e], offsets[e+1]), R = T*k rows).
+   * C > 0: the capacity-padded layout the write-ups compare the device-scheduled grouped
+   * GEMM against (deniz.in, "Yeni stack nasıl çalışıyor": padding every expert group to a
+   * common capacity): expert e owns rows [e*C, (e+1)*C), R = E*C; moe_route writes
+   * offsets[e] = e*C (counts stay the true counts), slot = e*C + the token's rank in e,
+   * and marks rows no token fills with row_token = -1, row_gate = 0; dispatch and
+   * combine-bwd zero those rows.  A token whose rank reaches C gets slot -1 and sets
+   * MOE_DEV_BAD_INDEX (choose C >= the largest count; results are then bit-identical to
+   * the ragged layout's).  Every R-sized buffer holds E*C rows. */
+  int32_t capacity;
 } moe_desc;
 
 /* Byte offsets (from the start of the caller's `saved` buffer) of the tensors that

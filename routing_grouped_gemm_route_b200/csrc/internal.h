@@ -31,17 +31,18 @@ cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A
                                bool accumulate, cudaStream_t s);
 
 // ----------------------------------------------------------------------------- permute
-cudaError_t launch_dispatch(bool fp32, int T, int d, int k, const void* x, const int32_t* slot,
-                            void* x_perm, int* status, cudaStream_t s);
+// R: the number of routed rows (slots must be in [0, R)): T*k, or E*capacity padded.
+cudaError_t launch_dispatch(bool fp32, int T, int d, int k, int R, const void* x,
+                            const int32_t* slot, void* x_perm, int* status, cudaStream_t s);
 // y[t] = sum_j w_tj * src[slot[t,j]] (+ extra[t] fp32 when given); w = gates or all ones.
 // y[t] = extra[t] + extra2[t] + sum_j gates[t,j] * src[slot[t,j]] (fp32 sum; null extras
 // and gates = 1 when gates is null)
-cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, const void* src,
+cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, int R, const void* src,
                               const float* gates, const int32_t* slot, const float* extra,
                               void* y, int* status, cudaStream_t s, const float* extra2 = nullptr);
 // y[i] += extra[i] for n elements (fp32 add, one rounding to the act type)
 cudaError_t launch_add_f32(bool fp32, int64_t n, void* y, const float* extra, cudaStream_t s);
-cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void* dy,
+cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, int R, const void* dy,
                                const void* y_perm, const float* gates, const int32_t* topk_idx,
                                const int32_t* slot, void* dy_perm, float* d_logits, int* status,
                                cudaStream_t s);

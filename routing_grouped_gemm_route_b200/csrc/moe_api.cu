@@ -29,7 +29,12 @@ constexpr size_t kAlign = 256;
 inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t act_bytes(const moe_desc& d) { return d.dtype == MOE_FP32 ? 4 : 2; }
-inline int64_t R_of(const moe_desc& d) { return (int64_t)d.T * d.k; }
+// Routed rows: T*k, or E*capacity in the capacity-padded layout (none without tokens).
+inline int64_t R_of(const moe_desc& d) {
+  if (d.T == 0) return 0;
+  return d.capacity > 0 ? (int64_t)d.E * d.capacity : (int64_t)d.T * d.k;
+}
+inline bool padded(const moe_desc& d) { return d.capacity > 0 && d.T > 0; }
 inline cudaStream_t S(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
 struct WsLayout {
@@ -129,6 +134,7 @@ moe_status check(const moe_desc* d) {
   if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE |
                    MOE_FLAG_SHARED_EXPERT))
     return MOE_EINVAL;
+  if (d->capacity < 0 || (int64_t)d->E * d->capacity >= (int64_t(1) << 31)) return MOE_EINVAL;
   if (d->flags & MOE_FLAG_SHARED_EXPERT) {
     if (d->dtype == MOE_MXFP8) return MOE_EUNSUPPORTED;
     if ((int64_t)(d->E + 1) * 2 * d->d_ff >= (int64_t(1) << 31) ||
@@ -210,6 +216,24 @@ GemmShape gshape(const moe_desc& d, int rows = -1) {
 }
 
 // ---------------------------------------------------------------------------- bodies
+// Permutation steps with the layout's row bound; the padded layout first clears the
+// expert buffers its rows scatter into (padding rows must be zero for the weight
+// gradients, which sum over every row of an expert).
+moe_status dispatch_body(const moe_desc& d, const void* x, const int32_t* slot, void* x_perm,
+                         int* st, cudaStream_t s) {
+  const int R = (int)R_of(d);
+  if (padded(d)) MOE_TRY(cu(cudaMemsetAsync(x_perm, 0, (size_t)R * d.d * act_bytes(d), s)));
+  return cu(launch_dispatch(d.dtype == MOE_FP32, d.T, d.d, d.k, R, x, slot, x_perm, st, s));
+}
+moe_status combine_bwd_body(const moe_desc& d, const void* dy, const void* y_perm,
+                            const float* gates, const int32_t* idx, const int32_t* slot,
+                            void* dy_perm, float* d_logits, int* st, cudaStream_t s) {
+  const int R = (int)R_of(d);
+  if (padded(d)) MOE_TRY(cu(cudaMemsetAsync(dy_perm, 0, (size_t)R * d.d * act_bytes(d), s)));
+  return cu(launch_combine_bwd(d.dtype == MOE_FP32, d.T, d.d, d.k, d.E, R, dy, y_perm, gates, idx,
+                               slot, dy_perm, d_logits, st, s));
+}
+
 moe_status route_body(const moe_desc& d, const float* logits, int32_t* idx, float* gates,
                       int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
                       float* row_gate, void* ws, cudaStream_t s) {
@@ -364,8 +388,7 @@ moe_status moe_dispatch(const moe_desc* desc, const void* x, const int32_t* slot
   if (x_perm_sf) return MOE_EINVAL;
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
-  return cu(launch_dispatch(d.dtype == MOE_FP32, d.T, d.d, d.k, x, slot, x_perm, status_ptr(ws),
-                            S(stream)));
+  return dispatch_body(d, x, slot, x_perm, status_ptr(ws), S(stream));
 }
 
 moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const void* x_perm_sf,
@@ -388,8 +411,8 @@ moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* ga
   MOE_TRY(tptrs(*desc, {y_perm, gates, slot, y}));
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
-  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, y_perm, gates, slot, nullptr, y,
-                              status_ptr(ws), S(stream)));
+  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, (int)R_of(d), y_perm, gates,
+                              slot, nullptr, y, status_ptr(ws), S(stream)));
 }
 
 moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_perm,
@@ -400,8 +423,8 @@ moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_p
   MOE_TRY(tptrs(*desc, {dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits}));
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
-  return cu(launch_combine_bwd(d.dtype == MOE_FP32, d.T, d.d, d.k, d.E, dy, y_perm, gates,
-                               topk_idx, slot, dy_perm, d_logits, status_ptr(ws), S(stream)));
+  return combine_bwd_body(d, dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits, status_ptr(ws),
+                          S(stream));
 }
 
 moe_status moe_mx_scale_bytes(int64_t rows, int32_t cols, int32_t num_segments, size_t* bytes) {
@@ -445,8 +468,8 @@ moe_status moe_dispatch_bwd(const moe_desc* desc, const void* dx_perm, const int
   MOE_TRY(tptrs(*desc, {dx_perm, slot, dx}));
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
-  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, dx_perm, nullptr, slot, nullptr,
-                              dx, status_ptr(ws), S(stream)));
+  return cu(launch_gather_sum(d.dtype == MOE_FP32, d.T, d.d, d.k, (int)R_of(d), dx_perm, nullptr,
+                              slot, nullptr, dx, status_ptr(ws), S(stream)));
 }
 
 moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
@@ -540,7 +563,7 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   // the activations the backward reads: in `saved`, or workspace scratch when the
   // backward recomputes them
   const Acts A = acts(d, saved, L, ws);
-  MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
+  MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
   MxWork mx = mx_work(d, ws);
   MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
   float* ys = nullptr;
@@ -551,7 +574,8 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
     MOE_TRY(shared_fwd(gshape(d, d.T), x, w13_slice(d, W13, es), w2_slice(d, W2, es), A.H13s, A.as,
                        ys, st, s));
   }
-  return cu(launch_gather_sum(f32, d.T, d.d, d.k, A.y_perm, gates, slot, ys, y, st, s));
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, (int)R_of(d), A.y_perm, gates, slot, ys, y, st,
+                              s));
 }
 
 moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, const void* saved,
@@ -587,7 +611,7 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
   if (recompute && d.T > 0) {
     // the forward's activations again, from x and the saved routing (same kernels,
     // same inputs: bit-identical to the ones the forward used)
-    MOE_TRY(cu(launch_dispatch(f32, d.T, d.d, d.k, x, slot, A.x_perm, st, s)));
+    MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
     MxWork mx = mx_work(d, ws);
     MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
     if (shared)
@@ -595,8 +619,7 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
                          A.as, at<float>(ws, w.sh_f32), st, s));
   }
 
-  MOE_TRY(cu(launch_combine_bwd(f32, d.T, d.d, d.k, d.E, dy, A.y_perm, gates, idx, slot, dy_perm,
-                                d_logits, st, s)));
+  MOE_TRY(combine_bwd_body(d, dy, A.y_perm, gates, idx, slot, dy_perm, d_logits, st, s));
   MOE_TRY(gemm_bwd_body(d, dy_perm, A.x_perm, A.H13, A.a, W13, W2, offsets, dH13, dx_perm, dW13,
                         dW2, ws, s));
   float* dxs = nullptr;
@@ -622,7 +645,8 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
     extra = at<float>(ws, w.dx_router);
     MOE_TRY(router_bwd_body(d, x, Wr, d_logits, extra, nullptr, dWr, ws, s));
   }
-  return cu(launch_gather_sum(f32, d.T, d.d, d.k, dx_perm, nullptr, slot, extra, dx, st, s, dxs));
+  return cu(launch_gather_sum(f32, d.T, d.d, d.k, (int)R_of(d), dx_perm, nullptr, slot, extra, dx,
+                              st, s, dxs));
 }
 
 }  // extern "C"

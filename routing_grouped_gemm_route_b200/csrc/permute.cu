@@ -260,11 +260,10 @@ cudaError_t launch_f32_to_bf16(int64_t n, const float* src, void* dst, cudaStrea
   return cudaGetLastError();
 }
 
-cudaError_t launch_dispatch(bool fp32, int T, int d, int k, const void* x, const int32_t* slot,
-                            void* x_perm, int* status, cudaStream_t s) {
+cudaError_t launch_dispatch(bool fp32, int T, int d, int k, int R, const void* x,
+                            const int32_t* slot, void* x_perm, int* status, cudaStream_t s) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kWarps - 1) / kWarps;
-  const int R = T * k;
   if (fp32)
     dispatch_kernel<float><<<blocks, kWarps * 32, 0, s>>>((const float*)x, slot, (float*)x_perm, T,
                                                           d, k, R, status);
@@ -292,16 +291,16 @@ static void gather_sum_t(int km, int blocks, cudaStream_t s, const void* src, co
 #undef MOE_GS
 }
 
-cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, const void* src,
+cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, int R, const void* src,
                               const float* gates, const int32_t* slot, const float* extra,
                               void* y, int* status, cudaStream_t s, const float* extra2) {
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kWarps - 1) / kWarps;
   const int km = kmax_of(k);
   if (fp32)
-    gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, T * k, status);
+    gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, R, status);
   else
-    gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, T * k,
+    gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, R,
                                 status);
   return cudaGetLastError();
 }
@@ -326,7 +325,7 @@ static void combine_bwd_t(int km, int blocks, cudaStream_t s, const void* dy, co
 #undef MOE_CB
 }
 
-cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void* dy,
+cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, int R, const void* dy,
                                const void* y_perm, const float* gates, const int32_t* topk_idx,
                                const int32_t* slot, void* dy_perm, float* d_logits, int* status,
                                cudaStream_t s) {
@@ -335,10 +334,10 @@ cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, const void
   const int km = kmax_of(k);
   if (fp32)
     combine_bwd_t<float>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits, T, d,
-                         k, E, T * k, status);
+                         k, E, R, status);
   else
     combine_bwd_t<__nv_bfloat16>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm,
-                                 d_logits, T, d, k, E, T * k, status);
+                                 d_logits, T, d, k, E, R, status);
   return cudaGetLastError();
 }
 

@@ -103,8 +103,10 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float* __restri
 }
 
 // One CTA of 1024 threads: per expert the scan over CTA histograms, then offsets.
+// capacity > 0: the padded layout, offsets[e] = e * capacity instead of the scan.
 __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ hist, int nctas,
-                                                    int E, int32_t* __restrict__ cta_base,
+                                                    int E, int capacity,
+                                                    int32_t* __restrict__ cta_base,
                                                     int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
   __shared__ int s_part[1024];
@@ -145,18 +147,18 @@ __global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ 
     }
     const int incl = s_part[threadIdx.x];
     const int carry = s_carry;
-    if (e < E) offsets[e] = carry + incl - run;
+    if (e < E) offsets[e] = capacity > 0 ? e * capacity : carry + incl - run;
     __syncthreads();
     if (threadIdx.x == 1023) s_carry = carry + incl;
     __syncthreads();
   }
-  if (threadIdx.x == 0) offsets[E] = s_carry;
+  if (threadIdx.x == 0) offsets[E] = capacity > 0 ? E * capacity : s_carry;
 }
 
 __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
     const int32_t* __restrict__ topk_idx, const float* __restrict__ gates,
     const int32_t* __restrict__ offsets, const int32_t* __restrict__ cta_base, int T, int E,
-    int k, int32_t* __restrict__ slot, int32_t* __restrict__ row_token,
+    int k, int capacity, int32_t* __restrict__ slot, int32_t* __restrict__ row_token,
     float* __restrict__ row_gate, int* status) {
   extern __shared__ unsigned s_mem[];
   unsigned* masks = s_mem;                                          // [kWarps][E]
@@ -192,6 +194,12 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
         continue;
       }
       const int s = wbase[warp * E + e] + __popc(masks[warp * E + e] & lower);
+      if (capacity > 0 && s - offsets[e] >= capacity) {
+        // padded layout: the expert's rows are full (the capacity is below its count)
+        set_status(status, MOE_DEV_BAD_INDEX);
+        slot[(int64_t)t * k + j] = -1;
+        continue;
+      }
       slot[(int64_t)t * k + j] = s;
       row_token[s] = t;
       row_gate[s] = gates[(int64_t)t * k + j];
@@ -319,7 +327,8 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   else if (npl <= 16) err = launch_topk<16>(logits, T, E, k, topk_idx, gates, hist, s);
   else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, s);
   if (err != cudaSuccess) return err;
-  scan_kernel<<<1, 1024, 0, s>>>(hist, ctas, E, cta_base, counts, offsets);
+  const int C = d.capacity;
+  scan_kernel<<<1, 1024, 0, s>>>(hist, ctas, E, C, cta_base, counts, offsets);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const size_t smem = size_t(2) * kWarps * E * sizeof(int);
   if (smem > 48 * 1024) {
@@ -327,7 +336,13 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
-  slot_kernel<<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, T, E, k, slot,
+  if (C > 0 && T > 0) {
+    // padded layout: rows no token fills are marked (token -1, gate 0)
+    const size_t rows = (size_t)E * C;
+    if ((err = cudaMemsetAsync(row_token, 0xff, rows * 4, s)) != cudaSuccess) return err;
+    if ((err = cudaMemsetAsync(row_gate, 0, rows * 4, s)) != cudaSuccess) return err;
+  }
+  slot_kernel<<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, T, E, k, C, slot,
                                               row_token, row_gate, status);
   return cudaGetLastError();
 }

@@ -44,7 +44,7 @@ class MoEError(RuntimeError):
 class moe_desc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int32), ("d", ctypes.c_int32), ("d_ff", ctypes.c_int32),
                 ("E", ctypes.c_int32), ("k", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("capacity", ctypes.c_int32)]
 
 
 class moe_saved_layout(ctypes.Structure):
@@ -136,8 +136,16 @@ def _check(st: int, what: str):
         raise MoEError(st, what)
 
 
-def make_desc(T, d, d_ff, E, k, dtype="bf16", flags=0) -> moe_desc:
-    return moe_desc(T, d, d_ff, E, k, DTYPES[dtype] if isinstance(dtype, str) else dtype, flags)
+def make_desc(T, d, d_ff, E, k, dtype="bf16", flags=0, capacity=0) -> moe_desc:
+    return moe_desc(T, d, d_ff, E, k, DTYPES[dtype] if isinstance(dtype, str) else dtype, flags,
+                    capacity)
+
+
+def rows_of(desc: moe_desc) -> int:
+    """Routed rows R: T*k, or E*capacity in the capacity-padded layout (0 without tokens)."""
+    if desc.T == 0:
+        return 0
+    return desc.E * desc.capacity if desc.capacity > 0 else desc.T * desc.k
 
 
 def act_dtype(desc: moe_desc) -> torch.dtype:
@@ -307,7 +315,7 @@ def saved_views(desc, saved: torch.Tensor) -> dict:
     """Typed views of the tensors moe_layer_fwd keeps in ``saved``."""
     L = moe_saved_layout_get(desc)
     T, k, E, d, f = desc.T, desc.k, desc.E, desc.d, desc.d_ff
-    R = T * k
+    R = rows_of(desc)
     act = act_dtype(desc)
 
     def view(off, n, dt, shape):

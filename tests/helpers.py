@@ -54,8 +54,8 @@ def run_route(desc, logits_dev):
                counts=torch.empty(E, dtype=torch.int32, device=dev),
                offsets=torch.empty(E + 1, dtype=torch.int32, device=dev),
                slot=torch.empty(T, k, dtype=torch.int32, device=dev),
-               row_token=torch.empty(T * k, dtype=torch.int32, device=dev),
-               row_gate=torch.empty(T * k, dtype=torch.float32, device=dev))
+               row_token=torch.empty(lib.rows_of(desc), dtype=torch.int32, device=dev),
+               row_gate=torch.empty(lib.rows_of(desc), dtype=torch.float32, device=dev))
     ws = lib.alloc_workspace(desc)
     lib.moe_route(desc, logits_dev, out["topk_idx"], out["gates"], out["counts"], out["offsets"],
                   out["slot"], out["row_token"], out["row_gate"], ws)
@@ -76,9 +76,10 @@ def assert_route_equal(gpu: dict, ref: dict, k: int):
     assert np.array_equal(f64(gpu["row_gate"])[npi(gpu["slot"])], g)
 
 
-def run_layer(w: Workload, inp: dict, flags=0):
+def run_layer(w: Workload, inp: dict, flags=0, capacity=0):
     """Layer fwd+bwd through moe_layer_fwd / moe_layer_bwd on the device."""
     desc = desc_of(w, flags)
+    desc.capacity = capacity
     layer = lib.Layer(desc)
     dv = to_dev(inp)
     y = layer.fwd(dv["x"], dv["W13"], dv["W2"], logits=dv["logits"], Wr=dv["Wr"])

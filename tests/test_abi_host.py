@@ -100,6 +100,20 @@ def test_shared_expert_layout_and_checks(L):
     assert lib.moe_check_desc(mx) == lib.MOE_EUNSUPPORTED
 
 
+def test_capacity_padded_layout_sizes(L):
+    T, d, f, E, k = 4096, 256, 128, 16, 4
+    ragged = lib.make_desc(T, d, f, E, k, "bf16")
+    padded = lib.make_desc(T, d, f, E, k, "bf16", capacity=1500)
+    assert lib.moe_check_desc(padded) == 0
+    assert lib.rows_of(padded) == E * 1500 and lib.rows_of(ragged) == T * k
+    sp = lib.moe_saved_layout_get(padded)
+    assert sp.H13 - sp.x_perm >= E * 1500 * d * 2
+    assert lib.moe_workspace_size(padded) > lib.moe_workspace_size(ragged)
+    assert lib.moe_check_desc(lib.make_desc(T, d, f, E, k, "bf16", capacity=-1)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(T, d, f, E, k, "bf16", capacity=1 << 28)) == \
+        lib.MOE_EINVAL
+
+
 def test_load_stats_struct_layout(L):
     # the C struct: int64 total, four int32, three doubles
     assert lib.LOAD_STATS_BYTES == 48

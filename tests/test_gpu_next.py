@@ -137,3 +137,59 @@ def test_shared_expert_no_tokens(cuda_lib):
     _, layer, _, y, g, status = run_layer(w, inp)
     assert status == 0
     assert torch.all(g["dW13"] == 0) and torch.all(g["dW2"] == 0)
+
+
+# ------------------------------------------------------- capacity-padded comparator
+
+def max_count(w, inp):
+    desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype)
+    L = inp["logits"] if inp["logits"] is not None else None
+    r = run_route(desc, L.cuda())
+    return int(r["counts"].max().item()), r
+
+
+def test_padded_routing_layout(cuda_lib):
+    w = Workload("cap", 3000, 256, 16, 4, 128, "bf16", router=False, skew=True, seed=11)
+    inp = make_inputs(w)
+    C, rr = max_count(w, inp)
+    desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, "bf16", capacity=C + 5)
+    rp = run_route(desc, inp["logits"].cuda())
+    E, Cp = w.E, C + 5
+    assert torch.equal(rp["counts"], rr["counts"])
+    assert np.array_equal(npi(rp["offsets"]), np.arange(E + 1) * Cp)
+    idx, off = npi(rr["topk_idx"]), npi(rr["offsets"])
+    # slot = e*C + (the token's rank in e), the rank being the ragged slot minus offsets[e]
+    assert np.array_equal(npi(rp["slot"]), idx * Cp + npi(rr["slot"]) - off[idx])
+    rt = npi(rp["row_token"]).reshape(E, Cp)
+    cnt = npi(rr["counts"])
+    for e in range(E):
+        assert np.array_equal(rt[e, :cnt[e]], npi(rr["row_token"])[off[e]:off[e + 1]])
+        assert np.all(rt[e, cnt[e]:] == -1)
+
+
+@pytest.mark.parametrize("T,d,E,k,f,dt,skew,router,shared", [
+    (3000, 256, 16, 4, 128, "bf16", False, False, False),
+    (3000, 256, 16, 4, 128, "bf16", True, False, False),
+    (1500, 256, 8, 4, 128, "mxfp8", False, False, False),
+    (333, 384, 12, 3, 192, "fp32", False, False, False),
+    (1000, 256, 64, 4, 128, "bf16", False, True, True),
+])
+def test_padded_layer_is_bit_identical_to_ragged(cuda_lib, T, d, E, k, f, dt, skew, router,
+                                                 shared):
+    w = Workload("pad", T, d, E, k, f, dt, router=router, skew=skew, seed=T + 9, shared=shared)
+    inp = make_inputs(w)
+    _, lay0, _, y0, g0, st0 = run_layer(w, inp)
+    C = int(lay0.views()["counts"].max().item())
+    _, lay1, _, y1, g1, st1 = run_layer(w, inp, capacity=C)
+    assert st0 == 0 and st1 == 0
+    assert torch.equal(y0, y1)
+    for name in ("dx", "d_logits", "dW13", "dW2") + (("dWr",) if router else ()):
+        assert torch.equal(g0[name], g1[name]), name
+
+
+def test_capacity_below_the_largest_count_is_reported(cuda_lib):
+    w = Workload("capx", 2000, 256, 16, 4, 128, "bf16", router=False, skew=True, seed=3)
+    inp = make_inputs(w)
+    C, _ = max_count(w, inp)
+    desc, layer, dv, y, g, status = run_layer(w, inp, capacity=C - 1)
+    assert status & lib.MOE_DEV_BAD_INDEX
