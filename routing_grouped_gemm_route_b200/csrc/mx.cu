@@ -129,15 +129,14 @@ __device__ __forceinline__ void staged32(const uint8_t* p, uint32_t* w) {
 }
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-// max |x| over packed bf16 pairs, pairwise (exact: the result is one of the inputs)
-__device__ __forceinline__ __nv_bfloat162 absmax2(__nv_bfloat162 m, uint32_t w) {
-  return __hmax2(m, __habs2(*reinterpret_cast<const __nv_bfloat162*>(&w)));
-}
+// |x| of both bf16 halves (the sign bits cleared).  Non-negative IEEE values order like
+// their bit patterns, so a per-half unsigned max of |x| bits is the exact max |x|.
+__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7fff7fffu; }
 __device__ __forceinline__ float amax32(const uint32_t* w) {
-  __nv_bfloat162 m = __float2bfloat162_rn(0.f);
+  uint32_t m = 0u;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) m = absmax2(m, w[i]);
-  return fmaxf(__low2float(m), __high2float(m));
+  for (int i = 0; i < 16; ++i) m = __vmaxu2(m, abs2(w[i]));
+  return fmaxf(bf_lo(m), bf_hi(m));
 }
 
 // 32 codes of the packed bf16 w[] times m[j] (PER_ELEM) or m[0] -> two 16-byte stores
@@ -214,6 +213,7 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
   }
   const int W = C / 128;
   const int row = t & 31, q = t >> 5;         // this thread's row and 32-column block
+  const int lane = t & 31;
   int it = 0;
   for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
     const int b = it % kQBufs;
@@ -222,7 +222,9 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
     if (t < 32 && ahead < ntiles) issue(ahead, (it + kQBufs - 1) % kQBufs);
     const bool ok = mbar_wait(&bar[b], (it / kQBufs) & 1u,
                               reinterpret_cast<volatile int*>(&abort_flag), status);
-    if (__syncthreads_or(!ok)) break;
+    // every step below is warp-local; the barrier at the end releases the buffer (and
+    // agrees on an abort)
+    if (ok) {
     const TilePos tp = pos[b];
     const int c0 = (tile % ctiles) * kQCols;
     const int ncols = min(kQCols, C - c0);
@@ -243,38 +245,42 @@ __global__ void __launch_bounds__(256, 4) quant_tile_kernel(
       sf_r[sf_byte((tile0 + p / 128) * W + col / 128, p, (col & 127) >> 5)] =
           static_cast<uint8_t>(s + 127);
     }
-    if (COL) {
-      if (2 * t < ncols) {
-        // columns 2t and 2t+1; rows past the segment's end take no part (they hold
-        // whatever the buffer had: masked out)
-        __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
+    if (COL && q * 32 < ncols) {   // warp-uniform: this warp's 32-column block exists
+      // The warp holds the block's 32 rows (one per lane; rows past the segment's end
+      // are masked to zero).  A butterfly reduce-scatter of |x| over the lanes leaves
+      // lane L with the max of column L: each step halves the words a lane keeps.
+      uint32_t a[16];
 #pragma unroll
-        for (int r = 0; r < kQRows; ++r) {
-          const uint32_t w = *reinterpret_cast<const uint32_t*>(tb + r * kQPitch + 4 * t);
-          m2 = absmax2(m2, r < tp.nrows ? w : 0u);
-        }
-        const int64_t chunk = (tile0 + tp.p0 / 128) * W + (c0 + 2 * t) / 128;
-        const int blk = (tp.p0 & 127) >> 5;
-        const bool last = tp.p0 + 32 >= seg_rows(g, tp.e);
+      for (int i = 0; i < 16; ++i) a[i] = active ? abs2(v[i]) : 0u;
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int s = mx_exponent(h ? __high2float(m2) : __low2float(m2));
-          const int col = c0 + 2 * t + h;
-          col_m[2 * t + h] = exp2_neg(s);
-          sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
-          // The segment's last chunk may hold fewer than four blocks.  A K-stage of a
-          // wgrad GEMM still reads all four scales (its rows past the segment are zero
-          // codes), so the absent blocks get the finite scale 2^-127 rather than whatever
-          // the buffer held (0xFF = NaN).
-          if (last)
-            for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
+      for (int m = 16; m >= 2; m >>= 1) {
+        const bool up = (lane & m) != 0;
+#pragma unroll
+        for (int i = 0; i < m / 2; ++i) {
+          const uint32_t send = up ? a[i] : a[i + m / 2];
+          const uint32_t keep = up ? a[i + m / 2] : a[i];
+          a[i] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, m));
         }
       }
-      __syncthreads();
+      const uint32_t mm = __vmaxu2(a[0], __shfl_xor_sync(0xffffffffu, a[0], 1));
+      const int s = mx_exponent((lane & 1) ? bf_hi(mm) : bf_lo(mm));
+      const int col = c0 + q * 32 + lane;
+      col_m[q * 32 + lane] = exp2_neg(s);
+      const int64_t chunk = (tile0 + tp.p0 / 128) * W + col / 128;
+      const int blk = (tp.p0 & 127) >> 5;
+      sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
+      // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad
+      // GEMM still reads all four scales (its rows past the segment are zero codes), so
+      // the absent blocks get the finite scale 2^-127 rather than whatever the buffer
+      // held (0xFF = NaN).
+      if (tp.p0 + 32 >= seg_rows(g, tp.e))
+        for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
+      __syncwarp();
       if (active)
         store_codes32<true>(codes_c + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, col_m + q * 32);
     }
-    __syncthreads();   // this buffer and col_m free for reuse
+    }
+    if (__syncthreads_or(!ok)) break;   // this buffer and col_m free for reuse
   }
   // After an abort, the copies still in flight (iterations it .. it+kQBufs-1 that have a
   // tile) must land before the CTA exits.
