@@ -258,8 +258,11 @@ def run_reference(args, w, world, rank):
 
 def run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d_logits, dW13,
             dW2, dWr):
-    """Same metric through the public whole-layer calls, with the step's inputs copied
-    from pinned host memory and its results copied back, all inside the timed region."""
+    """Same metric through the public whole-layer calls, with every step's inputs copied
+    from pinned host memory and its results (y, dx) copied back, all inside the timed
+    region.  The copies run on two copy streams, double-buffered: step i+1's inputs move
+    to the device and step i-1's results to the host while step i computes, as a
+    training loop would feed the layer."""
     from routing_grouped_gemm_route_b200 import lib
     T, d, E = w.T, w.d, w.E
     es = 4 if act == torch.float32 else 2
@@ -267,39 +270,73 @@ def run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d
 
     def z(*shape, dt=act):
         return torch.empty(*shape, dtype=dt, device=dev)
-    hx = torch.empty(T, d, dtype=act, pin_memory=True)
-    hx.copy_(x.cpu())
-    hdy = torch.empty(T, d, dtype=act, pin_memory=True)
-    hdy.copy_(dy.cpu())
-    hl = None
-    if not w.router:
-        hl = torch.empty(T, E, dtype=torch.float32, pin_memory=True)
-        hl.copy_(logits.cpu())
-    hy = torch.empty(T, d, dtype=act, pin_memory=True)
-    hdx = torch.empty(T, d, dtype=act, pin_memory=True)
+
+    def pinned(src, dt=act):
+        h = torch.empty(*src.shape, dtype=dt, pin_memory=True)
+        h.copy_(src.cpu())
+        return h
+    hx, hdy = pinned(x), pinned(dy)
+    hl = None if w.router else pinned(logits, torch.float32)
+    hy = [torch.empty(T, d, dtype=act, pin_memory=True) for _ in range(2)]
+    hdx = [torch.empty(T, d, dtype=act, pin_memory=True) for _ in range(2)]
     layer = lib.Layer(desc, device=dev)
-    x_in, dl_in, dy_in = z(T, d), (z(T, E, dt=torch.float32) if not w.router else None), z(T, d)
-    outs = dict(dx=dx, d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
+    x_in = [z(T, d) for _ in range(2)]
+    dy_in = [z(T, d) for _ in range(2)]
+    dl_in = [None if w.router else z(T, E, dt=torch.float32) for _ in range(2)]
+    y_out = [y, z(T, d)]
+    dx_out = [dx, z(T, d)]
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    ev = lambda: torch.cuda.Event()
+    in_done = [ev(), ev()]        # inputs of buffer b on the device
+    used = [ev(), ev()]           # step on buffer b finished reading its inputs / writing
+    out_done = [ev(), ev()]       # results of buffer b on the host
 
-    def e2e_step():
-        x_in.copy_(hx, non_blocking=True)
-        if dl_in is not None:
-            dl_in.copy_(hl, non_blocking=True)
-        dy_in.copy_(hdy, non_blocking=True)
-        layer.fwd(x_in, W13, W2, logits=dl_in, Wr=Wr, y=y)
-        layer.bwd(dy_in, W13, W2, x=x_in, Wr=Wr, out=outs)
-        hy.copy_(y, non_blocking=True)
-        hdx.copy_(dx, non_blocking=True)
+    def copy_in(i):
+        b = i % 2
+        with torch.cuda.stream(s_in):
+            if i >= 2:
+                s_in.wait_event(used[b])       # step i-2 no longer reads these buffers
+            x_in[b].copy_(hx, non_blocking=True)
+            if dl_in[b] is not None:
+                dl_in[b].copy_(hl, non_blocking=True)
+            dy_in[b].copy_(hdy, non_blocking=True)
+            in_done[b].record(s_in)
 
-    for _ in range(2):
-        e2e_step()
+    def compute(i):
+        b = i % 2
+        comp.wait_event(in_done[b])
+        if i >= 2:
+            comp.wait_event(out_done[b])       # step i-2's results have left y/dx[b]
+        outs = dict(dx=dx_out[b], d_logits=d_logits, dW13=dW13, dW2=dW2, dWr=dWr)
+        layer.fwd(x_in[b], W13, W2, logits=dl_in[b], Wr=Wr, y=y_out[b])
+        layer.bwd(dy_in[b], W13, W2, x=x_in[b], Wr=Wr, out=outs)
+        used[b].record(comp)
+
+    def copy_out(i):
+        b = i % 2
+        with torch.cuda.stream(s_out):
+            s_out.wait_event(used[b])
+            hy[b].copy_(y_out[b], non_blocking=True)
+            hdx[b].copy_(dx_out[b], non_blocking=True)
+            out_done[b].record(s_out)
+
+    def run(n):
+        copy_in(0)
+        for i in range(n):
+            if i + 1 < n:
+                copy_in(i + 1)
+            compute(i)
+            copy_out(i)
+
+    run(2)                                     # warm-up
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(E2E):
-        e2e_step()
-    e1.record()
+    e0.record(s_in)                            # before the first input copy
+    run(E2E)
+    comp.wait_stream(s_out)
+    e1.record(comp)                            # after the last result copy
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world)
@@ -307,10 +344,10 @@ def run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d
     d2h = T * d * es * 2
     e2e = {"value": world * T * E2E / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": E2E,
-           "api": "moe_layer_fwd + moe_layer_bwd with pinned-host x, logits, dy in and y, dx out"}
+           "api": "moe_layer_fwd + moe_layer_bwd; pinned-host x, logits, dy in and y, dx out "
+                  "every step on two copy streams, double-buffered against the compute"}
     if lib.moe_read_device_status(layer.ws) != 0:
         raise RuntimeError("device status set during the end-to-end run")
-
     return e2e
 
 
