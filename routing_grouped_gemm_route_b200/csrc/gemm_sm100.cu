@@ -127,7 +127,10 @@ struct Cfg {
   // activation type: bf16 for the 16-bit and MXFP8 kernels); the dH1/dH3 results are
   // staged in place in the slot they were computed from
   static constexpr int AES = ES == 4 ? 4 : 2;
-  static constexpr int IN_SLOTS = EPI == EPI_SWIGLU_BWD ? (AES == 2 ? (WCH < 2 ? WCH : 2) : 1) : 0;
+  // (one slot per warp: each warp's H1/H3 chunk loads overlap its previous chunk's math,
+  // and the 32 KB saved buy the operand ring a fifth stage, which the main loop needs
+  // more -- with four it waits on its loads a third of the time)
+  static constexpr int IN_SLOTS = EPI == EPI_SWIGLU_BWD ? 1 : 0;
   static constexpr int IN_CH = 2 * 32 * 32 * AES;
   static constexpr int EPI_WARP = ((NBUF * CH + IN_SLOTS * IN_CH) + 1023) / 1024 * 1024;
   static constexpr int EPI_BYTES = EPI_WARPS * EPI_WARP;
@@ -369,6 +372,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
+      int acquired_e = -1;   // RAGGED_K: expert whose A tensor map was last acquired
       int stage = 0;
       uint32_t phase = 0;
       uint32_t armed = 0, armed_par = 0;
@@ -430,7 +434,12 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
             }
           } else {
             const CUtensorMap* am = p.a_maps + tl.e;
-            if (kb == 0) fence_tmap_acquire(am);   // written by the map-building kernel
+            // written by the map-building kernel: acquired once per expert (consecutive
+            // tiles share it)
+            if (kb == 0 && tl.e != acquired_e) {
+              fence_tmap_acquire(am);
+              acquired_e = tl.e;
+            }
 #pragma unroll
             for (int i = 0; i < BM / C::MNB; ++i)
               load(sA + i * C::KB * 128, am, tl.m0 + arow + i * C::MNB, tl.row0 + k0);
