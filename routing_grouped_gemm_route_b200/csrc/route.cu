@@ -35,8 +35,14 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
+// Top-k runs up to 32 warps per 256-token CTA (8 tokens a warp): the CTA granularity is
+// the scan's and the slot kernel's, the extra warps hide latency.  Above 256 experts a
+// lane's logits need more registers than 32 warps a CTA allow: 8 warps there.
+template <int NPL>
+constexpr int topk_warps() { return NPL <= 8 ? 32 : 8; }
+
 template <int NPL>   // logits per lane = ceil(E / 32)
-__global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float* __restrict__ logits,
+__global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const float* __restrict__ logits,
                                                            int T, int E, int k,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ gates,
@@ -46,8 +52,8 @@ __global__ void __launch_bounds__(kWarps * 32) topk_kernel(const float* __restri
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
 
-  const int t0 = blockIdx.x * kRouteTokensPerCta + warp * 32;
-  for (int i = 0; i < 32; ++i) {
+  const int t0 = blockIdx.x * kRouteTokensPerCta;
+  for (int i = warp; i < kRouteTokensPerCta; i += topk_warps<NPL>()) {
     const int t = t0 + i;
     if (t >= T) break;
     const float* row = logits + (int64_t)t * E;
@@ -211,7 +217,8 @@ template <int NPL>
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gates,
                         int32_t* hist, cudaStream_t s) {
   const int ctas = route_ctas(T);
-  topk_kernel<NPL><<<ctas, kWarps * 32, E * sizeof(int), s>>>(logits, T, E, k, idx, gates, hist);
+  topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, E * sizeof(int), s>>>(logits, T, E, k, idx,
+                                                                        gates, hist);
   return cudaGetLastError();
 }
 
