@@ -259,6 +259,41 @@ __device__ __forceinline__ void staged_store(uint8_t* buf, const float* v, int l
   }
 }
 
+// The same for a chunk row already packed to bf16 (16 words = 32 values).
+template <int NBUF>
+__device__ __forceinline__ void staged_store_packed(uint8_t* buf, const uint32_t* w, int lane,
+                                                    const void* tmap, int x, int y) {
+  if (lane == 0) bulk_wait_read<NBUF - 1>();
+  __syncwarp();
+  uint8_t* row = buf + lane * 64;
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    *reinterpret_cast<uint4*>(row + swz_chunk<bf16>(j, lane) * 16) =
+        make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]);
+  fence_proxy_async_smem();
+  __syncwarp();
+  if (lane == 0) {
+    tma_store_2d(tmap, buf, x, y);
+    bulk_commit();
+  }
+}
+// 32 floats rounded to bf16 (nearest even), packed two to a word.
+__device__ __forceinline__ void pack_bf16x32(const float* v, uint32_t* w) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    Vec16<bf16> pk;
+    pk.from_float(v + 8 * j);
+    w[4 * j] = pk.raw.x;
+    w[4 * j + 1] = pk.raw.y;
+    w[4 * j + 2] = pk.raw.z;
+    w[4 * j + 3] = pk.raw.w;
+  }
+}
+__device__ __forceinline__ void store_packed32(bf16* dst, const uint32_t* w) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) stg16(dst + 8 * j, make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
+}
+
 template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
 __global__ void __launch_bounds__(Cfg<T, OutT, BN, EPI, PAIR, MODE>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -571,6 +606,96 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
+      if constexpr (C::NACC == 1 && EPI != EPI_SWIGLU_BWD && sizeof(OutT) == 2) {
+        // One accumulator: the next tile's MMAs wait for it.  Pull this warp's columns
+        // into registers (rounded to the bf16 outputs), free the accumulator, and only
+        // then stage and store them, so the stores overlap the next tile's main loop.
+        constexpr int RCH = EPI == EPI_SWIGLU_FWD ? (BN / 2 / C::COLGRP) / 32 : C::WCH;
+        uint32_t pk[EPI == EPI_SWIGLU_FWD ? 3 : 1][RCH][16];
+        const int c_sw = cg * RCH * 32;     // SwiGLU: my first gate (and up) column
+        bool any = true;                    // RAGGED_K: this tile has rows (else dW = 0)
+        if (MODE == RAGGED_K) any = tl.kb > 0;
+#pragma unroll
+        for (int i = 0; i < RCH; ++i) {
+          if (EPI == EPI_SWIGLU_FWD) {
+            uint32_t v3[32];
+            float h3[32], av[32];
+            tmem_ld32(tb + c_sw + 32 * i, v);
+            tmem_ld32(tb + BN / 2 + c_sw + 32 * i, v3);
+            tmem_ld_wait();
+            reg_fence32(v);
+            reg_fence32(v3);
+            bits_to_f32(v, fv);
+            bits_to_f32(v3, h3);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) av[j] = fv[j] * sigmoid_f(fv[j]) * h3[j];
+            pack_bf16x32(fv, pk[0][i]);
+            pack_bf16x32(h3, pk[EPI == EPI_SWIGLU_FWD ? 1 : 0][i]);
+            pack_bf16x32(av, pk[EPI == EPI_SWIGLU_FWD ? 2 : 0][i]);
+          } else {
+            if (any) {
+              tmem_ld32(tb + (cfirst + i) * 32, v);
+              tmem_ld_wait();
+              reg_fence32(v);
+              bits_to_f32(v, fv);
+            } else {
+#pragma unroll
+              for (int j = 0; j < 32; ++j) fv[j] = 0.f;
+            }
+            pack_bf16x32(fv, pk[0][i]);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (PAIR) mbar_arrive_remote(tempty_leader + static_cast<uint32_t>(acc) * 8u);
+          else mbar_arrive(&tempty[acc]);
+        }
+        if (MODE == RAGGED_M) {
+          const int64_t grow = rbase + lane;
+          const bool valid = lane < nvalid;
+          if (nvalid > 0) {
+#pragma unroll
+            for (int i = 0; i < RCH; ++i) {
+              if (EPI == EPI_SWIGLU_FWD) {
+                const int hc = tl.n0 / 2 + c_sw + 32 * i;   // H1/a column
+                if (whole) {
+                  staged_store_packed<C::NBUF>(stage_buf + 0 * C::CH, pk[0][i], lane, &tmO, hc, rbase);
+                  staged_store_packed<C::NBUF>(stage_buf + 1 * C::CH, pk[EPI == EPI_SWIGLU_FWD ? 1 : 0][i],
+                                               lane, &tmO, p.f + hc, rbase);
+                  staged_store_packed<C::NBUF>(stage_buf + 2 * C::CH, pk[EPI == EPI_SWIGLU_FWD ? 2 : 0][i],
+                                               lane, &tmO2, hc, rbase);
+                } else if (valid) {
+                  bf16* h13 = reinterpret_cast<bf16*>(p.out) + grow * (2 * (int64_t)p.f) + hc;
+                  store_packed32(h13, pk[0][i]);
+                  store_packed32(h13 + p.f, pk[EPI == EPI_SWIGLU_FWD ? 1 : 0][i]);
+                  store_packed32(reinterpret_cast<bf16*>(p.out_a) + grow * (int64_t)p.f + hc,
+                                 pk[EPI == EPI_SWIGLU_FWD ? 2 : 0][i]);
+                }
+              } else {
+                const int c = (cfirst + i) * 32;
+                if (whole) {
+                  staged_store_packed<C::NBUF>(stage_buf + sbuf * C::CH, pk[0][i], lane, &tmO,
+                                               tl.n0 + c, rbase);
+                  sbuf = sbuf + 1 == C::NBUF ? 0 : sbuf + 1;
+                } else if (valid) {
+                  store_packed32(reinterpret_cast<bf16*>(p.out) + grow * p.ldo + tl.n0 + c, pk[0][i]);
+                }
+              }
+            }
+          }
+        } else {
+          const int y = tl.e * p.M + tl.m0 + myrow + q * 32;
+#pragma unroll
+          for (int i = 0; i < RCH; ++i) {
+            staged_store_packed<C::NBUF>(stage_buf + sbuf * C::CH, pk[0][i], lane, &tmO,
+                                         tl.n0 + (cfirst + i) * 32, y);
+            sbuf = sbuf + 1 == C::NBUF ? 0 : sbuf + 1;
+          }
+        }
+        if (++acc == C::NACC) { acc = 0; acc_phase ^= 1u; }
+        continue;
+      }
       if (MODE == RAGGED_M) {
         const int64_t grow = rbase + lane;
         const bool valid = lane < nvalid;
