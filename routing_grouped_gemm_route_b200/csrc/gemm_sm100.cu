@@ -8,21 +8,27 @@
 // memory, builds the tile list itself and walks it; the host never learns the
 // per-expert sizes.
 //
-// Kernel structure (one CTA per SM):
+// Kernel structure (one CTA per SM; the 16-bit and MXFP8 kernels run as CTA pairs,
+// cta_group::2, on 256-row tiles):
 //   warp 0      TMA producer: 128-byte-swizzled operand tiles into a ring of stages
-//   warp 1      tcgen05.mma issuer (one thread) + tensor-memory allocation
-//   warps 2..   epilogue (4 warps, 8 for the math-heavy SwiGLU backward: two per
-//               tensor-memory lane quadrant, splitting the columns): tensor memory ->
-//               registers -> fused math -> swizzled shared memory -> TMA bulk tensor
-//               stores, one 32x32 chunk at a time
+//               (MXFP8: plus each stage's 512-byte scale chunks)
+//   warp 1      tcgen05.mma issuer (one thread of the pair's first CTA) + tensor-memory
+//               allocation
+//   warps 2..   epilogue (4 warps; 8 for the math-heavy SwiGLU backward and for
+//               single-accumulator tiles: two per tensor-memory lane quadrant,
+//               splitting the columns): tensor memory -> registers -> fused math ->
+//               swizzled shared memory -> TMA bulk tensor stores, one 32x32 chunk at a
+//               time
 // Two fp32 accumulators of 128 x BN live in tensor memory so the epilogue of one
-// tile overlaps the main loop of the next.
+// tile overlaps the main loop of the next (MXFP8 256-column tiles: one, beside the
+// scale columns, released before the stores).
 //
 // Two groupings:
 //   RAGGED_M  forward and dgrad: expert e owns rows [off_e, off_e+1) of the routed
-//             activations; tiles of 128 rows start at off_e and rows past the
-//             expert's end are computed but never stored (a 32-row slice that ends
-//             inside the expert is written with plain stores, row by row).
+//             activations; tiles of 128 (pairs: 256) rows start at off_e and rows
+//             past the expert's end are computed but never stored (a 32-row slice
+//             that ends inside the expert is written with plain stores, row by row).
+//             Without offsets (null) the whole R rows form one segment.
 //   RAGGED_K  wgrad: dW_e = G_e^T . X_e sums over the expert's rows.  G is read
 //             through a per-expert tensor map whose row extent ends at the
 //             expert's last row (built on the device from the offsets), so the
@@ -1193,7 +1199,7 @@ static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, cons
 // ------------------------------------------------------------------------ MXFP8 GEMMs
 // Operands are quantised (E4M3 + E8M0 per 32 along each GEMM's K) right before the GEMM
 // that reads them; all quantised tensors and scales live in the workspace (MxWork).
-// One CTA per 128 x 128 tile; scales stream through shared memory into TMEM per stage.
+// Scales stream through shared memory into TMEM per stage.
 static inline moe_status cuq(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 #define MOE_MX_TRY(x)              \
   do {                             \
