@@ -75,7 +75,7 @@ __global__ void seg_prefix_kernel(const int32_t* __restrict__ seg_off, int E,
 }
 
 // One tile = one 32-row block of a segment (its rows p0 .. p0+nrows-1, starting at row r0
-// of the tensor) x 256 columns.
+// of the tensor) x 128 columns.
 struct TilePos {
   int e, p0, r0, nrows;
 };
@@ -109,7 +109,9 @@ __device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
   return g.rows > 0 ? (int64_t)e * ((g.rows + 127) / 128) : (int64_t)g.tile_pref[e];
 }
 
-constexpr int kQRows = 32, kQCols = 256;
+constexpr int kQRows = 32, kQCols = 128;
+constexpr int kQThreads = kQCols;            // one warp per 32-column block
+constexpr int kQCtasPerSm = 8;
 constexpr int kQPitch = kQCols * 2 + 16;     // bytes per staged row (16-byte skew: no bank conflicts)
 constexpr int kQBufs = 2;                    // tiles in flight per CTA (one being quantised)
 constexpr int kQBufBytes = kQRows * kQPitch;
@@ -156,7 +158,7 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* w, c
   d[1] = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
-// Persistent quantiser.  A tile is one 32-row block of a segment x 256 columns; each CTA
+// Persistent quantiser.  A tile is one 32-row block of a segment x 128 columns; each CTA
 // walks tiles blockIdx.x, +gridDim.x, ... with kQBufs shared-memory buffers: while it
 // quantises one tile, the next ones' rows stream in by 1-D bulk copies (so the bytes in
 // flight do not depend on registers).  Per tile it writes the rowwise codes/scales (ROW:
@@ -167,7 +169,7 @@ __device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* w, c
 // order in which a 256-column tile of the fused SwiGLU GEMM takes 128 gate and 128 up
 // rows of B.
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256, 4) quant_tile_kernel(
+__global__ void __launch_bounds__(kQThreads, kQCtasPerSm) quant_tile_kernel(
     const __nv_bfloat16* __restrict__ x, int C, const MxSegs g, int perm_f,
     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ sf_r, uint8_t* __restrict__ codes_c,
     uint8_t* __restrict__ sf_c, int* status) {
@@ -312,7 +314,7 @@ cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, in
   const int64_t blocks = g.rows > 0 ? (int64_t)g.E * ((g.rows + 31) / 32) : (R + 31) / 32 + g.E;
   const int64_t tiles = blocks * ((C + kQCols - 1) / kQCols);
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const int64_t grid = std::min<int64_t>(tiles, (int64_t)num_sms() * 4);
+  const int64_t grid = std::min<int64_t>(tiles, (int64_t)num_sms() * kQCtasPerSm);
   const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
   const bool row = codes_r != nullptr, col = codes_c != nullptr;
   auto kern = row && col ? quant_tile_kernel<true, true>
@@ -322,7 +324,7 @@ cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, in
   cudaError_t err =
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQSmem);
   if (err != cudaSuccess) return err;
-  kern<<<(unsigned)grid, 256, kQSmem, s>>>(xb, C, g, row ? perm_f : 0, codes_r, sf_r, codes_c,
+  kern<<<(unsigned)grid, kQThreads, kQSmem, s>>>(xb, C, g, row ? perm_f : 0, codes_r, sf_r, codes_c,
                                            sf_c, status);
   return cudaGetLastError();
 }
