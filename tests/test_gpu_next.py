@@ -193,3 +193,47 @@ def test_capacity_below_the_largest_count_is_reported(cuda_lib):
     C, _ = max_count(w, inp)
     desc, layer, dv, y, g, status = run_layer(w, inp, capacity=C - 1)
     assert status & lib.MOE_DEV_BAD_INDEX
+
+
+# ------------------------------------------------------------------- CUDA graphs
+
+def _graph_matches_eager(w, flags=0, capacity=0):
+    """Capture fwd+bwd of the layer in one CUDA graph, replay it with new logits, and
+    compare against an uncaptured run on the same inputs (bit-identical)."""
+    inp = make_inputs(w)
+    desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags, capacity)
+    if w.shared:
+        desc.flags |= lib.MOE_FLAG_SHARED_EXPERT
+    layer = lib.Layer(desc)
+    dv = {k: (None if v is None else v.cuda()) for k, v in inp.items()}
+    y = torch.empty(w.T, w.d, dtype=torch.bfloat16, device="cuda")
+    out = dict(dx=torch.empty_like(y), d_logits=torch.empty(w.T, w.E, device="cuda"),
+               dW13=torch.empty_like(dv["W13"]), dW2=torch.empty_like(dv["W2"]))
+    run = lambda: (layer.fwd(dv["x"], dv["W13"], dv["W2"], logits=dv["logits"], y=y),  # noqa: E731
+                   layer.bwd(dv["dy"], dv["W13"], dv["W2"], x=dv["x"], out=out))
+    run()                                   # warm-up (kernel attributes, descriptor caches)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    newL = random_logits(w.T, w.E, seed=w.seed + 1000)
+    dv["logits"].copy_(newL)
+    g.replay()
+    torch.cuda.synchronize()
+    got = {k: v.clone() for k, v in dict(out, y=y).items()}
+    run()                                   # the same inputs, uncaptured
+    torch.cuda.synchronize()
+    for k, v in dict(out, y=y).items():
+        assert torch.equal(got[k], v), k
+    assert lib.moe_read_device_status(layer.ws) == 0
+
+
+def test_mxfp8_layer_replays_in_a_cuda_graph(cuda_lib):
+    _graph_matches_eager(Workload("gmx", 2000, 512, 16, 4, 256, "mxfp8", router=False,
+                                  skew=False, seed=21))
+
+
+def test_recompute_shared_padded_layer_replays_in_a_cuda_graph(cuda_lib):
+    w = Workload("gall", 2000, 256, 16, 4, 128, "bf16", router=False, skew=True, seed=22,
+                 shared=True)
+    _graph_matches_eager(w, flags=lib.MOE_FLAG_RECOMPUTE, capacity=2000)
