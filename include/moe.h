@@ -252,8 +252,8 @@ moe_status moe_combine_bwd(const moe_desc* desc, const void* dy, const void* y_p
  * block are written as 0 (scale 2^-127), so a reader of whole chunks sees finite scales;
  * other slots that no block reaches (rowwise rows past a segment's end) are left
  * untouched.  cols must be a multiple of 128.  ws: at least 256 + 8*(num_segments+1)
- * bytes of device scratch; its first 4 bytes are a device status word (MOE_DEV_TIMEOUT if
- * a copy wait gives up), read with moe_read_device_status. */
+ * bytes of device scratch; its first 4 bytes are a device status word, read with
+ * moe_read_device_status (the quantiser itself has no waits and sets no status). */
 moe_status moe_mx_scale_bytes(int64_t rows, int32_t cols, int32_t num_segments, size_t* bytes);
 moe_status moe_mx_quantize(const void* x, int64_t rows, int32_t cols, const int32_t* seg_offsets,
                            int32_t num_segments, int32_t colwise, uint8_t* codes, uint8_t* scales,

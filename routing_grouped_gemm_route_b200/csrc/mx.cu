@@ -38,11 +38,14 @@ namespace {
 
 using namespace sm100;
 
-// Shared exponent of a block with max magnitude `amax` (>= 0).
-__device__ __forceinline__ int mx_exponent(float amax) {
-  if (!(amax > 0.f)) return -127;
-  int s = ilogbf(amax) - 8;          // floor(log2(amax)) for finite non-zero amax
-  return s < -127 ? -127 : (s > 127 ? 127 : s);
+// Shared exponent of a block whose largest magnitude has the bf16 bit pattern `b`
+// (sign cleared).  For a normal value with exponent field E, floor(log2) = E - 127, so
+// s = E - 135; anything at or below 2^-119 (E <= 8, subnormals and zero) clamps to -127.
+// Non-finite blocks: infinity gives 127, NaN -127.
+__device__ __forceinline__ int mx_exponent_bits(uint32_t b) {
+  const int e = static_cast<int>((b >> 7) & 0xffu);
+  if (e == 0xff) return (b & 0x7fu) ? -127 : 127;
+  return (e < 8 ? 8 : e) - 135;
 }
 // 2^-s as a float, exactly (2^-127 is the subnormal 0x00400000).  Multiplying by it is
 // the same IEEE operation as scaling the exponent: exact, or one round to nearest even.
@@ -109,187 +112,162 @@ __device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
   return g.rows > 0 ? (int64_t)e * ((g.rows + 127) / 128) : (int64_t)g.tile_pref[e];
 }
 
-constexpr int kQRows = 32, kQCols = 128;
-constexpr int kQThreads = kQCols;            // one warp per 32-column block
-constexpr int kQCtasPerSm = 8;
-constexpr int kQPitch = kQCols * 2 + 16;     // bytes per staged row (16-byte skew: no bank conflicts)
-constexpr int kQBufs = 2;                    // tiles in flight per CTA (one being quantised)
-constexpr int kQBufBytes = kQRows * kQPitch;
-constexpr size_t kQSmem = 128 + (size_t)kQBufs * kQBufBytes;
-
-// 32 bf16 of a staged row (64 contiguous bytes), kept packed: w[i] holds elements
-// 2i (low half) and 2i+1 (high half).
-__device__ __forceinline__ void staged32(const uint8_t* p, uint32_t* w) {
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 u = *reinterpret_cast<const uint4*>(p + 16 * j);
-    w[4 * j] = u.x;
-    w[4 * j + 1] = u.y;
-    w[4 * j + 2] = u.z;
-    w[4 * j + 3] = u.w;
-  }
-}
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 // |x| of both bf16 halves (the sign bits cleared).  Non-negative IEEE values order like
 // their bit patterns, so a per-half unsigned max of |x| bits is the exact max |x|.
 __device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7fff7fffu; }
-__device__ __forceinline__ float amax32(const uint32_t* w) {
-  uint32_t m = 0u;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) m = __vmaxu2(m, abs2(w[i]));
-  return fmaxf(bf_lo(m), bf_hi(m));
-}
 
-// 32 codes of the packed bf16 w[] times m[j] (PER_ELEM) or m[0] -> two 16-byte stores
-template <bool PER_ELEM>
-__device__ __forceinline__ void store_codes32(uint8_t* dst, const uint32_t* w, const float* m) {
-  uint32_t o[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const int i = 4 * j;
-    const float m0 = m[PER_ELEM ? i : 0], m1 = m[PER_ELEM ? i + 1 : 0];
-    const float m2 = m[PER_ELEM ? i + 2 : 0], m3 = m[PER_ELEM ? i + 3 : 0];
-    o[j] = e4m3x2(bf_lo(w[2 * j]) * m0, bf_hi(w[2 * j]) * m1) |
-           (e4m3x2(bf_lo(w[2 * j + 1]) * m2, bf_hi(w[2 * j + 1]) * m3) << 16);
+// A lane's CPL consecutive bf16 of one row (CPL = 4: two words, 2: one word) and what is
+// done with them: the per-half max of |x|, the codes (one multiplier per column), stores.
+template <int CPL> struct Lane;
+template <> struct Lane<4> {
+  using V = uint2;
+  static __device__ __forceinline__ V load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint2*>(p)); }
+  static __device__ __forceinline__ V zero() { return make_uint2(0u, 0u); }
+  static __device__ __forceinline__ uint32_t absmax(V v) { return __vmaxu2(abs2(v.x), abs2(v.y)); }
+  static __device__ __forceinline__ void absmax_cols(uint32_t* m, V v) {
+    m[0] = __vmaxu2(m[0], abs2(v.x));
+    m[1] = __vmaxu2(m[1], abs2(v.y));
   }
-  uint4* d = reinterpret_cast<uint4*>(dst);
-  d[0] = make_uint4(o[0], o[1], o[2], o[3]);
-  d[1] = make_uint4(o[4], o[5], o[6], o[7]);
+  static __device__ __forceinline__ void store(uint8_t* p, V v, const float* m) {
+    *reinterpret_cast<uint32_t*>(p) = e4m3x2(bf_lo(v.x) * m[0], bf_hi(v.x) * m[1]) |
+                                      (e4m3x2(bf_lo(v.y) * m[2], bf_hi(v.y) * m[3]) << 16);
+  }
+};
+template <> struct Lane<2> {
+  using V = uint32_t;
+  static __device__ __forceinline__ V load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint32_t*>(p)); }
+  static __device__ __forceinline__ V zero() { return 0u; }
+  static __device__ __forceinline__ uint32_t absmax(V v) { return abs2(v); }
+  static __device__ __forceinline__ void absmax_cols(uint32_t* m, V v) { m[0] = __vmaxu2(m[0], abs2(v)); }
+  static __device__ __forceinline__ void store(uint8_t* p, V v, const float* m) {
+    *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(e4m3x2(bf_lo(v) * m[0], bf_hi(v) * m[1]));
+  }
+};
+
+// One level of the rowwise reduce-scatter over the lanes of a 32-column block: lanes
+// whose bit M is set keep the upper half of the CPL*2*M rows still held and take the
+// partner's (lane ^ M) maxima of them; the others keep the lower half.  Levels M, M/2,
+// .., 1 leave lane j with rows CPL*j .. CPL*j+CPL-1.
+template <int CPL, int M>
+__device__ __forceinline__ void row_reduce_scatter(uint32_t (&a)[32], int sub) {
+  constexpr int N = CPL * M;
+  const bool up = (sub & M) != 0;
+#pragma unroll
+  for (int i = 0; i < N; ++i) {
+    const uint32_t send = up ? a[i] : a[i + N];
+    const uint32_t keep = up ? a[i + N] : a[i];
+    a[i] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, M));
+  }
+  if constexpr (M > 1) row_reduce_scatter<CPL, M / 2>(a, sub);
 }
 
-// Persistent quantiser.  A tile is one 32-row block of a segment x 128 columns; each CTA
-// walks tiles blockIdx.x, +gridDim.x, ... with kQBufs shared-memory buffers: while it
-// quantises one tile, the next ones' rows stream in by 1-D bulk copies (so the bytes in
-// flight do not depend on registers).  Per tile it writes the rowwise codes/scales (ROW:
-// blocks of 32 along columns) and/or the colwise ones (COL: blocks of 32 along the
-// segment's rows; the tile is exactly one such block per column).
+constexpr int kQWarps = 4;                   // warps per CTA
+template <int CPL> constexpr int q_ctas_per_sm(bool both) { return CPL == 4 ? (both ? 3 : 4) : (both ? 5 : 6); }
+
+// Persistent quantiser; one warp per tile, no shared memory, no barriers.  A tile is one
+// 32-row block of a segment x 32*CPL columns; lane L holds columns CPL*L .. CPL*L+CPL-1
+// of all 32 rows in registers (each load instruction of the warp reads 64*CPL contiguous
+// bytes of one row; all 32 rows' loads are in flight together), so
+//   ROW (blocks of 32 along columns): a row's block spans G = 32/CPL lanes.  A butterfly
+//        reduce-scatter over them leaves lane j of the group with the maxima of rows
+//        CPL*j .. CPL*j+CPL-1 (each step halves the rows a lane keeps); it derives
+//        those rows' exponents and scale bytes, and shuffles return the multipliers;
+//   COL (blocks of 32 along the segment's rows; the tile is exactly one block per
+//        column): each lane's running max over its 32 rows, no communication.
+// Codes leave as CPL-byte stores, 32*CPL contiguous bytes per row and instruction.
 // perm_f > 0 (SwiGLU weights [W1; W3], d_ff = perm_f rows each): the rowwise scale of
 // row p is filed under the row order gate[0:128], up[0:128], gate[128:256], ..., the
 // order in which a 256-column tile of the fused SwiGLU GEMM takes 128 gate and 128 up
 // rows of B.
-template <bool ROW, bool COL>
-__global__ void __launch_bounds__(kQThreads, kQCtasPerSm) quant_tile_kernel(
+template <int CPL, bool ROW, bool COL>
+__global__ void __launch_bounds__(kQWarps * 32, q_ctas_per_sm<CPL>(ROW && COL)) quant_warp_kernel(
     const __nv_bfloat16* __restrict__ x, int C, const MxSegs g, int perm_f,
     uint8_t* __restrict__ codes_r, uint8_t* __restrict__ sf_r, uint8_t* __restrict__ codes_c,
-    uint8_t* __restrict__ sf_c, int* status) {
-  extern __shared__ uint8_t q_smem_raw[];
-  uint8_t* bufs = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(q_smem_raw) + 127) &
-                                             ~uintptr_t(127));
-  __shared__ float col_m[kQCols];
-  __shared__ uint64_t bar[kQBufs];
-  __shared__ TilePos pos[kQBufs];
-  __shared__ int abort_flag;
-  const int t = threadIdx.x;
-  const int ctiles = (C + kQCols - 1) / kQCols;
+    uint8_t* __restrict__ sf_c) {
+  using LN = Lane<CPL>;
+  using V = typename LN::V;
+  constexpr int TC = 32 * CPL;               // tile columns
+  constexpr int G = 32 / CPL;                // lanes of one 32-column block
+  const int lane = threadIdx.x & 31;
+  const int ctiles = C / TC;
+  const int W = C / 128;
   const int nblk = g.rows > 0 ? g.E * ((g.rows + 31) / 32) : g.blk_pref[g.E];
   const int ntiles = nblk * ctiles;
-  if ((int)blockIdx.x >= ntiles) return;      // uniform over the CTA
-  if (t == 0) {
-    for (int i = 0; i < kQBufs; ++i) mbar_init(&bar[i], 1);
-    abort_flag = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  // warp 0 loads tile `tile` into buffer `b`: lane 0 arms the barrier with the byte count,
-  // lane r copies row r (the phase cannot complete before lane 0's arrival)
-  auto issue = [&](int tile, int b) {
+  const int stride = static_cast<int>(gridDim.x) * kQWarps;
+  for (int tile = static_cast<int>(blockIdx.x) * kQWarps + static_cast<int>(threadIdx.x >> 5);
+       tile < ntiles; tile += stride) {
     TilePos tp;
     tile_pos(g, tile / ctiles, tp);
-    const int c0 = (tile % ctiles) * kQCols;
-    const int ncols = min(kQCols, C - c0);
-    if (t == 0) {
-      pos[b] = tp;
-      fence_proxy_async_smem();               // earlier generic reads of buf[b] before the copies
-      mbar_arrive_expect_tx(&bar[b], static_cast<uint32_t>(tp.nrows * ncols * 2));
-    }
-    __syncwarp();
-    if (t < tp.nrows)
-      bulk_load(bufs + b * kQBufBytes + t * kQPitch, x + (int64_t)(tp.r0 + t) * C + c0,
-                static_cast<uint32_t>(ncols * 2), &bar[b]);
-  };
-  // prologue: the first kQBufs-1 tiles
-  for (int i = 0; i < kQBufs - 1; ++i) {
-    const int tile = blockIdx.x + i * gridDim.x;
-    if (t < 32 && tile < ntiles) issue(tile, i);
-  }
-  const int W = C / 128;
-  const int row = t & 31, q = t >> 5;         // this thread's row and 32-column block
-  const int lane = t & 31;
-  int it = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++it) {
-    const int b = it % kQBufs;
-    // the buffer of iteration it-1 was released by the barrier that ended it
-    const int ahead = tile + (kQBufs - 1) * gridDim.x;
-    if (t < 32 && ahead < ntiles) issue(ahead, (it + kQBufs - 1) % kQBufs);
-    const bool ok = mbar_wait(&bar[b], (it / kQBufs) & 1u,
-                              reinterpret_cast<volatile int*>(&abort_flag), status);
-    // every step below is warp-local; the barrier at the end releases the buffer (and
-    // agrees on an abort)
-    if (ok) {
-    const TilePos tp = pos[b];
-    const int c0 = (tile % ctiles) * kQCols;
-    const int ncols = min(kQCols, C - c0);
+    const int c0 = (tile % ctiles) * TC;
+    const int col = c0 + CPL * lane;          // my first column
+    const int nrows = tp.nrows;               // warp-uniform
+    const __nv_bfloat16* src = x + (int64_t)tp.r0 * C + col;
+    V v[32];
+#pragma unroll
+    for (int r = 0; r < 32; ++r)
+      v[r] = r < nrows ? LN::load(src + (int64_t)r * C) : LN::zero();   // past the segment: 0
     const int64_t tile0 = seg_tile0(g, tp.e);
-    const uint8_t* tb = bufs + b * kQBufBytes;
-    const bool active = row < tp.nrows && q * 32 < ncols;
-    uint32_t v[16];
-    if (active) staged32(tb + row * kQPitch + q * 64, v);
-    if (ROW && active) {
-      const int s = mx_exponent(amax32(v));
-      const float m = exp2_neg(s);
-      store_codes32<false>(codes_r + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, &m);
-      int p = tp.p0 + row;
-      if (perm_f > 0)
-        p = p < perm_f ? (p / 128) * 256 + (p % 128)
-                       : ((p - perm_f) / 128) * 256 + 128 + (p - perm_f) % 128;
-      const int col = c0 + q * 32;
-      sf_r[sf_byte((tile0 + p / 128) * W + col / 128, p, (col & 127) >> 5)] =
-          static_cast<uint8_t>(s + 127);
-    }
-    if (COL && q * 32 < ncols) {   // warp-uniform: this warp's 32-column block exists
-      // The warp holds the block's 32 rows (one per lane; rows past the segment's end
-      // are masked to zero).  A butterfly reduce-scatter of |x| over the lanes leaves
-      // lane L with the max of column L: each step halves the words a lane keeps.
-      uint32_t a[16];
+    if (COL) {
+      uint32_t mc[CPL / 2] = {};              // column maxima (|x| bits, two per word)
 #pragma unroll
-      for (int i = 0; i < 16; ++i) a[i] = active ? abs2(v[i]) : 0u;
+      for (int r = 0; r < 32; ++r) LN::absmax_cols(mc, v[r]);
+      int sc[CPL];
+      float mul[CPL];
 #pragma unroll
-      for (int m = 16; m >= 2; m >>= 1) {
-        const bool up = (lane & m) != 0;
-#pragma unroll
-        for (int i = 0; i < m / 2; ++i) {
-          const uint32_t send = up ? a[i] : a[i + m / 2];
-          const uint32_t keep = up ? a[i + m / 2] : a[i];
-          a[i] = __vmaxu2(keep, __shfl_xor_sync(0xffffffffu, send, m));
-        }
+      for (int i = 0; i < CPL; ++i) {
+        sc[i] = mx_exponent_bits((i & 1) ? mc[i / 2] >> 16 : mc[i / 2] & 0xffffu);
+        mul[i] = exp2_neg(sc[i]);
       }
-      const uint32_t mm = __vmaxu2(a[0], __shfl_xor_sync(0xffffffffu, a[0], 1));
-      const int s = mx_exponent((lane & 1) ? bf_hi(mm) : bf_lo(mm));
-      const int col = c0 + q * 32 + lane;
-      col_m[q * 32 + lane] = exp2_neg(s);
-      const int64_t chunk = (tile0 + tp.p0 / 128) * W + col / 128;
+      uint8_t* dst = codes_c + (int64_t)tp.r0 * C + col;
+#pragma unroll
+      for (int r = 0; r < 32; ++r)
+        if (r < nrows) LN::store(dst + (int64_t)r * C, v[r], mul);
+      const int64_t chunk = (tile0 + tp.p0 / 128) * W + c0 / 128;
       const int blk = (tp.p0 & 127) >> 5;
-      sf_c[sf_byte(chunk, col, blk)] = static_cast<uint8_t>(s + 127);
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) sf_c[sf_byte(chunk, col + i, blk)] = static_cast<uint8_t>(sc[i] + 127);
       // The segment's last chunk may hold fewer than four blocks.  A K-stage of a wgrad
       // GEMM still reads all four scales (its rows past the segment are zero codes), so
       // the absent blocks get the finite scale 2^-127 rather than whatever the buffer
       // held (0xFF = NaN).
       if (tp.p0 + 32 >= seg_rows(g, tp.e))
-        for (int k = blk + 1; k < 4; ++k) sf_c[sf_byte(chunk, col, k)] = 0;
-      __syncwarp();
-      if (active)
-        store_codes32<true>(codes_c + (int64_t)(tp.r0 + row) * C + c0 + q * 32, v, col_m + q * 32);
+        for (int k = blk + 1; k < 4; ++k)
+#pragma unroll
+          for (int i = 0; i < CPL; ++i) sf_c[sf_byte(chunk, col + i, k)] = 0;
     }
+    if (ROW) {
+      const int sub = lane & (G - 1);
+      uint32_t a[32];
+#pragma unroll
+      for (int r = 0; r < 32; ++r) a[r] = LN::absmax(v[r]);
+      row_reduce_scatter<CPL, G / 2>(a, sub);
+      // rows CPL*sub + i (i < CPL) are mine; the segment's row p0 + r maps to the scale
+      // MN index pp0 + r (a 32-row block never straddles a 128-row gate/up group)
+      int pp0 = tp.p0;
+      if (perm_f > 0)
+        pp0 = pp0 < perm_f ? (pp0 / 128) * 256 + (pp0 % 128)
+                           : ((pp0 - perm_f) / 128) * 256 + 128 + (pp0 - perm_f) % 128;
+      const int blk = (c0 & 127) / 32 + lane / G;
+      uint8_t* sf = sf_r + sf_byte((tile0 + pp0 / 128) * W + c0 / 128, pp0, blk);
+      float mine[CPL];
+#pragma unroll
+      for (int i = 0; i < CPL; ++i) {
+        const int s = mx_exponent_bits(max(a[i] & 0xffffu, a[i] >> 16));
+        mine[i] = exp2_neg(s);
+        if (CPL * sub + i < nrows) sf[16 * (CPL * sub + i)] = static_cast<uint8_t>(s + 127);
+      }
+      uint8_t* dst = codes_r + (int64_t)tp.r0 * C + col;
+#pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        float m[CPL];
+        m[0] = __shfl_sync(0xffffffffu, mine[r % CPL], (lane & ~(G - 1)) | (r / CPL));
+#pragma unroll
+        for (int i = 1; i < CPL; ++i) m[i] = m[0];
+        if (r < nrows) LN::store(dst + (int64_t)r * C, v[r], m);
+      }
     }
-    if (__syncthreads_or(!ok)) break;   // this buffer and col_m free for reuse
-  }
-  // After an abort, the copies still in flight (iterations it .. it+kQBufs-1 that have a
-  // tile) must land before the CTA exits.
-  if (t == 0 && abort_flag) {
-    for (int j = it; j < it + kQBufs; ++j)
-      if (blockIdx.x + j * gridDim.x < ntiles)
-        mbar_wait_teardown(&bar[j % kQBufs], (j / kQBufs) & 1u);
   }
 }
 
@@ -306,27 +284,34 @@ cudaError_t launch_mx_prefix(const int32_t* seg_off, int E, int32_t* tile_pref, 
   return cudaGetLastError();
 }
 
+template <int CPL>
+static cudaError_t launch_quant(const __nv_bfloat16* x, int64_t tiles, int C, const MxSegs& g,
+                                int perm_f, uint8_t* codes_r, uint8_t* sf_r, uint8_t* codes_c,
+                                uint8_t* sf_c, cudaStream_t s) {
+  const bool row = codes_r != nullptr, col = codes_c != nullptr;
+  const int64_t grid = std::min<int64_t>((tiles + kQWarps - 1) / kQWarps,
+                                         (int64_t)num_sms() * q_ctas_per_sm<CPL>(row && col));
+  auto kern = row && col ? quant_warp_kernel<CPL, true, true>
+              : row      ? quant_warp_kernel<CPL, true, false>
+                         : quant_warp_kernel<CPL, false, true>;
+  kern<<<(unsigned)grid, kQWarps * 32, 0, s>>>(x, C, g, row ? perm_f : 0, codes_r, sf_r, codes_c,
+                                              sf_c);
+  return cudaGetLastError();
+}
+
+constexpr int kQCpl = 4;   // columns per lane
+
 cudaError_t launch_mx_quant(const void* x, int64_t R, int C, const MxSegs& g, int perm_f,
                             uint8_t* codes_r, uint8_t* sf_r, uint8_t* codes_c, uint8_t* sf_c,
                             int* status, cudaStream_t s) {
-  if (R == 0) return cudaSuccess;
+  (void)status;   // no waits, no data-dependent failure
+  if (R == 0 || (codes_r == nullptr && codes_c == nullptr)) return cudaSuccess;
   // tiles: sum_e ceil(rows_e/32) <= R/32 + E row blocks, times the column tiles
   const int64_t blocks = g.rows > 0 ? (int64_t)g.E * ((g.rows + 31) / 32) : (R + 31) / 32 + g.E;
-  const int64_t tiles = blocks * ((C + kQCols - 1) / kQCols);
+  const int64_t tiles = blocks * (C / (32 * kQCpl));
   if (tiles > 0x7fffffffLL) return cudaErrorInvalidValue;
-  const int64_t grid = std::min<int64_t>(tiles, (int64_t)num_sms() * kQCtasPerSm);
-  const __nv_bfloat16* xb = reinterpret_cast<const __nv_bfloat16*>(x);
-  const bool row = codes_r != nullptr, col = codes_c != nullptr;
-  auto kern = row && col ? quant_tile_kernel<true, true>
-              : row      ? quant_tile_kernel<true, false>
-                         : quant_tile_kernel<false, true>;
-  if (!row && !col) return cudaSuccess;
-  cudaError_t err =
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kQSmem);
-  if (err != cudaSuccess) return err;
-  kern<<<(unsigned)grid, kQThreads, kQSmem, s>>>(xb, C, g, row ? perm_f : 0, codes_r, sf_r, codes_c,
-                                           sf_c, status);
-  return cudaGetLastError();
+  return launch_quant<kQCpl>(reinterpret_cast<const __nv_bfloat16*>(x), tiles, C, g, perm_f,
+                             codes_r, sf_r, codes_c, sf_c, s);
 }
 
 cudaError_t launch_mx_quantize(const void* x, int64_t R, int C, const int32_t* seg_off, int E,
