@@ -23,6 +23,8 @@ CASES = [
     (1500, 256, 128, 6, 1, "bf16", "one"),      # nearly all rows on one expert
     (96, 256, 128, 4, 4, "bf16", None),         # k = E, fewer rows than one tile
     (4096, 1024, 512, 16, 4, "bf16", None),
+    (300, 256, 256, 5, 2, "bf16", None),        # d_ff % 256 == 0: every GEMM with tokens as N
+    (2048, 512, 256, 33, 4, "bf16", "empty"),   # ... with empty experts and short tails
 ]
 
 
