@@ -53,10 +53,10 @@ def make_x(R, C, seed):
     return x.to(torch.bfloat16)
 
 
+@pytest.mark.parametrize("C", [128, 384])
 @pytest.mark.parametrize("colwise", [False, True])
 @pytest.mark.parametrize("counts", [[300], [128, 0, 77, 256, 1, 33], [0, 0, 500], [40] * 9])
-def test_mx_quantize_bit_exact(cuda_lib, counts, colwise):
-    C = 384
+def test_mx_quantize_bit_exact(cuda_lib, counts, colwise, C):
     seg_off = np.concatenate([[0], np.cumsum(counts)]).astype(np.int64)
     R = int(seg_off[-1])
     E = len(counts)
