@@ -44,6 +44,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mx_block.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -83,6 +84,12 @@ struct Params {
     int W;
   } sfa, sfb;
   const int32_t* tile_pref;  // [E+1] prefix of ceil(count_e / 128)
+  // MXFP8 SwiGLU forward: also quantise the bf16 a that FC2 reads along its rows into
+  // E4M3 codes [R, q_ld] and scale chunks in the quantiser's rowwise layout (null: not
+  // asked for)
+  uint8_t* q_codes;
+  uint8_t* q_sf;
+  int q_ld;
   int* status;
 };
 
@@ -294,6 +301,14 @@ __device__ __forceinline__ void pack_bf16x32(const float* v, uint32_t* w) {
     w[4 * j + 2] = pk.raw.z;
     w[4 * j + 3] = pk.raw.w;
   }
+}
+// Rowwise MX block of an epilogue's output row: codes at (row, col) of q_codes and the
+// scale in the chunk of (expert e, row p of its segment, column col); col % 32 == 0.
+__device__ __forceinline__ void quantise_out_block(const Params& p, int e, int p_seg, int64_t row,
+                                                   int col, const uint32_t* w) {
+  const int s = mxb::quantise_block32(w, p.q_codes + row * p.q_ld + col);
+  const int64_t chunk = ((int64_t)p.tile_pref[e] + p_seg / 128) * (p.q_ld / 128) + col / 128;
+  p.q_sf[mxb::sf_byte(chunk, p_seg, (col & 127) >> 5)] = static_cast<uint8_t>(s + 127);
 }
 __device__ __forceinline__ void store_packed32(bf16* dst, const uint32_t* w) {
 #pragma unroll
@@ -678,6 +693,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                   store_packed32(reinterpret_cast<bf16*>(p.out_a) + grow * (int64_t)p.f + hc,
                                  pk[EPI == EPI_SWIGLU_FWD ? 2 : 0][i]);
                 }
+                if (kMX && p.q_codes && valid)
+                  quantise_out_block(p, tl.e, tl.m0 + myrow + q * 32 + lane, grow, hc,
+                                     pk[EPI == EPI_SWIGLU_FWD ? 2 : 0][i]);
               } else {
                 const int c = (cfirst + i) * 32;
                 if (whole) {
@@ -1000,6 +1018,9 @@ struct MxRefs {             // MXFP8 scale chunks of both operands (unused other
   Params::Sf a{}, b{};
   int64_t a_chunks = 0, b_chunks = 0;   // sizes of the two scale buffers in chunks
   const int32_t* tile_pref = nullptr;
+  uint8_t* q_codes = nullptr;           // SwiGLU forward: rowwise codes of a
+  uint8_t* q_sf = nullptr;
+  int q_ld = 0;
 };
 
 // Scale maps of an MXFP8 GEMM (copies of `dummy` for the other kernels, which never
@@ -1056,6 +1077,9 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.sfa = mx.a;
   p.sfb = mx.b;
   p.tile_pref = mx.tile_pref;
+  p.q_codes = mx.q_codes;
+  p.q_sf = mx.q_sf;
+  p.q_ld = mx.q_ld;
   p.status = status;
   CUtensorMap tsa, tsb;
   if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
@@ -1198,7 +1222,8 @@ static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, cons
 
 // ------------------------------------------------------------------------ MXFP8 GEMMs
 // Operands are quantised (E4M3 + E8M0 per 32 along each GEMM's K) right before the GEMM
-// that reads them; all quantised tensors and scales live in the workspace (MxWork).
+// that reads them, except a along d_ff, which FC1's SwiGLU epilogue quantises from the
+// bf16 values it stores; all quantised tensors and scales live in the workspace (MxWork).
 // Scales stream through shared memory into TMEM per stage.
 static inline moe_status cuq(cudaError_t e) { return e == cudaSuccess ? MOE_OK : MOE_ECUDA; }
 #define MOE_MX_TRY(x)              \
@@ -1262,10 +1287,12 @@ static moe_status mx_fwd(const GemmShape& g, const void* x_perm, const void* W13
   act_sf(m1.a, m1.a_chunks, g, w.xr_sf, d, true);
   weight_sf(m1.b, m1.b_chunks, g, w.w13r_sf, 2 * f, d, true);
   m1.tile_pref = w.act_pref;
+  m1.q_codes = w.ar;          // FC1's epilogue also writes a rowwise along d_ff (FC2's K)
+  m1.q_sf = w.ar_sf;
+  m1.q_ld = f;
   MOE_MX_TRY((run_m<fp8, false, EPI_SWIGLU_FWD, 256, true, bf16>(
       g, w.xr, d, w.w13r, 2 * f, 2 * f, d, H13, 2 * f, a, nullptr, off, st, s, m1)));
-  // FC2: a and W2 rowwise along d_ff
-  MOE_MX_TRY(cuq(launch_mx_quant(a, g.R, f, act, 0, w.ar, w.ar_sf, nullptr, nullptr, st, s)));
+  // FC2: W2 rowwise along d_ff (a's codes came from FC1)
   MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, w.w2r, w.w2r_sf,
                                  nullptr, nullptr, st, s)));
   MxRefs m2;
@@ -1320,7 +1347,8 @@ static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_
   m2.tile_pref = w.act_pref;
   MOE_MX_TRY(mx_wgrad<OutT>(g, w.dyc, d, w.ac, f, dW2, accum, off, maps, st, s, m2));
   // dH13 both ways (FC1 dgrad, FC1 wgrad), W13 colwise along its 2*d_ff rows, x_perm
-  // colwise along tokens
+  // colwise along tokens.  (Quantising dH13's rows in FC2 dgrad's epilogue instead was
+  // slower: that epilogue holds the single accumulator, so its MMAs wait for it.)
   MOE_MX_TRY(cuq(launch_mx_quant(dH13, g.R, 2 * f, act, 0, w.dhr, w.dhr_sf, w.dhc, w.dhc_sf, st, s)));
   MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), 0, nullptr,
                                  nullptr, w.w13c, w.w13c_sf, st, s)));

@@ -31,6 +31,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "mx_block.cuh"
 #include "sm100.cuh"
 
 namespace moe {
@@ -38,28 +39,13 @@ namespace {
 
 using namespace sm100;
 
-// Shared exponent of a block whose largest magnitude has the bf16 bit pattern `b`
-// (sign cleared).  For a normal value with exponent field E, floor(log2) = E - 127, so
-// s = E - 135; anything at or below 2^-119 (E <= 8, subnormals and zero) clamps to -127.
-// Non-finite blocks: infinity gives 127, NaN -127.
-__device__ __forceinline__ int mx_exponent_bits(uint32_t b) {
-  const int e = static_cast<int>((b >> 7) & 0xffu);
-  if (e == 0xff) return (b & 0x7fu) ? -127 : 127;
-  return (e < 8 ? 8 : e) - 135;
-}
-// 2^-s as a float, exactly (2^-127 is the subnormal 0x00400000).  Multiplying by it is
-// the same IEEE operation as scaling the exponent: exact, or one round to nearest even.
-__device__ __forceinline__ float exp2_neg(int s) {
-  return s <= 126 ? __int_as_float((127 - s) << 23) : __int_as_float(0x00400000);
-}
-// Two E4M3 codes (round to nearest even, saturating to +-448) of a and b; a in the low byte.
-__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
-  return static_cast<uint32_t>(
-      __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
-}
-__device__ __forceinline__ size_t sf_byte(int64_t chunk, int i, int block) {
-  return (size_t)chunk * 512 + 16 * (i & 31) + 4 * ((i & 127) >> 5) + block;
-}
+using mxb::exp2_neg;
+using mxb::e4m3x2;
+using mxb::sf_byte;
+using mxb::bf_lo;
+using mxb::bf_hi;
+using mxb::abs2;
+__device__ __forceinline__ int mx_exponent_bits(uint32_t b) { return mxb::exponent_bits(b); }
 
 // tile_pref[e] = sum_{e'<e} ceil(rows_e'/128); blk_pref[e] = sum_{e'<e} ceil(rows_e'/32).
 __global__ void seg_prefix_kernel(const int32_t* __restrict__ seg_off, int E,
@@ -111,12 +97,6 @@ __device__ __forceinline__ int seg_rows(const MxSegs& g, int e) {
 __device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
   return g.rows > 0 ? (int64_t)e * ((g.rows + 127) / 128) : (int64_t)g.tile_pref[e];
 }
-
-__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
-// |x| of both bf16 halves (the sign bits cleared).  Non-negative IEEE values order like
-// their bit patterns, so a per-half unsigned max of |x| bits is the exact max |x|.
-__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7fff7fffu; }
 
 // A lane's CPL consecutive bf16 of one row (CPL = 4: two words, 2: one word) and what is
 // done with them: the per-half max of |x|, the codes (one multiplier per column), stores.
