@@ -25,6 +25,12 @@ def npi(t) -> np.ndarray:
     return t.detach().cpu().numpy().astype(np.int64)
 
 
+def row_rel(got, ref) -> np.ndarray:
+    """Per-row relative error ||got - ref|| / ||ref|| of a GPU tensor against fp64 rows."""
+    g = f64(got)
+    return np.linalg.norm(g - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+
+
 def rel(a, b) -> float:
     return oracle.rel_fro(f64(a), f64(b))
 

@@ -9,7 +9,7 @@ import oracle
 from routing_grouped_gemm_route_b200 import lib
 from routing_grouped_gemm_route_b200.inputs import normal_tensor, random_logits
 
-from helpers import TOL, f64, npi, rel, run_route
+from helpers import TOL, f64, npi, rel, row_rel, run_route
 
 pytestmark = pytest.mark.gpu
 
@@ -79,6 +79,10 @@ def test_grouped_gemm_fwd(cuda_lib, T, d, f, E, k, dt, mode):
     for e in range(E):
         if off[e + 1] > off[e]:
             assert rel(yp[off[e]:off[e + 1]], refY[off[e]:off[e + 1]]) < 2 * TOL, e
+    # and per row: what remains is fp32 accumulation (TF32 operand rounding) and the
+    # output's own rounding, so one wrong row (a tile edge, a ragged tail) fails this
+    assert row_rel(H13, refH).max() < 1e-2
+    assert row_rel(yp, refY).max() < 1e-2
 
 
 @pytest.mark.parametrize("dw_fp32", [False, True])

@@ -10,7 +10,7 @@ from oracle.mx import mx_quantize_dequantize as mxq
 from routing_grouped_gemm_route_b200 import lib
 from routing_grouped_gemm_route_b200.inputs import Workload, make_inputs, normal_tensor, random_logits
 
-from helpers import f64, npi, rel, run_layer, run_route
+from helpers import f64, npi, rel, row_rel, run_layer, run_route
 
 pytestmark = pytest.mark.gpu
 TOL_MX = 3e-2
@@ -64,6 +64,12 @@ def test_mxfp8_grouped_gemm_fwd(cuda_lib, T, d, f, E, k, mode):
     assert rel(a, oracle.silu(h1) * h3) < TOL_MX
     assert rel(yp, refY) < TOL_MX
     assert not torch.isnan(yp).any()
+    # The references quantise exactly the bf16 operands the GPU quantised (FC2's: the a
+    # it stored), so what remains per row is fp32 accumulation and the bf16 rounding of
+    # the output (~2^-9): one wrong code or scale byte anywhere in a row's K fails this.
+    assert row_rel(H13, refH).max() < 1e-2
+    assert row_rel(yp, refY).max() < 1e-2
+
 
 
 @pytest.mark.parametrize("T,d,f,E,k,mode", CASES)
