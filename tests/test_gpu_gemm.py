@@ -120,6 +120,10 @@ def test_grouped_gemm_bwd(cuda_lib, T, d, f, E, k, dt, mode, dw_fp32):
     assert rel(dH13, ref_dH) < TOL
     assert rel(dxp, ref_dX) < TOL
     assert not torch.isnan(dH13).any() and not torch.isnan(dxp).any()
+    # the references start from the GPU's own bf16 H13 and dH13, so per row only
+    # accumulation and output rounding remain
+    assert row_rel(dH13, ref_dH).max() < 1e-2
+    assert row_rel(dxp, ref_dX).max() < 1e-2
 
 
 def test_accumulate_dw(cuda_lib):

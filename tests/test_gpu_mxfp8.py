@@ -101,6 +101,9 @@ def test_mxfp8_grouped_gemm_bwd(cuda_lib, T, d, f, E, k, mode):
         assert rel(dW13[e], mxq(dHg[s], 0).T @ mxq(X[s], 0)) < TOL_MX, ("dW13", e)
     assert rel(dH13, ref_dH) < TOL_MX
     assert rel(dxp, ref_dX) < TOL_MX
+    # the references quantise the same bf16 dY, H13 and dH13 the GPU quantised
+    assert row_rel(dH13, ref_dH).max() < 1e-2
+    assert row_rel(dxp, ref_dX).max() < 1e-2
 
 
 @pytest.mark.parametrize("T,d,E,k,f", [(700, 256, 8, 4, 128), (2000, 512, 128, 8, 256)])
