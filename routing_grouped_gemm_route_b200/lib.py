@@ -116,10 +116,17 @@ def status_string(status: int) -> str:
 
 
 def _ptr(t):
+    """Device address of a tensor argument.  The kernels read every buffer as a dense
+    row-major array in device memory, so a host tensor (whose address a kernel cannot
+    read) or a strided view is refused here, before anything is launched."""
     if t is None:
         return None
     if isinstance(t, int):
         return t
+    if not t.is_cuda:
+        raise ValueError("moe: tensor arguments must live in device memory")
+    if not t.is_contiguous():
+        raise ValueError("moe: tensor arguments must be contiguous (dense row-major)")
     return t.data_ptr()
 
 

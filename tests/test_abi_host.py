@@ -161,3 +161,17 @@ def test_pointer_and_workspace_errors_before_any_launch(L):
 def test_status_strings(L):
     for code in (0, -1, -2, -3, -4, -5, -6):
         assert lib.status_string(code) not in ("", "unknown status")
+
+
+def test_binding_refuses_host_and_strided_tensors():
+    """The binding passes raw addresses to device kernels: a host tensor or a strided
+    view is refused before the library is called."""
+    import torch
+    with pytest.raises(ValueError, match="device memory"):
+        lib._ptr(torch.zeros(4, 4))
+    t = torch.zeros(4, 4)
+    if torch.cuda.is_available():
+        t = t.cuda()
+        with pytest.raises(ValueError, match="contiguous"):
+            lib._ptr(t.t())
+    assert lib._ptr(None) is None and lib._ptr(1234) == 1234
