@@ -211,14 +211,14 @@ def host_inputs(w, dev_inp: dict) -> dict:
 
 
 def cpu_baseline(w, inp_cpu, target_s: float) -> dict:
-    """Oracle tokens/s on a bounded token sample: grown (at most 4 calls, each at most 4x
+    """Oracle tokens/s on a bounded token sample: grown (at most 5 calls, each at most 4x
     the last) until one call takes about target_s seconds."""
     # MXFP8: the oracle quantises the weights of every expert a sample touches (several
     # seconds per expert at d=4096), so the sample is one token (its k experts) and stays so
     mx = w.dtype == "mxfp8"
     T_s = min(1 if mx else 64, w.T)
     t = oracle_sample_run(w, inp_cpu, T_s)
-    for _ in range(0 if mx else 3):
+    for _ in range(0 if mx else 4):
         if t >= 0.6 * target_s or T_s >= w.T:
             break
         T_s = int(min(w.T, max(T_s + 1, T_s * min(4.0, target_s / max(t, 1e-3)))))
