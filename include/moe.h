@@ -220,13 +220,18 @@ moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm,
                                 const int32_t* offsets, void* H13, void* a, void* y_perm,
                                 void* ws, size_t ws_bytes, void* stream);
 
-/* S8, weighted combine: y[t] = sum_j gates[t,j] * y_perm[slot[t,j]], summed in fp32.
- * y_perm [R,d] act -> y [T,d] act.  A gather: no atomics, deterministic. */
+/* S8, weighted combine (deniz.in, "Hedeflediği kapasite sorunu": each token passes
+ * through only a few of the stored experts; their outputs, weighted by the token's
+ * gates, are the layer's output):
+ *   y[t] = sum_j gates[t,j] * y_perm[slot[t,j]], summed in fp32.
+ * y_perm [R,d] act -> y [T,d] act (device).  A gather: no atomics, deterministic.  A
+ * slot outside [0,R) sets MOE_DEV_BAD_INDEX and that term is skipped. */
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* gates,
                        const int32_t* slot, void* y, void* ws, size_t ws_bytes,
                        void* stream);
 
-/* S9, backward of the combine and of the gate softmax:
+/* S9, backward (chain rule) of moe_combine and of moe_route's gate softmax; device
+ * buffers:
  *   dy_perm[slot[t,j]] = gates[t,j] * dy[t]                        (act [R,d])
  *   dg[t,j] = <dy[t], y_perm[slot[t,j]]>                            (fp32)
  *   d_logits[t, topk_idx[t,j]] = g_tj * (dg_tj - sum_i g_ti dg_ti), 0 elsewhere  ([T,E] float) */
@@ -259,7 +264,8 @@ moe_status moe_mx_quantize(const void* x, int64_t rows, int32_t cols, const int3
                            int32_t num_segments, int32_t colwise, uint8_t* codes, uint8_t* scales,
                            void* ws, size_t ws_bytes, void* stream);
 
-/* S10-S13, grouped GEMM backward of the SwiGLU experts, per expert e:
+/* S10-S13, backward (chain rule) of moe_grouped_gemm_fwd, scheduled on the device from
+ * `offsets` like it (deniz.in, "Yeni stack nasıl çalışıyor"); per expert e:
  *   dA_e   = dY_e . W2_e                                   (dY_e = rows of dy_perm)
  *   dH1_e  = dA_e * H3_e * s * (1 + H1_e * (1 - s)),  s = sigmoid(H1_e)
  *   dH3_e  = dA_e * silu(H1_e)                            -> dH13 [R,2*d_ff] act
@@ -274,12 +280,15 @@ moe_status moe_grouped_gemm_bwd(const moe_desc* desc, const void* dy_perm, const
                                 void* dx_perm, void* dW13, void* dW2, void* ws,
                                 size_t ws_bytes, void* stream);
 
-/* S14, unpermute-reduce: dx[t] = sum_j dx_perm[slot[t,j]] (fp32 sum, act out). */
+/* S14, backward of moe_dispatch (unpermute-reduce; the adjoint of the row copy):
+ * dx[t] = sum_j dx_perm[slot[t,j]], fp32 sum, act out (device).  A gather: no atomics,
+ * deterministic. */
 moe_status moe_dispatch_bwd(const moe_desc* desc, const void* dx_perm, const int32_t* slot,
                             void* dx, void* ws, size_t ws_bytes, void* stream);
 
-/* Router backward (MOE_FLAG_ROUTER): dx[T,d] += d_logits . Wr^T and
- * dWr[d,E] (act) = x^T . d_logits, fp32 accumulation. */
+/* Router backward (MOE_FLAG_ROUTER), the chain rule of moe_router_logits:
+ * dx[T,d] += d_logits . Wr^T and dWr[d,E] (act) = x^T . d_logits, fp32 accumulation
+ * (device buffers). */
 moe_status moe_router_bwd(const moe_desc* desc, const void* x, const void* Wr,
                           const float* d_logits, void* dx, void* dWr, void* ws,
                           size_t ws_bytes, void* stream);
@@ -303,7 +312,9 @@ typedef struct moe_load_stats_t {
 moe_status moe_load_stats(const int32_t* counts, int32_t E, moe_load_stats_t* out,
                           int32_t* status, void* stream);
 
-/* Whole layer forward: [router] -> route -> dispatch -> grouped GEMM fwd -> combine.
+/* Whole layer forward, the path the write-ups describe end to end (deniz.in, "Yeni
+ * stack nasıl çalışıyor"): [router] -> route -> dispatch -> grouped GEMM fwd -> combine,
+ * in one call with no host synchronisation.
  * logits: injected routing logits [T,E] float, or NULL with MOE_FLAG_ROUTER and Wr.
  * y [T,d] act.  `saved` (moe_saved_layout.total bytes) receives the tensors listed in
  * moe_saved_layout, which moe_layer_bwd reads. */
@@ -312,7 +323,8 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
                          void* saved, size_t saved_bytes, void* ws, size_t ws_bytes,
                          void* stream);
 
-/* Whole layer backward for upstream gradient dy [T,d] act.  Out: dx [T,d] act,
+/* Whole layer backward (the chain rule of moe_layer_fwd, same calls in reverse) for
+ * upstream gradient dy [T,d] act.  Out: dx [T,d] act,
  * d_logits [T,E] float, dW13, dW2 (see moe_grouped_gemm_bwd), and dWr [d,E] act when
  * MOE_FLAG_ROUTER.  x (the forward's input) is required with MOE_FLAG_ROUTER,
  * MOE_FLAG_RECOMPUTE or MOE_FLAG_SHARED_EXPERT and may be NULL otherwise. */
