@@ -25,6 +25,7 @@ CASES = [
     (4096, 1024, 512, 16, 4, "bf16", None),
     (300, 256, 256, 5, 2, "bf16", None),        # d_ff % 256 == 0: every GEMM with tokens as N
     (2048, 512, 256, 33, 4, "bf16", "empty"),   # ... with empty experts and short tails
+    (700, 256, 128, 1024, 8, "bf16", None),     # the largest E: ~5 rows per expert, many empty
 ]
 
 
