@@ -16,7 +16,8 @@ pytestmark = pytest.mark.gpu
 TOL_MX = 3e-2
 
 CASES = [(600, 256, 128, 6, 2, None), (1000, 512, 256, 8, 4, "empty"), (96, 256, 128, 4, 4, None),
-         (3000, 1024, 512, 16, 4, None)]
+         (3000, 1024, 512, 16, 4, None),
+         (700, 256, 128, 1024, 8, None)]   # the largest E: ~5 rows per expert, many empty
 
 
 def make(T, d, f, E, k, mode, seed=0):
