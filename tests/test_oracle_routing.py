@@ -148,3 +148,29 @@ def test_load_stats_no_tokens():
     st = oracle.load_stats([0, 0, 0])
     assert st["total"] == 0 and st["num_empty"] == 3
     assert st["max_over_mean"] == 0.0 and st["cv"] == 0.0
+
+
+def test_route_matches_brute_force_with_many_ties():
+    """Random small routings whose logits come from a 4-value set, so most tokens have
+    tied logits at the top-k boundary: the oracle must still equal the brute-force
+    reading (ties to the lower expert index) in every output."""
+    from hypothesis import given, settings, strategies as st
+
+    @settings(max_examples=80, deadline=None)
+    @given(st.data())
+    def check(data):
+        T = data.draw(st.integers(1, 12))
+        E = data.draw(st.integers(1, 10))
+        k = data.draw(st.integers(1, E))
+        vals = data.draw(st.lists(st.lists(st.sampled_from([-1.0, 0.0, 0.5, 1.0]),
+                                           min_size=E, max_size=E), min_size=T, max_size=T))
+        L = np.array(vals, dtype=np.float32)
+        r = oracle.route(L, k, E)
+        idx, gates, counts, offsets, slot = brute_route(L.tolist(), k)
+        assert np.array_equal(r["topk_idx"], np.array(idx))
+        assert np.allclose(r["gates"], np.array(gates), rtol=1e-14, atol=0)
+        assert np.array_equal(r["counts"], counts)
+        assert np.array_equal(r["offsets"], offsets)
+        assert np.array_equal(r["slot"], np.array(slot))
+
+    check()
