@@ -98,8 +98,8 @@ __device__ __forceinline__ int64_t seg_tile0(const MxSegs& g, int e) {
   return g.rows > 0 ? (int64_t)e * ((g.rows + 127) / 128) : (int64_t)g.tile_pref[e];
 }
 
-// A lane's CPL consecutive bf16 of one row (CPL = 4: two words, 2: one word) and what is
-// done with them: the per-half max of |x|, the codes (one multiplier per column), stores.
+// A lane's CPL consecutive bf16 of one row (CPL = 4: two words) and what is done with
+// them: the per-half max of |x|, the codes (one multiplier per column), stores.
 template <int CPL> struct Lane;
 template <> struct Lane<4> {
   using V = uint2;
@@ -113,16 +113,6 @@ template <> struct Lane<4> {
   static __device__ __forceinline__ void store(uint8_t* p, V v, const float* m) {
     *reinterpret_cast<uint32_t*>(p) = e4m3x2(bf_lo(v.x) * m[0], bf_hi(v.x) * m[1]) |
                                       (e4m3x2(bf_lo(v.y) * m[2], bf_hi(v.y) * m[3]) << 16);
-  }
-};
-template <> struct Lane<2> {
-  using V = uint32_t;
-  static __device__ __forceinline__ V load(const __nv_bfloat16* p) { return __ldg(reinterpret_cast<const uint32_t*>(p)); }
-  static __device__ __forceinline__ V zero() { return 0u; }
-  static __device__ __forceinline__ uint32_t absmax(V v) { return abs2(v); }
-  static __device__ __forceinline__ void absmax_cols(uint32_t* m, V v) { m[0] = __vmaxu2(m[0], abs2(v)); }
-  static __device__ __forceinline__ void store(uint8_t* p, V v, const float* m) {
-    *reinterpret_cast<uint16_t*>(p) = static_cast<uint16_t>(e4m3x2(bf_lo(v) * m[0], bf_hi(v) * m[1]));
   }
 };
 
@@ -144,7 +134,9 @@ __device__ __forceinline__ void row_reduce_scatter(uint32_t (&a)[32], int sub) {
 }
 
 constexpr int kQWarps = 4;                   // warps per CTA
-template <int CPL> constexpr int q_ctas_per_sm(bool both) { return CPL == 4 ? (both ? 3 : 4) : (both ? 5 : 6); }
+// CTAs per SM: 4 (16 warps, <= 128 registers) for one direction; 3 (12 warps) when a
+// tile is quantised both ways, whose live set does not fit 128 registers
+template <int CPL> constexpr int q_ctas_per_sm(bool both) { return both ? 3 : 4; }
 
 // Persistent quantiser; one warp per tile, no shared memory, no barriers.  A tile is one
 // 32-row block of a segment x 32*CPL columns; lane L holds columns CPL*L .. CPL*L+CPL-1
