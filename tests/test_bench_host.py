@@ -1,0 +1,72 @@
+"""Host logic of the bench without a GPU: clock-sample parsing, the peak table, the
+whole-job rate and the DRAM-traffic figure's source check."""
+import json
+import os
+
+import bench
+
+
+class _Done:
+    """Stands in for a sampler process that has already exited."""
+
+    def terminate(self):
+        pass
+
+    def wait(self, timeout=None):
+        return 0
+
+
+def _sampler_with(tmp_path, text):
+    s = bench.ClockSampler(0)
+    f = tmp_path / "clocks.csv"
+    f.write_text(text)
+    s.tmp = open(f, "a")
+    s.proc = _Done()
+    return s
+
+
+def test_clock_sampler_median_max_and_reasons(tmp_path):
+    rows = [
+        "0, 1350, 1965, 812.5, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1400, 1965, 790.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1300, 1965, 805.0, 0x0000000000000008, Active, Not Active, Not Active, Active",
+        "garbage line",
+        "0, [N/A], 1965, 800.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    r = _sampler_with(tmp_path, "\n".join(rows) + "\n").stop()
+    assert r["sm_mhz"] == 1350.0                      # median of the three parsable samples
+    assert r["sm_max_mhz"] == 1965.0 and r["samples"] == 3
+    assert r["power_w_max"] == 812.5
+    assert r["reasons"] == ["hw_slowdown", "sw_power_cap"]
+
+
+def test_clock_sampler_without_samples(tmp_path):
+    assert _sampler_with(tmp_path, "").stop()["reasons"] == ["no samples"]
+    assert bench.ClockSampler(0).stop()["reasons"] == ["nvidia-smi unavailable"]
+
+
+def test_peaks_measured_and_fallback(tmp_path, monkeypatch):
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    fb = bench.peaks()
+    assert fb["source"] == "fallback" and fb["hbm"] == 6650.0 and fb["bf16"] == 1590.0
+    (tmp_path / "MEASURED_PEAKS.json").write_text(json.dumps(
+        {"hbm_gbs": 6548.2, "bf16_tflops": 1652.2, "bf16_tflops_sustained": 1379.2}))
+    m = bench.peaks()
+    assert m["source"] == "measured" and m["bf16_sustained"] == 1379.2 and m["hbm"] == 6548.2
+
+
+def test_whole_job_rate_counts_every_rank():
+    # 2 ranks x 16384 tokens x 10 steps in 40 ms of the slowest rank
+    assert bench.whole_job_rate(2, 16384, 10, 40.0) == 2 * 16384 * 10 / 0.040
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+
+
+def test_traffic_figure_names_its_gemm_source():
+    """profiles/gemm_dram_traffic.json carries the sha256 of the GEMM source its counters
+    were taken from; the bench reports the figure only while that source is unchanged
+    (null otherwise)."""
+    with open(os.path.join(bench.ROOT, "profiles", "gemm_dram_traffic.json")) as fh:
+        tr = json.load(fh)
+    sha = tr["source_sha256"]
+    assert len(sha) == 64 and all(c in "0123456789abcdef" for c in sha)
+    assert tr["bytes_per_step"] > 0 and tr["workload"]
