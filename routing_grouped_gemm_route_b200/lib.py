@@ -130,6 +130,27 @@ def _ptr(t):
     return t.data_ptr()
 
 
+def _arg(t, dtype, numel, name):
+    """_ptr after checking a tensor argument's element type and that it holds at least
+    the `numel` elements the call reads or writes: the library sees only the address,
+    so a buffer of the wrong type or too short would be misread or overrun."""
+    if t is None or isinstance(t, int):
+        return _ptr(t)
+    if t.dtype != dtype:
+        raise ValueError(f"moe: {name} must be {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"moe: {name} holds {t.numel()} elements, the call needs {numel}")
+    return _ptr(t)
+
+
+def _dims(desc):
+    """(T, d, d_ff, E, k, R, act dtype, dW dtype, weight slices) of a descriptor."""
+    act = act_dtype(desc)
+    dw = torch.float32 if desc.flags & MOE_FLAG_DW_FP32 else act
+    nw = desc.E + (1 if desc.flags & MOE_FLAG_SHARED_EXPERT else 0)
+    return desc.T, desc.d, desc.d_ff, desc.E, desc.k, rows_of(desc), act, dw, nw
+
+
 def _stream(stream=None):
     if stream is None:
         if torch.cuda.is_available():
@@ -203,24 +224,38 @@ def _nbytes(t):
 
 # ------------------------------------------------------------------------------ stages
 def moe_router_logits(desc, x, Wr, logits, stream=None):
-    _check(load().moe_router_logits(ctypes.byref(desc), _ptr(x), _ptr(Wr), _ptr(logits),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_router_logits(ctypes.byref(desc), _arg(x, act, T * d, "x"),
+                                    _arg(Wr, act, d * E, "Wr"),
+                                    _arg(logits, torch.float32, T * E, "logits"),
                                     _stream(stream)), "moe_router_logits")
 
 
 def moe_route(desc, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate, ws,
               stream=None):
-    _check(load().moe_route(ctypes.byref(desc), _ptr(logits), _ptr(topk_idx), _ptr(gates),
-                            _ptr(counts), _ptr(offsets), _ptr(slot), _ptr(row_token),
-                            _ptr(row_gate), _ptr(ws), _nbytes(ws), _stream(stream)), "moe_route")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    i32, f32 = torch.int32, torch.float32
+    _check(load().moe_route(ctypes.byref(desc), _arg(logits, f32, T * E, "logits"),
+                            _arg(topk_idx, i32, T * k, "topk_idx"), _arg(gates, f32, T * k, "gates"),
+                            _arg(counts, i32, E, "counts"), _arg(offsets, i32, E + 1, "offsets"),
+                            _arg(slot, i32, T * k, "slot"), _arg(row_token, i32, R, "row_token"),
+                            _arg(row_gate, f32, R, "row_gate"), _ptr(ws),
+                            _nbytes(ws), _stream(stream)), "moe_route")
 
 
 def moe_route_noalloc(desc, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate,
                       stream=None):
     """moe_route for callers that cannot provide a workspace: the scratch lives in a
     fixed static device array inside the library (see include/moe.h)."""
-    _check(load().moe_route_noalloc(ctypes.byref(desc), _ptr(logits), _ptr(topk_idx),
-                                    _ptr(gates), _ptr(counts), _ptr(offsets), _ptr(slot),
-                                    _ptr(row_token), _ptr(row_gate), _stream(stream)),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    i32, f32 = torch.int32, torch.float32
+    _check(load().moe_route_noalloc(ctypes.byref(desc), _arg(logits, f32, T * E, "logits"),
+                                    _arg(topk_idx, i32, T * k, "topk_idx"),
+                                    _arg(gates, f32, T * k, "gates"), _arg(counts, i32, E, "counts"),
+                                    _arg(offsets, i32, E + 1, "offsets"),
+                                    _arg(slot, i32, T * k, "slot"),
+                                    _arg(row_token, i32, R, "row_token"),
+                                    _arg(row_gate, f32, R, "row_gate"), _stream(stream)),
            "moe_route_noalloc")
 
 
@@ -234,53 +269,90 @@ def moe_mx_scale_bytes(rows, cols, num_segments) -> int:
 def moe_mx_quantize(x, seg_offsets, colwise, codes, scales, ws, stream=None):
     """MXFP8 quantisation of bf16 x [rows, cols] in row segments (see include/moe.h)."""
     rows, cols = x.shape
-    _check(load().moe_mx_quantize(_ptr(x), rows, cols, _ptr(seg_offsets),
-                                  seg_offsets.numel() - 1, 1 if colwise else 0, _ptr(codes),
-                                  _ptr(scales), _ptr(ws), _nbytes(ws), _stream(stream)),
+    nseg = seg_offsets.numel() - 1
+    nsf = moe_mx_scale_bytes(rows, cols, nseg)
+    _check(load().moe_mx_quantize(_arg(x, torch.bfloat16, rows * cols, "x"), rows, cols,
+                                  _arg(seg_offsets, torch.int32, nseg + 1, "seg_offsets"), nseg,
+                                  1 if colwise else 0, _arg(codes, torch.uint8, rows * cols, "codes"),
+                                  _arg(scales, torch.uint8, nsf, "scales"), _ptr(ws), _nbytes(ws),
+                                  _stream(stream)),
            "moe_mx_quantize")
 
 
 def moe_dispatch(desc, x, slot, x_perm, ws, x_perm_sf=None, stream=None):
-    _check(load().moe_dispatch(ctypes.byref(desc), _ptr(x), _ptr(slot), _ptr(x_perm),
-                               _ptr(x_perm_sf), _ptr(ws), _nbytes(ws), _stream(stream)),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_dispatch(ctypes.byref(desc), _arg(x, act, T * d, "x"),
+                               _arg(slot, torch.int32, T * k, "slot"),
+                               _arg(x_perm, act, R * d, "x_perm"), _ptr(x_perm_sf), _ptr(ws),
+                               _nbytes(ws), _stream(stream)),
            "moe_dispatch")
 
 
 def moe_grouped_gemm_fwd(desc, x_perm, W13, W2, offsets, H13, a, y_perm, ws, x_perm_sf=None,
                          stream=None):
-    _check(load().moe_grouped_gemm_fwd(ctypes.byref(desc), _ptr(x_perm), _ptr(x_perm_sf),
-                                       _ptr(W13), _ptr(W2), _ptr(offsets), _ptr(H13), _ptr(a),
-                                       _ptr(y_perm), _ptr(ws), _nbytes(ws), _stream(stream)),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_grouped_gemm_fwd(ctypes.byref(desc), _arg(x_perm, act, R * d, "x_perm"),
+                                       _ptr(x_perm_sf), _arg(W13, act, E * 2 * f * d, "W13"),
+                                       _arg(W2, act, E * d * f, "W2"),
+                                       _arg(offsets, torch.int32, E + 1, "offsets"),
+                                       _arg(H13, act, R * 2 * f, "H13"), _arg(a, act, R * f, "a"),
+                                       _arg(y_perm, act, R * d, "y_perm"), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)),
            "moe_grouped_gemm_fwd")
 
 
 def moe_combine(desc, y_perm, gates, slot, y, ws, stream=None):
-    _check(load().moe_combine(ctypes.byref(desc), _ptr(y_perm), _ptr(gates), _ptr(slot), _ptr(y),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_combine(ctypes.byref(desc), _arg(y_perm, act, R * d, "y_perm"),
+                              _arg(gates, torch.float32, T * k, "gates"),
+                              _arg(slot, torch.int32, T * k, "slot"), _arg(y, act, T * d, "y"),
                               _ptr(ws), _nbytes(ws), _stream(stream)), "moe_combine")
 
 
 def moe_combine_bwd(desc, dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits, ws, stream=None):
-    _check(load().moe_combine_bwd(ctypes.byref(desc), _ptr(dy), _ptr(y_perm), _ptr(gates),
-                                  _ptr(topk_idx), _ptr(slot), _ptr(dy_perm), _ptr(d_logits),
-                                  _ptr(ws), _nbytes(ws), _stream(stream)), "moe_combine_bwd")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    i32, f32 = torch.int32, torch.float32
+    _check(load().moe_combine_bwd(ctypes.byref(desc), _arg(dy, act, T * d, "dy"),
+                                  _arg(y_perm, act, R * d, "y_perm"),
+                                  _arg(gates, f32, T * k, "gates"),
+                                  _arg(topk_idx, i32, T * k, "topk_idx"),
+                                  _arg(slot, i32, T * k, "slot"),
+                                  _arg(dy_perm, act, R * d, "dy_perm"),
+                                  _arg(d_logits, f32, T * E, "d_logits"), _ptr(ws), _nbytes(ws),
+                                  _stream(stream)), "moe_combine_bwd")
 
 
 def moe_grouped_gemm_bwd(desc, dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13,
                          dW2, ws, stream=None):
-    _check(load().moe_grouped_gemm_bwd(ctypes.byref(desc), _ptr(dy_perm), _ptr(x_perm), _ptr(H13),
-                                       _ptr(a), _ptr(W13), _ptr(W2), _ptr(offsets), _ptr(dH13),
-                                       _ptr(dx_perm), _ptr(dW13), _ptr(dW2), _ptr(ws),
-                                       _nbytes(ws), _stream(stream)), "moe_grouped_gemm_bwd")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_grouped_gemm_bwd(ctypes.byref(desc), _arg(dy_perm, act, R * d, "dy_perm"),
+                                       _arg(x_perm, act, R * d, "x_perm"),
+                                       _arg(H13, act, R * 2 * f, "H13"), _arg(a, act, R * f, "a"),
+                                       _arg(W13, act, E * 2 * f * d, "W13"),
+                                       _arg(W2, act, E * d * f, "W2"),
+                                       _arg(offsets, torch.int32, E + 1, "offsets"),
+                                       _arg(dH13, act, R * 2 * f, "dH13"),
+                                       _arg(dx_perm, act, R * d, "dx_perm"),
+                                       _arg(dW13, dw, E * 2 * f * d, "dW13"),
+                                       _arg(dW2, dw, E * d * f, "dW2"), _ptr(ws), _nbytes(ws),
+                                       _stream(stream)), "moe_grouped_gemm_bwd")
 
 
 def moe_dispatch_bwd(desc, dx_perm, slot, dx, ws, stream=None):
-    _check(load().moe_dispatch_bwd(ctypes.byref(desc), _ptr(dx_perm), _ptr(slot), _ptr(dx),
-                                   _ptr(ws), _nbytes(ws), _stream(stream)), "moe_dispatch_bwd")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_dispatch_bwd(ctypes.byref(desc), _arg(dx_perm, act, R * d, "dx_perm"),
+                                   _arg(slot, torch.int32, T * k, "slot"),
+                                   _arg(dx, act, T * d, "dx"), _ptr(ws), _nbytes(ws),
+                                   _stream(stream)), "moe_dispatch_bwd")
 
 
 def moe_router_bwd(desc, x, Wr, d_logits, dx, dWr, ws, stream=None):
-    _check(load().moe_router_bwd(ctypes.byref(desc), _ptr(x), _ptr(Wr), _ptr(d_logits), _ptr(dx),
-                                 _ptr(dWr), _ptr(ws), _nbytes(ws), _stream(stream)),
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_router_bwd(ctypes.byref(desc), _arg(x, act, T * d, "x"),
+                                 _arg(Wr, act, d * E, "Wr"),
+                                 _arg(d_logits, torch.float32, T * E, "d_logits"),
+                                 _arg(dx, act, T * d, "dx"), _arg(dWr, act, d * E, "dWr"), _ptr(ws),
+                                 _nbytes(ws), _stream(stream)),
            "moe_router_bwd")
 
 
@@ -293,7 +365,8 @@ def moe_load_stats(counts, out, status=None, stream=None):
     device word for MOE_DEV_BAD_OFFSETS."""
     if out.numel() * out.element_size() < LOAD_STATS_BYTES:
         raise MoEError(MOE_EWORKSPACE, "moe_load_stats")
-    _check(load().moe_load_stats(_ptr(counts), int(counts.numel()), _ptr(out), _ptr(status),
+    _check(load().moe_load_stats(_arg(counts, torch.int32, 0, "counts"), int(counts.numel()),
+                                 _ptr(out), _arg(status, torch.int32, 1, "status"),
                                  _stream(stream)), "moe_load_stats")
 
 
@@ -305,16 +378,26 @@ def decode_load_stats(out) -> dict:
 
 
 def moe_layer_fwd(desc, x, logits, Wr, W13, W2, y, saved, ws, stream=None):
-    _check(load().moe_layer_fwd(ctypes.byref(desc), _ptr(x), _ptr(logits), _ptr(Wr), _ptr(W13),
-                                _ptr(W2), _ptr(y), _ptr(saved), _nbytes(saved), _ptr(ws),
-                                _nbytes(ws), _stream(stream)), "moe_layer_fwd")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_layer_fwd(ctypes.byref(desc), _arg(x, act, T * d, "x"),
+                                _arg(logits, torch.float32, T * E, "logits"),
+                                _arg(Wr, act, d * E, "Wr"), _arg(W13, act, nw * 2 * f * d, "W13"),
+                                _arg(W2, act, nw * d * f, "W2"), _arg(y, act, T * d, "y"),
+                                _ptr(saved), _nbytes(saved), _ptr(ws), _nbytes(ws),
+                                _stream(stream)), "moe_layer_fwd")
 
 
 def moe_layer_bwd(desc, dy, x, saved, W13, W2, Wr, dx, d_logits, dW13, dW2, dWr, ws, stream=None):
-    _check(load().moe_layer_bwd(ctypes.byref(desc), _ptr(dy), _ptr(x), _ptr(saved), _nbytes(saved),
-                                _ptr(W13), _ptr(W2), _ptr(Wr), _ptr(dx), _ptr(d_logits),
-                                _ptr(dW13), _ptr(dW2), _ptr(dWr), _ptr(ws), _nbytes(ws),
-                                _stream(stream)), "moe_layer_bwd")
+    T, d, f, E, k, R, act, dw, nw = _dims(desc)
+    _check(load().moe_layer_bwd(ctypes.byref(desc), _arg(dy, act, T * d, "dy"),
+                                _arg(x, act, T * d, "x"), _ptr(saved), _nbytes(saved),
+                                _arg(W13, act, nw * 2 * f * d, "W13"),
+                                _arg(W2, act, nw * d * f, "W2"), _arg(Wr, act, d * E, "Wr"),
+                                _arg(dx, act, T * d, "dx"),
+                                _arg(d_logits, torch.float32, T * E, "d_logits"),
+                                _arg(dW13, dw, nw * 2 * f * d, "dW13"),
+                                _arg(dW2, dw, nw * d * f, "dW2"), _arg(dWr, act, d * E, "dWr"),
+                                _ptr(ws), _nbytes(ws), _stream(stream)), "moe_layer_bwd")
 
 
 # ------------------------------------------------------------------------------ views

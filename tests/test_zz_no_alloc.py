@@ -8,6 +8,8 @@ ABI, that two calls in a row give exactly what moe_route gives with a workspace,
 that a problem too large for the static array is refused before anything runs.  It is
 collected last so a failure here never hides the other tests.
 """
+import ctypes
+
 import pytest
 import torch
 
@@ -58,6 +60,11 @@ def test_noalloc_route_refuses_problems_beyond_its_scratch(cuda_lib):
     T = 256 * (lib.MOE_ROUTE_NOALLOC_SCRATCH_BYTES // (8 * E) + 1)
     desc = lib.make_desc(T, 128, 64, E, 2, "bf16")
     small = _outputs(1, E, 2)
-    with pytest.raises(lib.MoEError) as ei:
-        lib.moe_route_noalloc(desc, torch.zeros(1, E, device="cuda"), *_args(small))
-    assert ei.value.status == lib.MOE_EWORKSPACE
+    logits = torch.zeros(1, E, device="cuda")
+    # the library itself refuses (buffers sized for one token: nothing may run) ...
+    st = lib.load().moe_route_noalloc(ctypes.byref(desc), logits.data_ptr(),
+                                      *[t.data_ptr() for t in _args(small)], lib._stream())
+    assert st == lib.MOE_EWORKSPACE
+    # ... and the binding does not let buffers this short through in the first place
+    with pytest.raises(ValueError):
+        lib.moe_route_noalloc(desc, logits, *_args(small))
