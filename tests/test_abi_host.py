@@ -175,3 +175,26 @@ def test_binding_refuses_host_and_strided_tensors():
         with pytest.raises(ValueError, match="contiguous"):
             lib._ptr(t.t())
     assert lib._ptr(None) is None and lib._ptr(1234) == 1234
+
+
+def test_binding_checks_element_types_and_sizes():
+    """Each tensor argument is checked against the descriptor (element type, at least
+    the elements the call touches) before the library is called."""
+    import torch
+    T, d, E, k = 8, 128, 4, 2
+    desc = lib.make_desc(T, d, 64, E, k, "bf16")
+    slot = torch.zeros(T, k, dtype=torch.int32)
+    x_perm = torch.zeros(T * k, d, dtype=torch.bfloat16)
+    ws = torch.zeros(16, dtype=torch.uint8)
+    with pytest.raises(ValueError, match="x must be torch.bfloat16"):
+        lib.moe_dispatch(desc, torch.zeros(T, d, dtype=torch.float32), slot, x_perm, ws)
+    with pytest.raises(ValueError, match="x holds"):
+        lib.moe_dispatch(desc, torch.zeros(T - 1, d, dtype=torch.bfloat16), slot, x_perm, ws)
+    # (arguments before the one under test are raw addresses, which pass unchecked; the
+    # library is never reached because a later argument is refused)
+    with pytest.raises(ValueError, match="slot must be torch.int32"):
+        lib.moe_dispatch(desc, 0x1000, slot.long(), x_perm, ws)
+    with pytest.raises(ValueError, match="x_perm holds"):
+        lib.moe_dispatch(desc, 0x1000, 0x2000, x_perm[:-1], ws)
+    with pytest.raises(ValueError, match="logits must be torch.float32"):
+        lib.moe_router_logits(desc, 0x1000, 0x2000, torch.zeros(T, E, dtype=torch.bfloat16))
