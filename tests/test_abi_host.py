@@ -198,3 +198,25 @@ def test_binding_checks_element_types_and_sizes():
         lib.moe_dispatch(desc, 0x1000, 0x2000, x_perm[:-1], ws)
     with pytest.raises(ValueError, match="logits must be torch.float32"):
         lib.moe_router_logits(desc, 0x1000, 0x2000, torch.zeros(T, E, dtype=torch.bfloat16))
+
+
+def test_product_code_never_reaches_the_oracle():
+    """The package (binding, input generators, build) and the CUDA sources share nothing
+    with oracle/: no import, include or path to it.  Only tests, the smoke check and the
+    bench's CPU-baseline / reference legs may use the oracle."""
+    pkg = os.path.join(ROOT, "routing_grouped_gemm_route_b200")
+    pat = re.compile(r"(^|\W)(import\s+oracle|from\s+oracle|oracle/|\"oracle|'oracle)")
+    bad = []
+    for dirpath, _, files in os.walk(pkg):
+        for name in files:
+            if name.endswith((".py", ".cu", ".cuh", ".h", ".cpp")):
+                path = os.path.join(dirpath, name)
+                with open(path, encoding="utf-8") as fh:
+                    for i, line in enumerate(fh, 1):
+                        if pat.search(line):
+                            bad.append(f"{os.path.relpath(path, ROOT)}:{i}")
+    for name in os.listdir(os.path.join(ROOT, "include")):
+        with open(os.path.join(ROOT, "include", name), encoding="utf-8") as fh:
+            if "oracle" in fh.read():
+                bad.append(f"include/{name}")
+    assert not bad, bad
