@@ -50,10 +50,15 @@ extern "C" moe_status moe_route_noalloc(const moe_desc* desc, const float* logit
   moe_status st = moe_check_desc(desc);
   if (st != MOE_OK) return st;
   const moe_desc& d = *desc;
-  // scratch: histogram [ctas][E] then CTA bases [ctas][E], int32 each, 256-byte aligned
-  const size_t part = size_t(route_ctas(d.T)) * d.E * sizeof(int32_t);
-  const size_t part_al = (part + 255) / 256 * 256;
-  if (part_al + part > size_t(MOE_ROUTE_NOALLOC_SCRATCH_BYTES)) return MOE_EWORKSPACE;
+  // The padded layout flags tokens beyond an expert's capacity in a status word, and
+  // this call has none to report it through: refused rather than dropped silently.
+  if (d.capacity > 0) return MOE_EUNSUPPORTED;
+  // scratch: histogram [ceil(T/64)][E] then slot-CTA bases [ceil(T/256)][E], int32 each,
+  // 256-byte aligned
+  const size_t hist_bytes = size_t(route_hist_rows(d.T)) * d.E * sizeof(int32_t);
+  const size_t base_bytes = size_t(route_ctas(d.T)) * d.E * sizeof(int32_t);
+  const size_t part_al = (hist_bytes + 255) / 256 * 256;
+  if (part_al + base_bytes > size_t(MOE_ROUTE_NOALLOC_SCRATCH_BYTES)) return MOE_EWORKSPACE;
   if (!counts || !offsets) return MOE_EINVAL;
   if (!aligned16(counts) || !aligned16(offsets)) return MOE_EALIGN;
   const void* tok[] = {logits, topk_idx, gates, slot, row_token, row_gate};
@@ -71,8 +76,9 @@ extern "C" moe_status moe_route_noalloc(const moe_desc* desc, const float* logit
   st = scratch_address(&base);
   if (st != MOE_OK) return st;
   // Both scratch arrays are written in full before they are read, so nothing has to
-  // be cleared between calls.  No status word: routing produces its own indices, so
-  // no index can be out of range here.
+  // be cleared between calls.  No status word: in the ragged layout routing writes
+  // only expert indices it selected itself (always in [0, E)) and slots inside its own
+  // counts, so the kernels have no error to flag.
   int32_t* hist = reinterpret_cast<int32_t*>(base);
   int32_t* cta_base = reinterpret_cast<int32_t*>(static_cast<char*>(base) + part_al);
   return launch_route(d, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate, hist,

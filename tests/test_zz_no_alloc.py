@@ -4,15 +4,19 @@ Some callers own every device buffer themselves (a host framework or plugin that
 its memory ahead and passes only inputs and outputs) or must not call cudaMalloc on a
 latency-critical path, since it synchronises the device.  For them the library keeps
 the routing scratch in a fixed static device array.  This file checks, through the C
-ABI, that two calls in a row give exactly what moe_route gives with a workspace, and
-that a problem too large for the static array is refused before anything runs.  It is
-collected last so a failure here never hides the other tests.
+ABI, that two calls in a row give exactly what moe_route gives with a workspace and
+what the fp64 oracle gives, that a problem too large for the static array is refused
+before anything runs, and that the capacity-padded layout (whose overflow it could not
+report) is refused too.  It is collected last so a failure here never hides the other
+tests.
 """
 import ctypes
 
+import numpy as np
 import pytest
 import torch
 
+import oracle
 from routing_grouped_gemm_route_b200 import lib
 from routing_grouped_gemm_route_b200.inputs import random_logits
 
@@ -52,12 +56,19 @@ def test_noalloc_route_matches_workspace_route_twice(cuda_lib, T, E, k, skew):
         assert torch.max(torch.abs(got["row_gate"] - ref["row_gate"])).item() < 2e-6
         assert int(got["counts"].sum()) == T * k
         assert lib.moe_read_device_status(ws) == 0
+        # and against the oracle: indices, counts, offsets and the permutation bit-exact
+        ref = oracle.route(L.cpu().numpy().astype(np.float64), k, E)
+        for name in ("topk_idx", "counts", "offsets", "slot", "row_token"):
+            assert np.array_equal(got[name].cpu().numpy().astype(np.int64),
+                                  np.asarray(ref[name]).reshape(got[name].shape)), (call, name)
+        assert np.max(np.abs(got["gates"].cpu().double().numpy() - ref["gates"])) < 2e-6
 
 
 def test_noalloc_route_refuses_problems_beyond_its_scratch(cuda_lib):
-    # 2 * ceil(T/256) * E * 4 bytes above the fixed array: refused before any launch
+    # (ceil(T/64) + ceil(T/256)) * E * 4 bytes (20 * E per 256 tokens) above the fixed
+    # array: refused before any launch
     E = 1024
-    T = 256 * (lib.MOE_ROUTE_NOALLOC_SCRATCH_BYTES // (8 * E) + 1)
+    T = 256 * (lib.MOE_ROUTE_NOALLOC_SCRATCH_BYTES // (20 * E) + 1)
     desc = lib.make_desc(T, 128, 64, E, 2, "bf16")
     small = _outputs(1, E, 2)
     logits = torch.zeros(1, E, device="cuda")
@@ -68,3 +79,17 @@ def test_noalloc_route_refuses_problems_beyond_its_scratch(cuda_lib):
     # ... and the binding does not let buffers this short through in the first place
     with pytest.raises(ValueError):
         lib.moe_route_noalloc(desc, logits, *_args(small))
+
+
+def test_noalloc_route_refuses_the_padded_layout(cuda_lib):
+    # capacity > 0 can overflow an expert; with no status word to report it, the call
+    # refuses the layout before any launch instead of dropping tokens silently
+    T, E, k = 1000, 16, 2
+    desc = lib.make_desc(T, 128, 64, E, k, "bf16", capacity=(T * k) // E)
+    o = _outputs(T, E, k)
+    o["row_token"] = torch.empty(E * desc.capacity, dtype=torch.int32, device="cuda")
+    o["row_gate"] = torch.empty(E * desc.capacity, dtype=torch.float32, device="cuda")
+    L = random_logits(T, E, seed=5).cuda()
+    with pytest.raises(lib.MoEError) as err:
+        lib.moe_route_noalloc(desc, L, *_args(o))
+    assert err.value.status == lib.MOE_EUNSUPPORTED
