@@ -84,6 +84,15 @@ typedef enum moe_dtype {
  * It runs as the grouped GEMM with one segment of all T tokens; x is required in
  * moe_layer_bwd.  Not with MOE_MXFP8 (MOE_EUNSUPPORTED). */
 #define MOE_FLAG_SHARED_EXPERT 16
+/* Test hook, off by default; the paper has no counterpart.  Every expert grouped-GEMM
+ * launch (routed and shared experts) made under a descriptor with this flag issues no
+ * operand loads and gives each of its
+ * device waits 10 ms instead of 2 s, so the waits run out: the call sets
+ * MOE_DEV_TIMEOUT in the workspace status word, writes none of its GEMM outputs, frees
+ * the tensor memory it took and returns.  It exists so the bounded-wait and teardown
+ * path can be exercised without faulting a GPU; after it, clear the status word with
+ * moe_workspace_init before the next call. */
+#define MOE_FLAG_TEST_WAIT_TIMEOUT (1 << 30)
 
 /* device status bits */
 #define MOE_DEV_BAD_INDEX   1  /* an expert index or slot was out of range; the row was skipped */
@@ -168,7 +177,9 @@ moe_status moe_router_logits(const moe_desc* desc, const void* x, const void* Wr
  *      slot [T,k] int32: row of pair (t,j) in the expert-sorted order, rows of one
  *      expert in token order: slot[t,j] = offsets[e] + #{t' < t routed to e};
  *      row_token [R] int32 and row_gate [R] float: token and gate of each sorted row.
- * Every output is fully written; counts/offsets never leave the device. */
+ * Every output is fully written; counts/offsets never leave the device.  A NaN logit
+ * ranks as -inf (so a token always gets k distinct experts in [0,E)); a token whose
+ * kept logits are all -inf gets NaN gates. */
 moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_idx,
                      float* gates, int32_t* counts, int32_t* offsets, int32_t* slot,
                      int32_t* row_token, float* row_gate, void* ws, size_t ws_bytes,
@@ -182,12 +193,17 @@ moe_status moe_route(const moe_desc* desc, const float* logits, int32_t* topk_id
  * own -- for example a host framework or plugin that plans every device buffer ahead
  * and passes only its input and output tensors, or a latency-critical caller that
  * must not call cudaMalloc because it synchronises the device.
- * Same arguments, outputs and results as moe_route, minus ws/ws_bytes.  Its scratch
- * (per-CTA expert histograms and bases, 2 * ceil(T/256) * E int32) lives in one
- * static device array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES that every GPU which loads
- * this library holds until the process exits; a descriptor that needs more returns
- * MOE_EWORKSPACE before any launch (with E = 128 that allows T up to about 1M tokens,
- * with E = 1024 about 130k).  The call allocates nothing and frees nothing.
+ * Same arguments, outputs and results as moe_route, minus ws/ws_bytes, for the
+ * ragged layout only: a descriptor with capacity > 0 returns MOE_EUNSUPPORTED before
+ * any launch (the padded layout reports a capacity below an expert's count through
+ * the workspace status word, which this call does not have; with capacity 0 routing
+ * writes only indices it produced itself, so no device-side error can arise).  Its scratch
+ * (expert histograms per 64 tokens and bases per 256 tokens, (ceil(T/64) + ceil(T/256))
+ * * E int32) lives in one static device array of MOE_ROUTE_NOALLOC_SCRATCH_BYTES that
+ * every GPU which loads this library holds until the process exits; a descriptor that
+ * needs more returns MOE_EWORKSPACE before any launch (with E = 128 that allows T up to
+ * about 419k tokens, with E = 1024 about 52k).  The call allocates nothing and frees
+ * nothing.
  * The first call on a device looks up the array's device address (once per device,
  * with that device current); make that first call before any stream capture.
  * All calls share the one array and it keeps the last call's contents (every call

@@ -12,10 +12,14 @@ namespace moe {
 int num_sms();
 
 // ----------------------------------------------------------------------------- routing
-// Tokens per routing CTA (8 warps x 32 tokens); the histogram has one row per CTA.
+// Top-k CTAs take 64 tokens each and write one row of the expert histogram; the slot
+// CTAs take 256 (8 warps x 32 tokens) and read the expert bases at their first token.
+constexpr int kRouteTokensPerHistRow = 64;
 constexpr int kRouteTokensPerCta = 256;
+inline int route_hist_rows(int T) { return (T + kRouteTokensPerHistRow - 1) / kRouteTokensPerHistRow; }
 inline int route_ctas(int T) { return (T + kRouteTokensPerCta - 1) / kRouteTokensPerCta; }
 
+// hist: route_hist_rows(T) x E int32; cta_base: route_ctas(T) x E int32 (scratch).
 cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
                          int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
                          float* row_gate, int32_t* hist, int32_t* cta_base, int* status,
@@ -87,6 +91,7 @@ struct GemmShape {
   int E, R, d, f;
   bool fp32;   // fp32 storage / TF32 MMA, else bf16
   bool mx;     // bf16 storage, MXFP8 (E4M3 + E8M0 per 32) GEMM operands
+  bool test_stall = false;   // MOE_FLAG_TEST_WAIT_TIMEOUT: no loads, 10 ms waits
 };
 // FC1 (+SwiGLU epilogue) and FC2 forward.
 moe_status gemm_fwd(const GemmShape& g, const void* x_perm, const void* W13, const void* W2,

@@ -50,10 +50,10 @@ WsLayout ws_layout(const moe_desc& d) {
   WsLayout w;
   const size_t es = act_bytes(d);
   const size_t R = (size_t)R_of(d);
-  const size_t ctas = (size_t)route_ctas(d.T);
+  const size_t hrows = (size_t)route_hist_rows(d.T), ctas = (size_t)route_ctas(d.T);
   size_t o = 0;
   w.status = o; o += kAlign;
-  w.hist = o; o = up(o + ctas * d.E * 4);
+  w.hist = o; o = up(o + hrows * d.E * 4);
   w.cta_base = o; o = up(o + ctas * d.E * 4);
   w.maps = o; o = up(o + 2 * (size_t)d.E * kTensorMapBytes);
   w.dy_perm = o; o = up(o + R * d.d * es);
@@ -132,7 +132,7 @@ moe_status check(const moe_desc* d) {
     return MOE_EINVAL;
   if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
   if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE |
-                   MOE_FLAG_SHARED_EXPERT))
+                   MOE_FLAG_SHARED_EXPERT | MOE_FLAG_TEST_WAIT_TIMEOUT))
     return MOE_EINVAL;
   if (d->capacity < 0 || (int64_t)d->E * d->capacity >= (int64_t(1) << 31)) return MOE_EINVAL;
   if (d->flags & MOE_FLAG_SHARED_EXPERT) {
@@ -212,6 +212,7 @@ GemmShape gshape(const moe_desc& d, int rows = -1) {
   g.f = d.d_ff;
   g.fp32 = d.dtype == MOE_FP32;
   g.mx = d.dtype == MOE_MXFP8;
+  g.test_stall = (d.flags & MOE_FLAG_TEST_WAIT_TIMEOUT) != 0;
   return g;
 }
 

@@ -8,10 +8,12 @@
 // और मेमोरी तकनीकें").  Three launches, no atomics on global memory, no host sync:
 //   1. topk:  one warp per token, logits in registers, k rounds of warp arg-max
 //             (ties to the lower expert index); gates = softmax over the kept
-//             logits; a per-CTA expert histogram in shared memory.
-//   2. scan:  one CTA: per expert, an exclusive scan of the CTA histograms (the
-//             CTA's base inside the expert), counts, and offsets = exclusive scan
-//             of counts.
+//             logits; an expert histogram per 64 tokens (one CTA each, so even a
+//             few thousand tokens spread over every SM).
+//   2. scan:  one CTA: per expert, an exclusive scan of the histogram rows (each
+//             expert's column split over several threads), giving the base of every
+//             256-token slot CTA inside the expert, the counts, and offsets =
+//             exclusive scan of counts.
 //   3. slots: per warp of 32 tokens, a bitmask per expert of the lanes that chose
 //             it; a token's rank inside the expert is the population count of the
 //             lower lanes' bits plus the bases of earlier warps and CTAs.  So the
@@ -29,15 +31,17 @@ namespace {
 
 constexpr int kWarps = 8;
 static_assert(kWarps * 32 == kRouteTokensPerCta, "one token per lane in the slot pass");
+constexpr int kHistRowsPerCta = kRouteTokensPerCta / kRouteTokensPerHistRow;
+static_assert(kHistRowsPerCta * kRouteTokensPerHistRow == kRouteTokensPerCta, "whole rows");
 
 // a beats b: larger logit, or equal logit and smaller index
 __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
-// Top-k runs up to 32 warps per 256-token CTA (8 tokens a warp): the CTA granularity is
-// the scan's and the slot kernel's, the extra warps hide latency.  Above 256 experts a
-// lane's logits need more registers than 32 warps a CTA allow: 8 warps there.
+// Top-k runs 32 warps per 64-token CTA (2 tokens a warp; the work of a token is a chain
+// of dependent shuffles, so many warps per SM hide it).  Above 256 experts a lane's
+// logits need more registers than 32 warps a CTA allow: 8 warps there.
 template <int NPL>
 constexpr int topk_warps() { return NPL <= 8 ? 32 : 8; }
 
@@ -52,8 +56,8 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
 
-  const int t0 = blockIdx.x * kRouteTokensPerCta;
-  for (int i = warp; i < kRouteTokensPerCta; i += topk_warps<NPL>()) {
+  const int t0 = blockIdx.x * kRouteTokensPerHistRow;
+  for (int i = warp; i < kRouteTokensPerHistRow; i += topk_warps<NPL>()) {
     const int t = t0 + i;
     if (t >= T) break;
     const float* row = logits + (int64_t)t * E;
@@ -62,6 +66,9 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
     for (int c = 0; c < NPL; ++c) {
       const int e = c * 32 + lane;
       v[c] = e < E ? row[e] : -INFINITY;
+      // a NaN logit ranks as -inf (it would lose every comparison, and a row of them
+      // would select no expert at all)
+      if (v[c] != v[c]) v[c] = -INFINITY;
     }
     unsigned taken = 0;           // bit c: v[c] already selected
     float my_val = 0.f;
@@ -101,64 +108,68 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
     if (lane < k) {
       topk_idx[(int64_t)t * k + lane] = my_idx;
       gates[(int64_t)t * k + lane] = z / sum;
-      atomicAdd(&s_hist[my_idx], 1);
+      if (my_idx < E) atomicAdd(&s_hist[my_idx], 1);   // always true for k <= E
     }
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
 }
 
-// One CTA of 1024 threads: per expert the scan over CTA histograms, then offsets.
-// capacity > 0: the padded layout, offsets[e] = e * capacity instead of the scan.
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ hist, int nctas,
+// One CTA of 1024 threads.  Expert e's histogram column (nrows rows of 64 tokens) is
+// cut into J = 1024 / Ep chunks of consecutive rows (Ep = E rounded up to 32), one
+// thread each: a first pass sums the chunk, the chunk sums give each thread its
+// starting base, and a second pass writes the base at every 256-token slot CTA's first
+// row.  Then offsets = exclusive scan of the experts' totals.  capacity > 0: the padded
+// layout, offsets[e] = e * capacity instead.
+__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ hist, int nrows,
                                                     int E, int capacity,
                                                     int32_t* __restrict__ cta_base,
                                                     int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
   __shared__ int s_part[1024];
-  __shared__ int s_carry;
-  if (threadIdx.x == 0) s_carry = 0;
+  const int Ep = (E + 31) & ~31;                  // <= 1024
+  const int J = 1024 / Ep;                        // chunks per expert
+  const int e = threadIdx.x % Ep, j = threadIdx.x / Ep;
+  const bool live = e < E && j < J;
+  const int per = (nrows + J - 1) / J;
+  const int r0 = min(nrows, j * per), r1 = min(nrows, r0 + per);
+  int sum = 0;
+  if (live) {
+#pragma unroll 4
+    for (int r = r0; r < r1; ++r) sum += hist[(int64_t)r * E + e];
+  }
+  if (j < J) s_part[j * Ep + e] = sum;
   __syncthreads();
-  for (int e0 = 0; e0 < E; e0 += 1024) {
-    const int e = e0 + threadIdx.x;
+  int tot = 0;
+  if (live) {
     int run = 0;
-    if (e < E) {
-      int c = 0;
-      for (; c + 4 <= nctas; c += 4) {
-        const int h0 = hist[(int64_t)(c + 0) * E + e];
-        const int h1 = hist[(int64_t)(c + 1) * E + e];
-        const int h2 = hist[(int64_t)(c + 2) * E + e];
-        const int h3 = hist[(int64_t)(c + 3) * E + e];
-        cta_base[(int64_t)(c + 0) * E + e] = run;
-        cta_base[(int64_t)(c + 1) * E + e] = run + h0;
-        cta_base[(int64_t)(c + 2) * E + e] = run + h0 + h1;
-        cta_base[(int64_t)(c + 3) * E + e] = run + h0 + h1 + h2;
-        run += h0 + h1 + h2 + h3;
-      }
-      for (; c < nctas; ++c) {
-        const int h = hist[(int64_t)c * E + e];
-        cta_base[(int64_t)c * E + e] = run;
-        run += h;
-      }
-      counts[e] = run;
+    for (int jj = 0; jj < J; ++jj) {
+      const int v = s_part[jj * Ep + e];
+      if (jj < j) run += v;
+      tot += v;
     }
-    // block-wide inclusive scan of `run` (Hillis-Steele)
-    s_part[threadIdx.x] = run;
-    __syncthreads();
-    for (int o = 1; o < 1024; o <<= 1) {
-      const int add = threadIdx.x >= o ? s_part[threadIdx.x - o] : 0;
-      __syncthreads();
-      s_part[threadIdx.x] += add;
-      __syncthreads();
+#pragma unroll 4
+    for (int r = r0; r < r1; ++r) {
+      if (r % kHistRowsPerCta == 0) cta_base[(int64_t)(r / kHistRowsPerCta) * E + e] = run;
+      run += hist[(int64_t)r * E + e];
     }
-    const int incl = s_part[threadIdx.x];
-    const int carry = s_carry;
-    if (e < E) offsets[e] = capacity > 0 ? e * capacity : carry + incl - run;
+    if (j == 0) counts[e] = tot;
+  }
+  __syncthreads();                                // every chunk sum read
+  // block-wide inclusive scan of the totals (thread i: expert i; Hillis-Steele)
+  if (j == 0 && e < Ep) s_part[e] = e < E ? tot : 0;
+  if (threadIdx.x >= Ep) s_part[threadIdx.x] = 0;
+  __syncthreads();
+  const int x = threadIdx.x;
+  const int own = s_part[x];
+  for (int o = 1; o < 1024; o <<= 1) {
+    const int add = x >= o ? s_part[x - o] : 0;
     __syncthreads();
-    if (threadIdx.x == 1023) s_carry = carry + incl;
+    s_part[x] += add;
     __syncthreads();
   }
-  if (threadIdx.x == 0) offsets[E] = capacity > 0 ? E * capacity : s_carry;
+  if (x < E) offsets[x] = capacity > 0 ? x * capacity : s_part[x] - own;
+  if (x == 1023) offsets[E] = capacity > 0 ? E * capacity : s_part[1023];
 }
 
 __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
@@ -216,7 +227,7 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
 template <int NPL>
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gates,
                         int32_t* hist, cudaStream_t s) {
-  const int ctas = route_ctas(T);
+  const int ctas = route_hist_rows(T);
   topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, E * sizeof(int), s>>>(logits, T, E, k, idx,
                                                                         gates, hist);
   return cudaGetLastError();
@@ -335,7 +346,7 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, s);
   if (err != cudaSuccess) return err;
   const int C = d.capacity;
-  scan_kernel<<<1, 1024, 0, s>>>(hist, ctas, E, C, cta_base, counts, offsets);
+  scan_kernel<<<1, 1024, 0, s>>>(hist, route_hist_rows(T), E, C, cta_base, counts, offsets);
   if ((err = cudaGetLastError()) != cudaSuccess) return err;
   const size_t smem = size_t(2) * kWarps * E * sizeof(int);
   if (smem > 48 * 1024) {

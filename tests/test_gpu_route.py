@@ -76,3 +76,31 @@ def test_route_replays_in_a_cuda_graph_with_new_logits(cuda_lib):
         g.replay()
         torch.cuda.synchronize()
         assert_route_equal(outs, oracle.route(Lh.numpy(), k, E), k)
+
+
+@pytest.mark.parametrize("E,k", [(40, 7), (128, 4)])
+def test_nan_logits_rank_as_minus_infinity(cuda_lib, E, k):
+    """A NaN logit ranks as -inf: every token still gets k distinct experts in range,
+    and the routing equals the oracle's on the logits with NaN replaced by -inf (the
+    reading the library documents; a row of NaNs gets NaN gates)."""
+    T = 3000
+    L = random_logits(T, E, seed=E + k)
+    g = torch.Generator().manual_seed(1)
+    L[0] = float("nan")                                        # a whole row
+    L[1:200][torch.rand(199, E, generator=g) < 0.3] = float("nan")
+    L[200:260, :k + 1] = float("nan")                          # NaN where the top would be
+    desc = lib.make_desc(T, 128, 64, E, k, "bf16")
+    gpu = run_route(desc, L.cuda())
+    Lr = L.clone()
+    Lr[torch.isnan(Lr)] = float("-inf")
+    ref = oracle.route(Lr.numpy(), k, E)
+    idx = gpu["topk_idx"].cpu().numpy()
+    assert idx.min() >= 0 and idx.max() < E
+    assert all(len(set(r)) == k for r in idx.tolist())
+    for name in ("topk_idx", "counts", "offsets", "slot", "row_token"):
+        assert np.array_equal(gpu[name].cpu().numpy().astype(np.int64),
+                              np.asarray(ref[name]).reshape(gpu[name].shape)), name
+    gg = gpu["gates"].cpu().double().numpy()
+    assert np.array_equal(np.isnan(gg), np.isnan(ref["gates"]))
+    fin = ~np.isnan(ref["gates"])
+    assert np.max(np.abs(gg[fin] - ref["gates"][fin])) < 2e-6
