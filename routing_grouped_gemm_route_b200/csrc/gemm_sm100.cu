@@ -91,6 +91,10 @@ struct Params {
   uint8_t* q_sf;
   int q_ld;
   int* status;
+  // Test hook (MOE_FLAG_TEST_WAIT_TIMEOUT): the producers issue no loads, so every wait
+  // for operands runs out after wait_ns and the kernel takes its abort path.
+  int stall;
+  uint64_t wait_ns;        // limit of each bounded wait (2 s; 10 ms with the hook)
 };
 
 __device__ __forceinline__ int64_t sf_chunk(const Params::Sf& f, const int32_t* tile_pref, int e,
@@ -440,10 +444,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       const uint32_t full_leader = PAIR ? map_to_rank(smem_u32(full), 0) : 0u;
       const int arow = PAIR ? static_cast<int>(rank) * BM : 0;         // my rows of A
       const int bcol = PAIR ? static_cast<int>(rank) * C::BNC : 0;     // my rows of B
+      if (p.stall) stop = true;   // test hook: nothing is loaded, nothing is in flight
       for (int t = unit; t < total && !stop; t += n_units) {
         const Tile tl = decode_tile<MODE, BN, C::KB, C::TM>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
         for (int kb = 0; kb < tl.kb; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status)) { stop = true; break; }
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.status, p.wait_ns)) { stop = true; break; }
           uint8_t* sA = tiles + stage * C::STAGE;
           uint8_t* sB = sA + C::A_BYTES;
           if (leader) {
@@ -533,11 +538,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
       for (int t = unit; t < total && !stop; t += n_units) {
         const Tile tl =
             decode_tile<MODE, BN, C::KB, C::TM>(t, n_tiles, m_tiles, s_off, s_mt, E, p.K);
-        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status)) break;
+        if (!mbar_wait(&tempty[acc], acc_phase ^ 1u, abort_flag, p.status, p.wait_ns)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(acc * BN);
         for (int kb = 0; kb < tl.kb; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, p.status)) { stop = true; break; }
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.status, p.wait_ns)) { stop = true; break; }
           tc_fence_after();
           const uint32_t so = static_cast<uint32_t>(stage * C::STAGE) >> 4;
           uint32_t sfa_t = 0, sfb_t = 0;
@@ -569,6 +574,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
           else umma_commit(&empty[stage]);
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
+        // an aborted tile is never handed to the epilogue (its accumulator is incomplete);
+        // the epilogue warps see the abort flag or time out themselves
+        if (stop) break;
         if (PAIR) umma_commit_pair(&tfull[acc], 3);
         else umma_commit(&tfull[acc]);
         if (++acc == C::NACC) { acc = 0; acc_phase ^= 1u; }
@@ -623,7 +631,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
         }
         in_issued = __shfl_sync(0xffffffffu, in_issued, 0);
       }
-      if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, p.status)) break;
+      if (!mbar_wait_warp(&tfull[acc], acc_phase, abort_flag, p.status, p.wait_ns)) break;
       tc_fence_after();
       const uint32_t tb = tmem_base + (static_cast<uint32_t>(q * 32) << 16) +
                           static_cast<uint32_t>(acc * BN);
@@ -780,7 +788,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               tmem_ld_wait();
               reg_fence32(v);
               bits_to_f32(v, fv);
-              if (!mbar_wait_warp(&my_in_full[slot], par, abort_flag, p.status)) break;
+              if (!mbar_wait_warp(&my_in_full[slot], par, abort_flag, p.status, p.wait_ns)) break;
               uint8_t* sl = in_buf + slot * C::IN_CH;
               unstage_row<ActT>(sl, lane, h1);
               unstage_row<ActT>(sl + C::IN_CH / 2, lane, h3);
@@ -1081,6 +1089,8 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.q_sf = mx.q_sf;
   p.q_ld = mx.q_ld;
   p.status = status;
+  p.stall = g.test_stall ? 1 : 0;
+  p.wait_ns = g.test_stall ? 10000000ull : kWaitLimitNs;
   CUtensorMap tsa, tsb;
   if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
   return launch<T, OutT, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
@@ -1113,6 +1123,8 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
   p.sfb = mx.b;
   p.tile_pref = mx.tile_pref;
   p.status = status;
+  p.stall = g.test_stall ? 1 : 0;
+  p.wait_ns = g.test_stall ? 10000000ull : kWaitLimitNs;
   CUtensorMap tsa, tsb;
   if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
   const long long tiles = (long long)g.E * (M / C::TM) * (N / BN);
@@ -1527,7 +1539,7 @@ moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, con
 
 moe_status shared_fwd(const GemmShape& g, const void* x, const void* W13s, const void* W2s,
                       void* H13s, void* as, float* ys, int* status, cudaStream_t s) {
-  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false};
+  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false, g.test_stall};
   if (g.fp32) return gemm::shared_fwd_t<float>(g1, x, W13s, W2s, H13s, as, ys, status, s);
   return gemm::shared_fwd_t<__nv_bfloat16>(g1, x, W13s, W2s, H13s, as, ys, status, s);
 }
@@ -1535,7 +1547,7 @@ moe_status shared_bwd(const GemmShape& g, const void* dy, const void* x, const v
                       const void* as, const void* W13s, const void* W2s, void* dH13s, float* dxs,
                       void* dW13s, void* dW2s, bool dw_fp32, bool dw_accum, void* maps_ws,
                       int* status, cudaStream_t s) {
-  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false};
+  const GemmShape g1{1, g.R, g.d, g.f, g.fp32, false, g.test_stall};
   CUtensorMap* maps = reinterpret_cast<CUtensorMap*>(maps_ws);
   if (g.fp32)
     return gemm::shared_bwd_t<float>(g1, dy, x, H13s, as, W13s, W2s, dH13s, dxs, dW13s, dW2s,

@@ -49,7 +49,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // CTA-wide abort flag is raised or the time limit passes (then it raises the flag and
 // sets MOE_DEV_TIMEOUT in the status word).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                          int* status) {
+                                          int* status, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
@@ -57,7 +57,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 63u) == 0) {
       if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         set_status(status, MOE_DEV_TIMEOUT);
         return false;
@@ -68,8 +68,9 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 // Warp-wide bounded wait: every lane waits, and all lanes agree on the outcome, so a
 // warp never splits in front of a .sync.aligned instruction.
 __device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
-                                               volatile int* abort_flag, int* status) {
-  const bool ok = mbar_wait(bar, parity, abort_flag, status);
+                                               volatile int* abort_flag, int* status,
+                                               uint64_t limit_ns = kWaitLimitNs) {
+  const bool ok = mbar_wait(bar, parity, abort_flag, status, limit_ns);
   return __all_sync(0xffffffffu, ok) != 0;
 }
 // Bounded wait used during teardown (ignores the abort flag).

@@ -171,3 +171,30 @@ def test_bad_offsets_set_status_and_write_nothing(cuda_lib):
     lib.moe_workspace_init(ws)
     lib.moe_grouped_gemm_fwd(desc, xp, W13, W2, bad2, H13, a, yp, ws)
     assert lib.moe_read_device_status(ws) & lib.MOE_DEV_BAD_OFFSETS
+
+
+@pytest.mark.parametrize("dt", ["bf16", "fp32", "mxfp8"])
+def test_bounded_waits_run_out_and_the_next_call_succeeds(cuda_lib, dt):
+    """The bounded-wait path, without faulting anything: with the test hook the GEMMs'
+    producers load nothing, so the MMA and epilogue waits give up after 10 ms.  The call
+    must report MOE_DEV_TIMEOUT, write none of its outputs and leave the context usable:
+    its tensor memory freed (an allocation left behind would stall the next GEMM on that
+    SM) and the next normal call on the same workspace correct against the oracle."""
+    T, d, f, E, k = 256, 128, 128, 4, 2
+    desc, act, r, x, W13, W2, ws, xp = make(T, d, f, E, k, dt, None, seed=5)
+    R = T * k
+    stall = lib.make_desc(T, d, f, E, k, dt, lib.MOE_FLAG_TEST_WAIT_TIMEOUT)
+    H13 = torch.full((R, 2 * f), float("nan"), dtype=act, device="cuda")
+    a = torch.full((R, f), float("nan"), dtype=act, device="cuda")
+    yp = torch.full((R, d), float("nan"), dtype=act, device="cuda")
+    lib.moe_grouped_gemm_fwd(stall, xp, W13, W2, r["offsets"], H13, a, yp, ws)
+    bits = lib.moe_read_device_status(ws)
+    assert bits & lib.MOE_DEV_TIMEOUT
+    assert torch.isnan(H13).all() and torch.isnan(a).all() and torch.isnan(yp).all()
+    lib.moe_workspace_init(ws)
+    H13, a, yp = fwd(desc, act, r, W13, W2, ws, xp)     # asserts a clear status word
+    mx = dt == "mxfp8"
+    refH, refA, refY = oracle.experts_fwd(f64(xp), npi(r["offsets"]), f64(W13), f64(W2), mx=mx)
+    tol = 3e-2 if mx else TOL
+    assert rel(H13, refH) < tol
+    assert rel(yp, refY) < tol
