@@ -187,6 +187,48 @@ def test_padded_layer_is_bit_identical_to_ragged(cuda_lib, T, d, E, k, f, dt, sk
         assert torch.equal(g0[name], g1[name]), name
 
 
+@pytest.mark.parametrize("T,d,E,k,f,dt,skew,extra", [
+    (3000, 256, 16, 4, 128, "bf16", False, 0),
+    (3000, 256, 16, 4, 128, "bf16", True, 37),
+    (2000, 256, 128, 4, 128, "bf16", False, 3),
+    (333, 384, 12, 3, 192, "fp32", False, 11),
+])
+def test_padded_layer_matches_oracle(cuda_lib, T, d, E, k, f, dt, skew, extra):
+    """The capacity-padded layout against the fp64 oracle, not only against the ragged
+    layer: every expert owns C rows (deniz.in, "Yeni stack nasil calisiyor": padding
+    every expert group to a common capacity), offsets are e*C, a token's slot is
+    e*C + its rank among the expert's tokens, padding rows of x_perm are zero and
+    marked row_token = -1, and the layer's outputs match the oracle's."""
+    w = Workload("padx", T, d, E, k, f, dt, router=False, skew=skew, seed=T + 31)
+    inp = make_inputs(w)
+    C = max_count(w, inp)[0] + extra
+    desc, layer, dv, y, g, status = run_layer(w, inp, capacity=C)
+    assert status == 0
+    v = layer.views()
+    x, dy = f64(inp["x"]), f64(inp["dy"])
+    W13, W2 = inp["W13"].float().numpy(), inp["W2"].float().numpy()
+    fwd = oracle.layer_fwd(x, W13, W2, logits=f64(inp["logits"]), k=k)
+    bwd = oracle.layer_bwd(fwd, dy, x, W13, W2)
+    idx = fwd["topk_idx"].astype(np.int64)
+    assert np.array_equal(npi(v["topk_idx"]), idx)
+    assert np.array_equal(npi(v["counts"]), fwd["counts"])
+    assert np.array_equal(npi(v["offsets"]), np.arange(E + 1) * C)
+    rank = fwd["slot"] - fwd["offsets"][idx]
+    assert np.array_equal(npi(v["slot"]), idx * C + rank)
+    rt = npi(v["row_token"]).reshape(E, C)
+    xp = f64(v["x_perm"]).reshape(E, C, d)
+    for e in range(E):
+        c = int(fwd["counts"][e])
+        o = int(fwd["offsets"][e])
+        assert np.array_equal(rt[e, :c], fwd["row_token"][o:o + c])
+        assert np.all(rt[e, c:] == -1)
+        assert np.array_equal(xp[e, :c], x[fwd["row_token"][o:o + c]])
+        assert np.all(xp[e, c:] == 0)
+    assert rel(y, fwd["y"]) < TOL
+    for name in ("dx", "d_logits", "dW13", "dW2"):
+        assert rel(g[name], bwd[name]) < TOL, name
+
+
 def test_capacity_below_the_largest_count_is_reported(cuda_lib):
     w = Workload("capx", 2000, 256, 16, 4, 128, "bf16", router=False, skew=True, seed=3)
     inp = make_inputs(w)
