@@ -52,6 +52,8 @@ def parse():
                     help="one shared expert (dense SwiGLU FFN on every token); the step is then "
                          "timed through the whole-layer calls")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--flushed-reps", type=int, default=10,
+                    help="L2-flushed timings of the HBM-bound stages (0 skips them)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--e2e-steps", type=int, default=30, help="0 skips the end-to-end leg")
     ap.add_argument("--tokens", type=int, default=None,
@@ -71,8 +73,39 @@ def peaks():
             d = json.load(fh)
         return dict(hbm=d["hbm_gbs"], bf16=d["bf16_tflops"],
                     bf16_sustained=d.get("bf16_tflops_sustained", d["bf16_tflops"]),
-                    source="measured")
-    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+                    sm_max_mhz=d.get("sm_max_mhz"), source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback",
+                sm_max_mhz=1965.0)
+
+
+# Nominal B200 figures (context beside the measured denominators): dense bf16 tensor
+# throughput and the HGX HBM3e bandwidth.  Other precisions scale by the nominal ratios.
+NOMINAL_BF16_TFLOPS = 2250.0
+NOMINAL_HBM_GBS = 7700.0
+DTYPE_RATIO = {"bf16": 1.0, "tf32": 1.1 / 2.25, "fp8": 4.5 / 2.25}
+
+
+def tensor_peak(pk: dict, kind: str, clk: dict, timed_s: float) -> dict:
+    """Tensor-core denominators of a GEMM of dtype `kind` timed in this run.
+
+    The measured burst figure (a matmul timed alone, at full clock) applies when the
+    run held the SM clock near its maximum through a short timed region; otherwise the
+    sustained figure (the same matmul looped for seconds under the power cap).  Both
+    fractions are reported, with the nominal dense peak for context."""
+    r = DTYPE_RATIO[kind]
+    burst, sustained = pk["bf16"] * r, pk["bf16_sustained"] * r
+    sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz") or pk.get("sm_max_mhz")
+    at_max = bool(sm and smax and sm >= 0.95 * smax)
+    use_burst = at_max and timed_s < 5.0
+    how = {"bf16": "", "tf32": " x 1.1/2.25 (nominal tf32/bf16)",
+           "fp8": " x 4.5/2.25 (nominal fp8/bf16)"}[kind]
+    why = (f"burst: median SM clock {sm} MHz within 5% of {smax} MHz over a {timed_s:.2f} s "
+           f"timed region" if use_burst else
+           f"sustained: median SM clock {sm} MHz (max {smax} MHz) over a {timed_s:.2f} s "
+           f"timed region")
+    return {"peak": burst if use_burst else sustained, "burst": burst, "sustained": sustained,
+            "nominal": NOMINAL_BF16_TFLOPS * r, "which": "burst" if use_burst else "sustained",
+            "why": why, "kind": f"dense bf16{how}"}
 
 
 def workload_desc(w):
@@ -254,6 +287,24 @@ def run_reference(args, w, world, rank):
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+def flushed_stage_ms(run_stage, names, dev, reps: int) -> dict:
+    """Median CUDA-event time of each named stage run alone after writing a 256 MB
+    buffer (twice the 126 MB L2), so none of its inputs starts in L2."""
+    flush = torch.empty(256 * 2 ** 20, dtype=torch.uint8, device=dev)
+    out = {}
+    for s in names:
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(reps)]
+        for e0, e1 in ev:
+            flush.fill_(1)
+            e0.record()
+            run_stage(s)
+            e1.record()
+        torch.cuda.synchronize()
+        out[s] = statistics.median(e0.elapsed_time(e1) for e0, e1 in ev)
+    return out
 
 
 def run_e2e(args, w, desc, act, dev, world, x, dy, logits, W13, W2, Wr, y, dx, d_logits, dW13,
@@ -525,23 +576,39 @@ def main():
     gemm_flops = {"gemm_fwd": 6.0 * Ra * d * f, "gemm_bwd": 12.0 * Ra * d * f,
                   "re_gemm_fwd": 6.0 * Ra * d * f}
     hbm_bytes = {
-        "route": T * E * 4 + T * k * 12 + Ra * 8 + 2 * 4 * ((T + 255) // 256) * E,
+        # logits in; idx, gates, slot, row_token, row_gate out; the histogram (per 64
+        # tokens) and slot-CTA bases (per 256) written and read once each
+        "route": T * E * 4 + T * k * 12 + Ra * 8 + 2 * 4 * E * ((T + 63) // 64 + (T + 255) // 256),
         "dispatch": T * d * es + T * k * 4 + Ra * d * es,
         "combine": Ra * d * es + T * k * 8 + T * d * es,
         "combine_bwd": T * d * es + 2 * Ra * d * es + T * k * 12 + T * E * 4,
         "dispatch_bwd": Ra * d * es + T * k * 4 + T * d * es,
     }
     hbm_bytes["re_dispatch"] = hbm_bytes["dispatch"]
+    kind = "tf32" if act == torch.float32 else ("fp8" if mx else "bf16")
+    tp = tensor_peak(pk, kind, clk, ms_local / 1e3)
     stage_rep = {}
     for s, ms in stage_ms.items():
         r = {"ms": round(ms, 4)}
         if s in gemm_flops:
             tf = gemm_flops[s] / (ms * 1e-3) / 1e12
-            r.update({"TFLOP/s": round(tf, 1), "frac_of_sustained_bf16": round(tf / pk["bf16_sustained"], 3)})
+            r.update({"TFLOP/s": round(tf, 1), "frac_of_peak": round(tf / tp["peak"], 3),
+                      "frac_of_nominal": round(tf / tp["nominal"], 3)})
         elif s in hbm_bytes:
             gbs = hbm_bytes[s] / (ms * 1e-3) / 1e9
-            r.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm"], 3)})
+            r.update({"GB/s": round(gbs, 1), "frac_of_hbm": round(gbs / pk["hbm"], 3),
+                      "frac_of_nominal_hbm": round(gbs / NOMINAL_HBM_GBS, 3)})
         stage_rep[s] = r
+    if args.flushed_reps > 0:
+        # the HBM-bound stages again, one at a time, each after a 256 MB write that
+        # evicts the 126 MB L2 (the main loop runs them back to back, where a stage can
+        # find part of its input still in L2: combine reads the y_perm FC2 just wrote)
+        flushed = flushed_stage_ms(run_stage, [s for s in stages if s in hbm_bytes], dev,
+                                   args.flushed_reps)
+        for s, ms in flushed.items():
+            gbs = hbm_bytes[s] / (ms * 1e-3) / 1e9
+            stage_rep[s].update({"l2_flushed_ms": round(ms, 4), "l2_flushed_GB/s": round(gbs, 1),
+                                 "l2_flushed_frac_of_hbm": round(gbs / pk["hbm"], 3)})
 
     if layer is None:
         gemm_ms = stage_ms["gemm_fwd"] + stage_ms["gemm_bwd"]
@@ -552,14 +619,7 @@ def main():
         gemm_ms = stage_ms["layer_fwd"] + stage_ms["layer_bwd"]
         gemm_work = 18.0 * (Ra + T) * d * f
     gemm_tflops = gemm_work / (gemm_ms * 1e-3) / 1e12
-    peak_tf = pk["bf16_sustained"]
-    peak_kind = "sustained dense bf16"
-    if act == torch.float32:
-        peak_tf = pk["bf16_sustained"] * 1.1 / 2.25     # TF32 = bf16 x nominal ratio
-        peak_kind = "sustained dense bf16 x 1.1/2.25 (nominal tf32/bf16)"
-    elif mx:
-        peak_tf = pk["bf16_sustained"] * 4.5 / 2.25     # FP8 = bf16 x nominal ratio
-        peak_kind = "sustained dense bf16 x 4.5/2.25 (nominal fp8/bf16)"
+    peak_tf = tp["peak"]
     traffic = None
     tfile = os.path.join(ROOT, "profiles", "gemm_dram_traffic.json")
     if os.path.exists(tfile):
@@ -571,12 +631,18 @@ def main():
         if tr.get("source_sha256") == hashlib.sha256(src).hexdigest() and \
                 tr.get("workload") == w.name:
             traffic = tr.get("bytes_per_step")
-    roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": peak_tf,
+    roofline = {"bound": "tensor", "achieved": round(gemm_tflops, 1), "peak": round(peak_tf, 1),
                 "unit": "TFLOP/s", "frac": round(gemm_tflops / peak_tf, 4), "traffic": traffic,
+                "frac_burst": round(gemm_tflops / tp["burst"], 4),
+                "frac_sustained": round(gemm_tflops / tp["sustained"], 4),
+                "frac_nominal": round(gemm_tflops / tp["nominal"], 4),
+                "frac_is": tp["which"],
                 "kernel": "grouped GEMM, 6 launches per step (FC1+SwiGLU, FC2, FC2 dgrad+SwiGLU "
                           "bwd, FC2 wgrad, FC1 dgrad, FC1 wgrad), algorithmic 18*T*k*d*d_ff flops",
-                "peak_source": f"{pk['source']} {peak_kind} (MEASURED_PEAKS.json)"
-                if pk["source"] == "measured" else f"fallback 1.4 PFLOP/s, {peak_kind}"}
+                "peak_source": (f"{pk['source']} {tp['which']} {tp['kind']} (MEASURED_PEAKS.json; "
+                                f"{tp['why']}); nominal {tp['nominal']:.0f} TFLOP/s"
+                                if pk["source"] == "measured" else
+                                f"fallback {tp['which']} {tp['kind']} ({tp['why']})")}
     if mx:
         roofline["kernel"] += "; the GEMM stages include the MXFP8 quantisers of their operands"
     if layer is not None:

@@ -70,3 +70,24 @@ def test_traffic_figure_names_its_gemm_source():
     sha = tr["source_sha256"]
     assert len(sha) == 64 and all(c in "0123456789abcdef" for c in sha)
     assert tr["bytes_per_step"] > 0 and tr["workload"]
+
+
+def test_tensor_peak_burst_only_at_full_clock():
+    pk = dict(bf16=1652.2, bf16_sustained=1379.2, sm_max_mhz=1965.0, hbm=6548.2)
+    # a short run at the maximum clock: the burst figure (a matmul timed alone)
+    short = bench.tensor_peak(pk, "bf16", {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}, 0.06)
+    assert short["which"] == "burst" and short["peak"] == 1652.2
+    assert short["sustained"] == 1379.2 and short["nominal"] == 2250.0
+    # power-capped clocks, or a long timed region: the sustained figure
+    capped = bench.tensor_peak(pk, "bf16", {"sm_mhz": 1327.0, "sm_max_mhz": 1965.0}, 0.06)
+    assert capped["which"] == "sustained" and capped["peak"] == 1379.2
+    long = bench.tensor_peak(pk, "bf16", {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}, 30.0)
+    assert long["which"] == "sustained"
+    # no clock record: the sustained figure (the conservative one)
+    assert bench.tensor_peak(pk, "bf16", {"sm_mhz": None, "sm_max_mhz": None}, 0.06)["which"] \
+        == "sustained"
+    # other precisions scale by the nominal ratio to bf16
+    fp8 = bench.tensor_peak(pk, "fp8", {"sm_mhz": 1965.0, "sm_max_mhz": 1965.0}, 0.06)
+    assert abs(fp8["peak"] - 1652.2 * 2) < 1e-9 and fp8["nominal"] == 4500.0
+    tf32 = bench.tensor_peak(pk, "tf32", {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0}, 0.06)
+    assert abs(tf32["peak"] - 1379.2 * 1.1 / 2.25) < 1e-9
