@@ -19,11 +19,13 @@ constexpr int kRouteTokensPerCta = 256;
 inline int route_hist_rows(int T) { return (T + kRouteTokensPerHistRow - 1) / kRouteTokensPerHistRow; }
 inline int route_ctas(int T) { return (T + kRouteTokensPerCta - 1) / kRouteTokensPerCta; }
 
-// hist: route_hist_rows(T) x E int32; cta_base: route_ctas(T) x E int32 (scratch).
+// hist: route_hist_rows(T) x E int32; cta_base: route_ctas(T) x E int32 (scratch);
+// done_counter: one word that is zero before the launch (the routing leaves it zero), or
+// null to run the scan as a launch of its own.
 cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
                          int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
-                         float* row_gate, int32_t* hist, int32_t* cta_base, int* status,
-                         cudaStream_t s);
+                         float* row_gate, int32_t* hist, int32_t* cta_base,
+                         unsigned int* done_counter, int* status, cudaStream_t s);
 
 // C[M,N] (fp32 out, or act out) = A . B with arbitrary element strides; a plain
 // CUDA-core kernel for the small router projections.

@@ -26,6 +26,9 @@ int num_sms() {
 namespace {
 
 constexpr size_t kAlign = 256;
+// The workspace's first 256 bytes (zeroed by moe_workspace_init): the status word at 0,
+// the routing's CTA counter here (every routing launch leaves it zero again).
+constexpr size_t kRouteCounterOffset = 128;
 inline size_t up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline size_t act_bytes(const moe_desc& d) { return d.dtype == MOE_FP32 ? 4 : 2; }
@@ -244,7 +247,8 @@ moe_status route_body(const moe_desc& d, const float* logits, int32_t* idx, floa
     return cu(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (d.E + 1), s));
   }
   return cu(launch_route(d, logits, idx, gates, counts, offsets, slot, row_token, row_gate,
-                         at<int32_t>(ws, w.hist), at<int32_t>(ws, w.cta_base), status_ptr(ws), s));
+                         at<int32_t>(ws, w.hist), at<int32_t>(ws, w.cta_base),
+                         at<unsigned int>(ws, kRouteCounterOffset), status_ptr(ws), s));
 }
 
 moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_perm,

@@ -5,15 +5,17 @@
 // path's host round trip for the expert-group sizes, so the CPU can queue work
 // without waiting for a copy back (deniz.in, "Ai2, Olmo-core 3'ü Apache 2.0 ile
 // yayınladı", section "Yeni stack nasıl çalışıyor"; unite.ai, "पैरालेलिज़्म, प्रिसीजन,
-// और मेमोरी तकनीकें").  Three launches, no atomics on global memory, no host sync:
+// और मेमोरी तकनीकें").  Two launches (three above 256 experts), no host sync:
 //   1. topk:  one warp per token, logits in registers, k rounds of warp arg-max
 //             (ties to the lower expert index); gates = softmax over the kept
 //             logits; an expert histogram per 64 tokens (one CTA each, so even a
 //             few thousand tokens spread over every SM).
-//   2. scan:  one CTA: per expert, an exclusive scan of the histogram rows (each
-//             expert's column split over several threads), giving the base of every
-//             256-token slot CTA inside the expert, the counts, and offsets =
-//             exclusive scan of counts.
+//   2. scan:  the last top-k CTA to finish (a counter in global memory, the
+//             classic fence-then-count pattern: no CTA waits for another): per expert,
+//             an exclusive scan of the histogram rows (each expert's column split over
+//             several threads), giving the base of every 256-token slot CTA inside the
+//             expert, the counts, and offsets = exclusive scan of counts.  (Above 256
+//             experts, where top-k runs 8-warp CTAs, it is a separate one-CTA launch.)
 //   3. slots: per warp of 32 tokens, a bitmask per expert of the lanes that chose
 //             it; a token's rank inside the expert is the population count of the
 //             lower lanes' bits plus the bases of earlier warps and CTAs.  So the
@@ -39,18 +41,117 @@ __device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
   return va > vb || (va == vb && ia < ib);
 }
 
+// The scan, run by one CTA of 1024 threads.  Expert e's histogram column (nrows rows
+// of 64 tokens) is cut into J = 1024 / Ep chunks of consecutive rows (Ep = E rounded up
+// to 32), one thread each: a first pass sums the chunk (up to 32 rows held in
+// registers, so all of a chunk's loads are in flight at once), the chunk sums give each
+// thread its starting base, and a second pass writes the base at every 256-token slot
+// CTA's first row.  Then offsets = exclusive scan of the experts' totals.  capacity > 0:
+// the padded layout, offsets[e] = e * capacity instead.  The histogram is read with
+// L1-bypassing loads: other CTAs of the same launch may have written it.
+constexpr int kScanThreads = 1024;
+constexpr int kScanKeep = 32;
+__device__ __forceinline__ void scan_body(const int32_t* __restrict__ hist, int nrows, int E,
+                                          int capacity, int32_t* __restrict__ cta_base,
+                                          int32_t* __restrict__ counts,
+                                          int32_t* __restrict__ offsets, int* s_part) {
+  const int Ep = (E + 31) & ~31;                  // <= 1024
+  const int J = kScanThreads / Ep;                // chunks per expert
+  const int e = threadIdx.x % Ep, j = threadIdx.x / Ep;
+  const bool live = e < E && j < J;
+  const int per = (nrows + J - 1) / J;
+  const int r0 = min(nrows, j * per), r1 = min(nrows, r0 + per);
+  const bool keep = per <= kScanKeep;
+  int vals[kScanKeep];
+  int sum = 0;
+  if (live) {
+    if (keep) {
+#pragma unroll
+      for (int i = 0; i < kScanKeep; ++i) {
+        const int r = r0 + i;
+        vals[i] = r < r1 ? __ldcg(hist + (int64_t)r * E + e) : 0;
+        sum += vals[i];
+      }
+    } else {
+#pragma unroll 8
+      for (int r = r0; r < r1; ++r) sum += __ldcg(hist + (int64_t)r * E + e);
+    }
+  }
+  if (j < J) s_part[j * Ep + e] = sum;
+  __syncthreads();
+  int tot = 0;
+  if (live) {
+    int run = 0;
+    for (int jj = 0; jj < J; ++jj) {
+      const int v = s_part[jj * Ep + e];
+      if (jj < j) run += v;
+      tot += v;
+    }
+    if (keep) {
+#pragma unroll
+      for (int i = 0; i < kScanKeep; ++i) {
+        const int r = r0 + i;
+        if (r < r1 && r % kHistRowsPerCta == 0)
+          cta_base[(int64_t)(r / kHistRowsPerCta) * E + e] = run;
+        run += vals[i];
+      }
+    } else {
+#pragma unroll 8
+      for (int r = r0; r < r1; ++r) {
+        if (r % kHistRowsPerCta == 0) cta_base[(int64_t)(r / kHistRowsPerCta) * E + e] = run;
+        run += __ldcg(hist + (int64_t)r * E + e);
+      }
+    }
+    if (j == 0) counts[e] = tot;
+  }
+  __syncthreads();                                // every chunk sum read
+  // block-wide inclusive scan of the totals (thread i: expert i; Hillis-Steele)
+  if (j == 0 && e < Ep) s_part[e] = e < E ? tot : 0;
+  if (threadIdx.x >= Ep) s_part[threadIdx.x] = 0;
+  __syncthreads();
+  const int x = threadIdx.x;
+  const int own = s_part[x];
+  for (int o = 1; o < kScanThreads; o <<= 1) {
+    const int add = x >= o ? s_part[x - o] : 0;
+    __syncthreads();
+    s_part[x] += add;
+    __syncthreads();
+  }
+  if (x < E) offsets[x] = capacity > 0 ? x * capacity : s_part[x] - own;
+  if (x == kScanThreads - 1) offsets[E] = capacity > 0 ? E * capacity : s_part[kScanThreads - 1];
+}
+
+__global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t* __restrict__ hist,
+                                                            int nrows, int E, int capacity,
+                                                            int32_t* __restrict__ cta_base,
+                                                            int32_t* __restrict__ counts,
+                                                            int32_t* __restrict__ offsets) {
+  __shared__ int s_part[kScanThreads];
+  scan_body(hist, nrows, E, capacity, cta_base, counts, offsets, s_part);
+}
+
 // Top-k runs 32 warps per 64-token CTA (2 tokens a warp; the work of a token is a chain
 // of dependent shuffles, so many warps per SM hide it).  Above 256 experts a lane's
 // logits need more registers than 32 warps a CTA allow: 8 warps there.
 template <int NPL>
 constexpr int topk_warps() { return NPL <= 8 ? 32 : 8; }
 
+// Scan arguments for the top-k CTAs that finish last (fused: 32-warp CTAs, E <= 256).
+struct FusedScan {
+  unsigned int* done;      // CTAs finished so far (zero between launches; reset by the last)
+  int capacity;
+  int32_t* cta_base;
+  int32_t* counts;
+  int32_t* offsets;
+};
+
 template <int NPL>   // logits per lane = ceil(E / 32)
 __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const float* __restrict__ logits,
                                                            int T, int E, int k,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ gates,
-                                                           int32_t* __restrict__ hist) {
+                                                           int32_t* __restrict__ hist,
+                                                           FusedScan fs) {
   extern __shared__ int s_hist[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
@@ -113,63 +214,20 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
-}
-
-// One CTA of 1024 threads.  Expert e's histogram column (nrows rows of 64 tokens) is
-// cut into J = 1024 / Ep chunks of consecutive rows (Ep = E rounded up to 32), one
-// thread each: a first pass sums the chunk, the chunk sums give each thread its
-// starting base, and a second pass writes the base at every 256-token slot CTA's first
-// row.  Then offsets = exclusive scan of the experts' totals.  capacity > 0: the padded
-// layout, offsets[e] = e * capacity instead.
-__global__ void __launch_bounds__(1024) scan_kernel(const int32_t* __restrict__ hist, int nrows,
-                                                    int E, int capacity,
-                                                    int32_t* __restrict__ cta_base,
-                                                    int32_t* __restrict__ counts,
-                                                    int32_t* __restrict__ offsets) {
-  __shared__ int s_part[1024];
-  const int Ep = (E + 31) & ~31;                  // <= 1024
-  const int J = 1024 / Ep;                        // chunks per expert
-  const int e = threadIdx.x % Ep, j = threadIdx.x / Ep;
-  const bool live = e < E && j < J;
-  const int per = (nrows + J - 1) / J;
-  const int r0 = min(nrows, j * per), r1 = min(nrows, r0 + per);
-  int sum = 0;
-  if (live) {
-#pragma unroll 4
-    for (int r = r0; r < r1; ++r) sum += hist[(int64_t)r * E + e];
-  }
-  if (j < J) s_part[j * Ep + e] = sum;
-  __syncthreads();
-  int tot = 0;
-  if (live) {
-    int run = 0;
-    for (int jj = 0; jj < J; ++jj) {
-      const int v = s_part[jj * Ep + e];
-      if (jj < j) run += v;
-      tot += v;
-    }
-#pragma unroll 4
-    for (int r = r0; r < r1; ++r) {
-      if (r % kHistRowsPerCta == 0) cta_base[(int64_t)(r / kHistRowsPerCta) * E + e] = run;
-      run += hist[(int64_t)r * E + e];
-    }
-    if (j == 0) counts[e] = tot;
-  }
-  __syncthreads();                                // every chunk sum read
-  // block-wide inclusive scan of the totals (thread i: expert i; Hillis-Steele)
-  if (j == 0 && e < Ep) s_part[e] = e < E ? tot : 0;
-  if (threadIdx.x >= Ep) s_part[threadIdx.x] = 0;
-  __syncthreads();
-  const int x = threadIdx.x;
-  const int own = s_part[x];
-  for (int o = 1; o < 1024; o <<= 1) {
-    const int add = x >= o ? s_part[x - o] : 0;
+  if constexpr (topk_warps<NPL>() * 32 == kScanThreads) {
+    if (fs.done == nullptr) return;
+    // the last CTA to finish scans every CTA's histogram row
+    __shared__ int s_last;
+    __shared__ int s_part[kScanThreads];
+    __threadfence();                     // this CTA's row, visible before it is counted
     __syncthreads();
-    s_part[x] += add;
+    if (threadIdx.x == 0) s_last = atomicAdd(fs.done, 1u) == gridDim.x - 1;
     __syncthreads();
+    if (!s_last) return;
+    __threadfence();                     // every counted CTA's row is visible from here
+    scan_body(hist, gridDim.x, E, fs.capacity, fs.cta_base, fs.counts, fs.offsets, s_part);
+    if (threadIdx.x == 0) *fs.done = 0u;   // ready for the next launch
   }
-  if (x < E) offsets[x] = capacity > 0 ? x * capacity : s_part[x] - own;
-  if (x == 1023) offsets[E] = capacity > 0 ? E * capacity : s_part[1023];
 }
 
 __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
@@ -226,10 +284,10 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
 
 template <int NPL>
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gates,
-                        int32_t* hist, cudaStream_t s) {
+                        int32_t* hist, const FusedScan& fs, cudaStream_t s) {
   const int ctas = route_hist_rows(T);
   topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, E * sizeof(int), s>>>(logits, T, E, k, idx,
-                                                                        gates, hist);
+                                                                        gates, hist, fs);
   return cudaGetLastError();
 }
 
@@ -332,22 +390,28 @@ __global__ void __launch_bounds__(1024) load_stats_kernel(const int32_t* __restr
 
 cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_idx, float* gates,
                          int32_t* counts, int32_t* offsets, int32_t* slot, int32_t* row_token,
-                         float* row_gate, int32_t* hist, int32_t* cta_base, int* status,
-                         cudaStream_t s) {
+                         float* row_gate, int32_t* hist, int32_t* cta_base,
+                         unsigned int* done_counter, int* status, cudaStream_t s) {
   const int T = d.T, E = d.E, k = d.k;
   const int ctas = route_ctas(T);
   cudaError_t err;
   const int npl = (E + 31) / 32;
-  if (npl <= 1) err = launch_topk<1>(logits, T, E, k, topk_idx, gates, hist, s);
-  else if (npl <= 2) err = launch_topk<2>(logits, T, E, k, topk_idx, gates, hist, s);
-  else if (npl <= 4) err = launch_topk<4>(logits, T, E, k, topk_idx, gates, hist, s);
-  else if (npl <= 8) err = launch_topk<8>(logits, T, E, k, topk_idx, gates, hist, s);
-  else if (npl <= 16) err = launch_topk<16>(logits, T, E, k, topk_idx, gates, hist, s);
-  else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, s);
-  if (err != cudaSuccess) return err;
   const int C = d.capacity;
-  scan_kernel<<<1, 1024, 0, s>>>(hist, route_hist_rows(T), E, C, cta_base, counts, offsets);
-  if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  // up to 256 experts the last top-k CTA runs the scan (the CTAs have 1024 threads)
+  const bool fused = npl <= 8 && done_counter != nullptr;
+  FusedScan fs{fused ? done_counter : nullptr, C, cta_base, counts, offsets};
+  if (npl <= 1) err = launch_topk<1>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  else if (npl <= 2) err = launch_topk<2>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  else if (npl <= 4) err = launch_topk<4>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  else if (npl <= 8) err = launch_topk<8>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  else if (npl <= 16) err = launch_topk<16>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, fs, s);
+  if (err != cudaSuccess) return err;
+  if (!fused) {
+    scan_kernel<<<1, kScanThreads, 0, s>>>(hist, route_hist_rows(T), E, C, cta_base, counts,
+                                           offsets);
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+  }
   const size_t smem = size_t(2) * kWarps * E * sizeof(int);
   if (smem > 48 * 1024) {
     err = cudaFuncSetAttribute(slot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

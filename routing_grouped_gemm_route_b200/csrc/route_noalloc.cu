@@ -53,12 +53,12 @@ extern "C" moe_status moe_route_noalloc(const moe_desc* desc, const float* logit
   // The padded layout flags tokens beyond an expert's capacity in a status word, and
   // this call has none to report it through: refused rather than dropped silently.
   if (d.capacity > 0) return MOE_EUNSUPPORTED;
-  // scratch: histogram [ceil(T/64)][E] then slot-CTA bases [ceil(T/256)][E], int32 each,
-  // 256-byte aligned
+  // scratch: a 256-byte header (the routing's CTA counter), the histogram [ceil(T/64)][E],
+  // then the slot-CTA bases [ceil(T/256)][E], int32 each, 256-byte aligned
   const size_t hist_bytes = size_t(route_hist_rows(d.T)) * d.E * sizeof(int32_t);
   const size_t base_bytes = size_t(route_ctas(d.T)) * d.E * sizeof(int32_t);
   const size_t part_al = (hist_bytes + 255) / 256 * 256;
-  if (part_al + base_bytes > size_t(MOE_ROUTE_NOALLOC_SCRATCH_BYTES)) return MOE_EWORKSPACE;
+  if (256 + part_al + base_bytes > size_t(MOE_ROUTE_NOALLOC_SCRATCH_BYTES)) return MOE_EWORKSPACE;
   if (!counts || !offsets) return MOE_EINVAL;
   if (!aligned16(counts) || !aligned16(offsets)) return MOE_EALIGN;
   const void* tok[] = {logits, topk_idx, gates, slot, row_token, row_gate};
@@ -75,14 +75,17 @@ extern "C" moe_status moe_route_noalloc(const moe_desc* desc, const float* logit
   void* base = nullptr;
   st = scratch_address(&base);
   if (st != MOE_OK) return st;
-  // Both scratch arrays are written in full before they are read, so nothing has to
-  // be cleared between calls.  No status word: in the ragged layout routing writes
-  // only expert indices it selected itself (always in [0, E)) and slots inside its own
-  // counts, so the kernels have no error to flag.
-  int32_t* hist = reinterpret_cast<int32_t*>(base);
-  int32_t* cta_base = reinterpret_cast<int32_t*>(static_cast<char*>(base) + part_al);
+  // The histogram and the bases are written in full before they are read; the CTA
+  // counter must start at zero and is cleared here (every routing launch also leaves it
+  // zero).  No status word: in the ragged layout routing writes only expert indices it
+  // selected itself (always in [0, E)) and slots inside its own counts, so the kernels
+  // have no error to flag.
+  unsigned int* counter = static_cast<unsigned int*>(base);
+  int32_t* hist = reinterpret_cast<int32_t*>(static_cast<char*>(base) + 256);
+  int32_t* cta_base = reinterpret_cast<int32_t*>(static_cast<char*>(base) + 256 + part_al);
+  if (cudaMemsetAsync(counter, 0, sizeof(unsigned int), s) != cudaSuccess) return MOE_ECUDA;
   return launch_route(d, logits, topk_idx, gates, counts, offsets, slot, row_token, row_gate, hist,
-                      cta_base, nullptr, s) == cudaSuccess
+                      cta_base, counter, nullptr, s) == cudaSuccess
              ? MOE_OK
              : MOE_ECUDA;
 }
