@@ -36,9 +36,15 @@ static_assert(kWarps * 32 == kRouteTokensPerCta, "one token per lane in the slot
 constexpr int kHistRowsPerCta = kRouteTokensPerCta / kRouteTokensPerHistRow;
 static_assert(kHistRowsPerCta * kRouteTokensPerHistRow == kRouteTokensPerCta, "whole rows");
 
-// a beats b: larger logit, or equal logit and smaller index
-__device__ __forceinline__ bool better(float va, int ia, float vb, int ib) {
-  return va > vb || (va == vb && ia < ib);
+// Order-preserving 32-bit key of a logit: a > b as floats iff key(a) > key(b), with -0
+// taken as +0 (they compare equal as floats).  Every logit's key is above 0, the key of
+// "no candidate" (NaN is mapped to -inf before it gets here).
+__device__ __forceinline__ uint32_t logit_key(float f) {
+  const uint32_t b = __float_as_uint(f == 0.f ? 0.f : f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7fffffffu) : ~key);
 }
 
 // The scan, run by one CTA of 1024 threads.  Expert e's histogram column (nrows rows
@@ -130,11 +136,12 @@ __global__ void __launch_bounds__(kScanThreads) scan_kernel(const int32_t* __res
   scan_body(hist, nrows, E, capacity, cta_base, counts, offsets, s_part);
 }
 
-// Top-k runs 32 warps per 64-token CTA (2 tokens a warp; the work of a token is a chain
-// of dependent shuffles, so many warps per SM hide it).  Above 256 experts a lane's
-// logits need more registers than 32 warps a CTA allow: 8 warps there.
+// Top-k runs 32 warps per 64-token CTA (2 tokens a warp), two CTAs per SM.  Above 256
+// experts a lane's logits need more registers than that allows: 8 warps there.
 template <int NPL>
 constexpr int topk_warps() { return NPL <= 8 ? 32 : 8; }
+template <int NPL>
+constexpr int topk_ctas_per_sm() { return NPL <= 8 ? 2 : 1; }
 
 // Scan arguments for the top-k CTAs that finish last (fused: 32-warp CTAs, E <= 256).
 struct FusedScan {
@@ -145,14 +152,15 @@ struct FusedScan {
   int32_t* offsets;
 };
 
+// One warp per token.  Each round of the selection takes the largest remaining key of
+// every lane (its lowest index on ties), the warp's largest key by one reduction and the
+// lowest index holding it by a second: ties go to the lower expert index, as the
+// descending stable order of the logits has it.
 template <int NPL>   // logits per lane = ceil(E / 32)
-__global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const float* __restrict__ logits,
-                                                           int T, int E, int k,
-                                                           int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ gates,
-                                                           int32_t* __restrict__ hist,
-                                                           FusedScan fs) {
-  extern __shared__ int s_hist[];
+__global__ void __launch_bounds__(topk_warps<NPL>() * 32, topk_ctas_per_sm<NPL>())
+topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ topk_idx,
+            float* __restrict__ gates, int32_t* __restrict__ hist, FusedScan fs) {
+  extern __shared__ int s_hist[];          // [E] (fused: [max(E, kScanThreads)], then the scan's)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
@@ -162,49 +170,44 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
     const int t = t0 + i;
     if (t >= T) break;
     const float* row = logits + (int64_t)t * E;
-    float v[NPL];
+    uint32_t key[NPL];
 #pragma unroll
     for (int c = 0; c < NPL; ++c) {
       const int e = c * 32 + lane;
-      v[c] = e < E ? row[e] : -INFINITY;
+      float f = e < E ? row[e] : 0.f;
       // a NaN logit ranks as -inf (it would lose every comparison, and a row of them
       // would select no expert at all)
-      if (v[c] != v[c]) v[c] = -INFINITY;
+      if (f != f) f = -INFINITY;
+      key[c] = e < E ? logit_key(f) : 0u;
     }
-    unsigned taken = 0;           // bit c: v[c] already selected
-    float my_val = 0.f;
+    uint32_t my_key = 0u, top_key = 0u;
     int my_idx = 0;
-    float top = 0.f;
     for (int j = 0; j < k; ++j) {
-      // lane-local best among the not-yet-taken entries (index ascending on ties)
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
+      uint32_t bk = 0u;
+      int bc = 0;
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
-        const int e = c * 32 + lane;
-        if (e < E && !(taken & (1u << c)) && better(v[c], e, bv, bi)) {
-          bv = v[c];
-          bi = e;
+        if (key[c] > bk) {                 // strict: the lowest c wins a tie inside the lane
+          bk = key[c];
+          bc = c;
         }
       }
+      const uint32_t wmax = __reduce_max_sync(0xffffffffu, bk);
+      const uint32_t widx =
+          __reduce_min_sync(0xffffffffu, bk == wmax ? static_cast<uint32_t>(bc * 32 + lane) : ~0u);
+      if (static_cast<int>(widx & 31u) == lane) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (better(ov, oi, bv, bi)) {
-          bv = ov;
-          bi = oi;
-        }
+        for (int c = 0; c < NPL; ++c)
+          if (c == static_cast<int>(widx >> 5)) key[c] = 0u;   // taken
       }
-      if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-      if (j == 0) top = bv;
+      if (j == 0) top_key = wmax;
       if (lane == j) {
-        my_val = bv;
-        my_idx = bi;
+        my_key = wmax;
+        my_idx = static_cast<int>(widx);
       }
     }
     // gates: softmax over the kept logits, lane j holds entry j
-    const float z = lane < k ? expf(my_val - top) : 0.f;
+    const float z = lane < k ? expf(key_logit(my_key) - key_logit(top_key)) : 0.f;
     const float sum = warp_sum(z);
     if (lane < k) {
       topk_idx[(int64_t)t * k + lane] = my_idx;
@@ -218,14 +221,13 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32) topk_kernel(const floa
     if (fs.done == nullptr) return;
     // the last CTA to finish scans every CTA's histogram row
     __shared__ int s_last;
-    __shared__ int s_part[kScanThreads];
     __threadfence();                     // this CTA's row, visible before it is counted
-    __syncthreads();
+    __syncthreads();                     // (and every read of s_hist done)
     if (threadIdx.x == 0) s_last = atomicAdd(fs.done, 1u) == gridDim.x - 1;
     __syncthreads();
     if (!s_last) return;
     __threadfence();                     // every counted CTA's row is visible from here
-    scan_body(hist, gridDim.x, E, fs.capacity, fs.cta_base, fs.counts, fs.offsets, s_part);
+    scan_body(hist, gridDim.x, E, fs.capacity, fs.cta_base, fs.counts, fs.offsets, s_hist);
     if (threadIdx.x == 0) *fs.done = 0u;   // ready for the next launch
   }
 }
@@ -286,8 +288,10 @@ template <int NPL>
 cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, float* gates,
                         int32_t* hist, const FusedScan& fs, cudaStream_t s) {
   const int ctas = route_hist_rows(T);
-  topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, E * sizeof(int), s>>>(logits, T, E, k, idx,
-                                                                        gates, hist, fs);
+  // the fused scan reuses the histogram's shared memory (kScanThreads ints)
+  const int words = fs.done != nullptr && E < kScanThreads ? kScanThreads : E;
+  topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(logits, T, E, k, idx,
+                                                                            gates, hist, fs);
   return cudaGetLastError();
 }
 
