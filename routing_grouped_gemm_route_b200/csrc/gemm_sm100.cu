@@ -128,18 +128,20 @@ struct Cfg {
   // other), except for MXFP8 256-column tiles, where the scale columns leave room for one
   static constexpr int NACC = MX && BN == 256 ? 1 : 2;
   static constexpr int TMEM_COLS = MX ? 512 : 2 * BN;
-  // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there)
-  // and for single-accumulator tiles (the MMAs wait for the whole epilogue, so it is
-  // split over two warps per lane quadrant); elsewhere 4 warps keep up and leave more
-  // shared memory to the operand ring
-  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD || NACC == 1 ? 8 : 4;
+  // 8 epilogue warps for the math-heavy SwiGLU backward (4 leave the MMA waiting there),
+  // for single-accumulator tiles (the MMAs wait for the whole epilogue, so it is split
+  // over two warps per lane quadrant) and for the wgrads (~8 K-stages a tile leave the
+  // epilogue the bottleneck: with 4 warps the MMAs waited on it ~20% of the time);
+  // elsewhere 4 warps keep up and leave more shared memory to the operand ring
+  static constexpr int EPI_WARPS = EPI == EPI_SWIGLU_BWD || NACC == 1 || MODE == RAGGED_K ? 8 : 4;
   static constexpr int THREADS = 64 + 32 * EPI_WARPS;
   static constexpr int COLGRP = EPI_WARPS / 4;          // warps sharing one lane quadrant
   static constexpr int NCH = BN / 32;                   // 32-column chunks per tile
   static constexpr int WCH = NCH / COLGRP;              // chunks per epilogue warp
   // epilogue shared memory per warp: output staging chunks of 32 rows x 32 columns
   static constexpr int CH = 32 * 32 * sizeof(OutT);
-  static constexpr int NBUF = EPI == EPI_SWIGLU_FWD ? 3 : EPI == EPI_SWIGLU_BWD ? 0 : 2;
+  // (the wgrads' 8 warps take one staging chunk each, so the operand ring keeps 6 stages)
+  static constexpr int NBUF = EPI == EPI_SWIGLU_FWD ? 3 : EPI == EPI_SWIGLU_BWD ? 0 : MODE == RAGGED_K ? 1 : 2;
   // SwiGLU backward: slots of prefetched H1/H3 input chunks (32 x 32 each, in the
   // activation type: bf16 for the 16-bit and MXFP8 kernels); the dH1/dH3 results are
   // staged in place in the slot they were computed from
@@ -501,12 +503,25 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               fence_tmap_acquire(am);
               acquired_e = tl.e;
             }
+            if constexpr (!kMX) {
+              // one request per operand: the maps' third dimension steps through the
+              // 128-byte column blocks, so A's (and B's) blocks arrive as consecutive
+              // [KB rows x 128 B] slices, the layout of separate 2-D loads
+              if (PAIR) {
+                tma_load_3d_pair(sA, am, fb, 0, tl.row0 + k0, (tl.m0 + arow) / C::MNB);
+                tma_load_3d_pair(sB, &tmB, fb, 0, tl.row0 + k0, (tl.n0 + bcol) / C::MNB);
+              } else {
+                tma_load_3d(sA, am, &full[stage], 0, tl.row0 + k0, (tl.m0 + arow) / C::MNB);
+                tma_load_3d(sB, &tmB, &full[stage], 0, tl.row0 + k0, (tl.n0 + bcol) / C::MNB);
+              }
+            } else {
 #pragma unroll
-            for (int i = 0; i < BM / C::MNB; ++i)
-              load(sA + i * C::KB * 128, am, tl.m0 + arow + i * C::MNB, tl.row0 + k0);
+              for (int i = 0; i < BM / C::MNB; ++i)
+                load(sA + i * C::KB * 128, am, tl.m0 + arow + i * C::MNB, tl.row0 + k0);
 #pragma unroll
-            for (int i = 0; i < C::BNC / C::MNB; ++i)
-              load(sB + i * C::KB * 128, &tmB, tl.n0 + bcol + i * C::MNB, tl.row0 + k0);
+              for (int i = 0; i < C::BNC / C::MNB; ++i)
+                load(sB + i * C::KB * 128, &tmB, tl.n0 + bcol + i * C::MNB, tl.row0 + k0);
+            }
           }
           if (++stage == C::STAGES) { stage = 0; phase ^= 1u; }
         }
@@ -897,7 +912,7 @@ __global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
 #pragma unroll
   for (int j = 0; j < 8; ++j) dst[j] = src[j];
   const int rows = offsets ? offsets[e + 1] : R;   // no offsets: one segment of R rows
-  tmap_replace_outer_dim(maps + i, static_cast<uint32_t>(rows > 0 ? rows : 1));
+  tmap_replace_row_dim(maps + i, static_cast<uint32_t>(rows > 0 ? rows : 1));
   fence_tmap_release();
 }
 
@@ -965,6 +980,30 @@ static bool make_tmap(CUtensorMap* m, const void* base, int es_, uint64_t cols, 
                    CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// M/N-major operand [rows, cols] (bf16 or fp32, cols a multiple of 128 bytes) as a 3-D
+// map {128-byte column block, rows, blocks}: strides {cols * es, 128 B}, box {one block,
+// box_rows, nblk}.  One load brings nblk consecutive column blocks of box_rows rows,
+// each as its own [box_rows x 128 B] slice, swizzled like the 2-D M/N-major tiles.
+static bool make_tmap_mn3(CUtensorMap* m, const void* base, int es_, uint64_t cols,
+                          uint64_t rows, uint32_t box_rows, uint32_t nblk) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const uint64_t es = static_cast<uint64_t>(es_);
+  const uint64_t blk = 128 / es;                       // elements per column block
+  cuuint64_t dims[3] = {blk, rows, cols / blk};
+  cuuint64_t strides[2] = {cols * es, 128};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(blk), box_rows, nblk};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const bool fp32 = es == 4;
+  const CUtensorMapSwizzle swz =
+      fp32 ? CU_TENSOR_MAP_SWIZZLE_128B_ATOM_32B : CU_TENSOR_MAP_SWIZZLE_128B;
+  const CUtensorMapDataType dt =
+      fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+  return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
@@ -1105,8 +1144,14 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
   using C = Cfg<T, OutT, BN, EPI_STORE, PAIR, RAGGED_K>;
   constexpr int ES = sizeof(T);
   CUtensorMap ta, tb, to;
-  if (!make_tmap(&ta, G, ES, M, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
-  if (!make_tmap(&tb, X, ES, N, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if constexpr (C::MX) {
+    if (!make_tmap(&ta, G, ES, M, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+    if (!make_tmap(&tb, X, ES, N, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  } else {
+    // 16-bit / fp32: one 3-D request per operand and stage (the kernel's wgrad loads)
+    if (!make_tmap_mn3(&ta, G, ES, M, g.R, C::KB, BM / C::MNB)) return MOE_ECUDA;
+    if (!make_tmap_mn3(&tb, X, ES, N, g.R, C::KB, C::BNC / C::MNB)) return MOE_ECUDA;
+  }
   if (!make_tmap(&to, dW, (int)sizeof(OutT), N, (uint64_t)g.E * M, 32, 32, Box::Chunk))
     return MOE_ECUDA;
   Params p{};
@@ -1224,9 +1269,16 @@ static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, cons
   using C = Cfg<T, T, 128, EPI_STORE>;
   constexpr int ES = sizeof(T);
   CUtensorMap t0, t1;
-  if (!make_tmap(&t0, dy_perm, ES, g.d, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
-  if (!make_tmap(&t1, dH13, ES, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
-    return MOE_ECUDA;
+  if constexpr (C::MX) {
+    if (!make_tmap(&t0, dy_perm, ES, g.d, g.R, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+    if (!make_tmap(&t1, dH13, ES, 2 * (uint64_t)g.f, g.R, C::MNB, C::KB, Box::MNMajor))
+      return MOE_ECUDA;
+  } else {
+    // the 3-D maps of the kernel's A loads (BM columns, i.e. BM / MNB blocks, a request)
+    if (!make_tmap_mn3(&t0, dy_perm, ES, g.d, g.R, C::KB, BM / C::MNB)) return MOE_ECUDA;
+    if (!make_tmap_mn3(&t1, dH13, ES, 2 * (uint64_t)g.f, g.R, C::KB, BM / C::MNB))
+      return MOE_ECUDA;
+  }
   const int threads = 2 * g.E;
   expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, g.R, maps);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
@@ -1424,7 +1476,7 @@ static moe_status router_dwr_tc(int T, int d, int E, const void* x, const void* 
   // dWr[d,E] = x^T . d_logits: a ragged-K GEMM over the one segment (K = T)
   using C = Cfg<bf16, bf16, 128, EPI_STORE>;
   CUtensorMap t0;
-  if (!make_tmap(&t0, x, 2, d, T, C::MNB, C::KB, Box::MNMajor)) return MOE_ECUDA;
+  if (!make_tmap_mn3(&t0, x, 2, d, T, C::KB, BM / C::MNB)) return MOE_ECUDA;
   expert_maps_kernel<<<1, 128, 0, s>>>(t0, t0, nullptr, 1, T, maps);
   if (cudaGetLastError() != cudaSuccess) return MOE_ECUDA;
   const int bn = bn_of(E);

@@ -164,13 +164,35 @@ __device__ __forceinline__ void tma_load_2d_pair(void* smem_dst, const void* tma
       "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
+// 3-D forms: coordinates (x, y, z) of a map whose third dimension steps through
+// 128-byte column blocks of a row-major matrix (see make_tmap_mn3 on the host), so one
+// request brings several M/N-major 128-byte blocks, each landing as its own
+// [rows x 128 B] slice of shared memory.
+__device__ __forceinline__ void tma_load_3d(void* smem_dst, const void* tmap, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d_pair(void* smem_dst, const void* tmap,
+                                                 uint32_t bar_cluster, int32_t x, int32_t y,
+                                                 int32_t z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(tmap)), "r"(bar_cluster), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
 __device__ __forceinline__ void tma_prefetch_desc(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
 }
 // Per-expert tensor maps live in global memory: they are written by a kernel (copy of
 // a host-encoded template, then tensormap.replace of one field) and read by the TMA
-// unit in a later kernel.
-__device__ __forceinline__ void tmap_replace_outer_dim(void* gmem_map, uint32_t rows) {
+// unit in a later kernel.  Replaces the extent of dimension 1, the rows, in the 2-D
+// maps and in the 3-D column-block maps alike.
+__device__ __forceinline__ void tmap_replace_row_dim(void* gmem_map, uint32_t rows) {
   asm volatile("tensormap.replace.tile.global_dim.global.b1024.b32 [%0], 1, %1;" ::"l"(
                    reinterpret_cast<uint64_t>(gmem_map)),
                "r"(rows)
