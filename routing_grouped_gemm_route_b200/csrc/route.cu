@@ -232,15 +232,89 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
   }
 }
 
+// Slots of one 256-token CTA.  NPL = 0: the expert bases of the CTA come from the scan
+// (cta_base, offsets).  NPL > 0 (E <= 32 * NPL <= 256, at most kSlotScanRows histogram
+// rows): the CTA sums the histogram rows itself -- its warps stride over the rows, lane L
+// holds experts L + 32c -- into the rows before it (its base in each expert) and all rows
+// (the counts), then scans the counts into offsets; CTA 0 writes counts and offsets.  No
+// CTA waits for another and no separate scan runs: every CTA reads the histogram
+// (nrows x E int32, 128 KB at 16384 tokens and 128 experts) from L2.
+constexpr int kSlotScanRows = 512;
+template <int NPL>
 __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
     const int32_t* __restrict__ topk_idx, const float* __restrict__ gates,
-    const int32_t* __restrict__ offsets, const int32_t* __restrict__ cta_base, int T, int E,
+    int32_t* __restrict__ offsets, const int32_t* __restrict__ cta_base,
+    const int32_t* __restrict__ hist, int nrows, int32_t* __restrict__ counts, int T, int E,
     int k, int capacity, int32_t* __restrict__ slot, int32_t* __restrict__ row_token,
     float* __restrict__ row_gate, int* status) {
   extern __shared__ unsigned s_mem[];
   unsigned* masks = s_mem;                                          // [kWarps][E]
   int* wbase = reinterpret_cast<int*>(s_mem + kWarps * E);          // [kWarps][E]
+  int* s_off = wbase + kWarps * E;                                  // [E] (NPL > 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int start = 0;                     // thread e: the CTA's first row in expert e
+  if constexpr (NPL > 0) {
+    // per-warp sums of the rows before this CTA and of all rows, into masks / wbase
+    const int r_cta = blockIdx.x * kHistRowsPerCta;
+    int pre[NPL], tot[NPL];
+#pragma unroll
+    for (int c = 0; c < NPL; ++c) pre[c] = tot[c] = 0;
+#pragma unroll 4
+    for (int r = warp; r < nrows; r += kWarps) {
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        const int e = c * 32 + lane;
+        const int v = e < E ? hist[(int64_t)r * E + e] : 0;
+        tot[c] += v;
+        if (r < r_cta) pre[c] += v;
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < NPL; ++c) {
+      const int e = c * 32 + lane;
+      if (e < E) {
+        reinterpret_cast<int*>(masks)[warp * E + e] = pre[c];
+        wbase[warp * E + e] = tot[c];
+      }
+    }
+    __syncthreads();
+    // thread e: base and count of expert e; offsets = exclusive scan of the counts
+    const int e = threadIdx.x;                 // E <= 256 = blockDim.x
+    int base = 0, cnt = 0;
+    if (e < E) {
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        base += reinterpret_cast<int*>(masks)[w * E + e];
+        cnt += wbase[w * E + e];
+      }
+    }
+    int incl = cnt;                            // warp-inclusive scan, then across warps
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += v;
+    }
+    __shared__ int s_warp[kWarps];
+    __syncthreads();                           // masks / wbase reads done
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      before += w < warp ? s_warp[w] : 0;
+      total += s_warp[w];
+    }
+    const int off = capacity > 0 ? e * capacity : before + incl - cnt;
+    if (e < E) {
+      s_off[e] = off;
+      start = off + base;
+      if (blockIdx.x == 0) {
+        counts[e] = cnt;
+        offsets[e] = off;
+      }
+    }
+    if (blockIdx.x == 0 && e == 0) offsets[E] = capacity > 0 ? E * capacity : total;
+  }
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
   __syncthreads();
   const int t = blockIdx.x * kRouteTokensPerCta + threadIdx.x;
@@ -253,7 +327,7 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = offsets[e] + cta_base[(int64_t)blockIdx.x * E + e];
+    int run = NPL > 0 ? start : offsets[e] + cta_base[(int64_t)blockIdx.x * E + e];
 #pragma unroll
     for (int w = 0; w < kWarps; ++w) {
       wbase[w * E + e] = run;
@@ -271,7 +345,8 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
         continue;
       }
       const int s = wbase[warp * E + e] + __popc(masks[warp * E + e] & lower);
-      if (capacity > 0 && s - offsets[e] >= capacity) {
+      const int off_e = NPL > 0 ? s_off[e] : offsets[e];
+      if (capacity > 0 && s - off_e >= capacity) {
         // padded layout: the expert's rows are full (the capacity is below its count)
         set_status(status, MOE_DEV_BAD_INDEX);
         slot[(int64_t)t * k + j] = -1;
@@ -401,8 +476,12 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   cudaError_t err;
   const int npl = (E + 31) / 32;
   const int C = d.capacity;
-  // up to 256 experts the last top-k CTA runs the scan (the CTAs have 1024 threads)
-  const bool fused = npl <= 8 && done_counter != nullptr;
+  const int nrows = route_hist_rows(T);
+  // up to 256 experts and kSlotScanRows histogram rows the slot CTAs sum the histogram
+  // themselves; else, up to 256 experts, the last top-k CTA runs the scan (the CTAs have
+  // 1024 threads); above that a one-CTA scan launch
+  const bool in_slot = npl <= 8 && nrows <= kSlotScanRows;
+  const bool fused = !in_slot && npl <= 8 && done_counter != nullptr;
   FusedScan fs{fused ? done_counter : nullptr, C, cta_base, counts, offsets};
   if (npl <= 1) err = launch_topk<1>(logits, T, E, k, topk_idx, gates, hist, fs, s);
   else if (npl <= 2) err = launch_topk<2>(logits, T, E, k, topk_idx, gates, hist, fs, s);
@@ -411,14 +490,13 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   else if (npl <= 16) err = launch_topk<16>(logits, T, E, k, topk_idx, gates, hist, fs, s);
   else err = launch_topk<32>(logits, T, E, k, topk_idx, gates, hist, fs, s);
   if (err != cudaSuccess) return err;
-  if (!fused) {
-    scan_kernel<<<1, kScanThreads, 0, s>>>(hist, route_hist_rows(T), E, C, cta_base, counts,
-                                           offsets);
+  if (!fused && !in_slot) {
+    scan_kernel<<<1, kScanThreads, 0, s>>>(hist, nrows, E, C, cta_base, counts, offsets);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const size_t smem = size_t(2) * kWarps * E * sizeof(int);
+  const size_t smem = (size_t(2) * kWarps * E + (in_slot ? E : 0)) * sizeof(int);
   if (smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(slot_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    err = cudaFuncSetAttribute(slot_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                static_cast<int>(smem));
     if (err != cudaSuccess) return err;
   }
@@ -428,8 +506,16 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
     if ((err = cudaMemsetAsync(row_token, 0xff, rows * 4, s)) != cudaSuccess) return err;
     if ((err = cudaMemsetAsync(row_gate, 0, rows * 4, s)) != cudaSuccess) return err;
   }
-  slot_kernel<<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, T, E, k, C, slot,
-                                              row_token, row_gate, status);
+#define MOE_SLOT(NP)                                                                            \
+  slot_kernel<NP><<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, hist, nrows, \
+                                                  counts, T, E, k, C, slot, row_token, row_gate,  \
+                                                  status)
+  if (!in_slot) MOE_SLOT(0);
+  else if (npl <= 1) MOE_SLOT(1);
+  else if (npl <= 2) MOE_SLOT(2);
+  else if (npl <= 4) MOE_SLOT(4);
+  else MOE_SLOT(8);
+#undef MOE_SLOT
   return cudaGetLastError();
 }
 
