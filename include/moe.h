@@ -60,7 +60,13 @@ typedef enum moe_status {
 } moe_status;
 
 typedef enum moe_dtype {
-  MOE_FP32 = 0,   /* fp32 storage, TF32 tensor-core GEMMs with fp32 accumulation */
+  MOE_FP32 = 0,   /* fp32 storage, TF32 tensor-core GEMMs with fp32 accumulation.  The
+                     GEMM operands are rounded to the nearest TF32 value (ties away from
+                     zero) where they are produced: x_perm (moe_dispatch), a (FC1's
+                     epilogue), dy_perm (moe_combine_bwd) and dH13 (FC2 dgrad's epilogue)
+                     are stored rounded, and the GEMM calls read workspace copies of
+                     W13 / W2 rounded the same way -- instead of the tensor core dropping
+                     the low 13 mantissa bits (a bias towards zero) */
   MOE_BF16 = 1,   /* bf16 storage, bf16 tensor-core GEMMs with fp32 accumulation */
   MOE_MXFP8 = 2   /* bf16 storage; the grouped GEMMs quantise their operands to E4M3 with
                      an E8M0 scale per 32 along K (moe_mx_quantize) and run block-scaled

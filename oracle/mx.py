@@ -49,6 +49,24 @@ def bf16_round(v) -> np.ndarray:
     return np.where(big, np.copysign(np.inf, v), r)
 
 
+def tf32_round(v) -> np.ndarray:
+    """fp32 values rounded to the nearest TF32 value, ties away from zero (fp32 result).
+
+    TF32 keeps fp32's sign and 8 exponent bits and 10 of its 23 mantissa bits: the value
+    is the fp32 bit pattern with the low 13 bits cleared after adding half of their
+    range to the magnitude.  This is the precision the fp32 layer's tensor-core GEMMs
+    read their operands in; the layer rounds each operand once where it is produced.
+    """
+    a = np.asarray(v, dtype=np.float32)
+    bits = a.view(np.uint32)
+    mag = bits & np.uint32(0x7FFFFFFF)
+    sign = bits & np.uint32(0x80000000)
+    finite = mag < np.uint32(0x7F800000)
+    rounded = (mag + np.uint32(0x1000)) & np.uint32(0xFFFFE000)
+    out = np.where(finite, sign | rounded, bits).astype(np.uint32)
+    return out.view(np.float32)
+
+
 def _floor_log2(a: np.ndarray) -> np.ndarray:
     """floor(log2(a)) for a > 0, exact (from the binary exponent)."""
     _, ex = np.frexp(a)

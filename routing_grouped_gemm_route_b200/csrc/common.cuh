@@ -60,6 +60,24 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// fp32 value rounded to the nearest TF32 value (10 explicit mantissa bits, ties away from
+// zero; the low 13 bits come out zero).  GEMM operands of the fp32 dtype are rounded
+// where they are produced, so the tensor core (which reads fp32 operands as TF32 by
+// dropping those bits) sees values it represents exactly, instead of truncating them
+// towards zero.
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
+// The same for the four floats of a 16-byte vector.
+__device__ __forceinline__ uint4 tf32_round4(uint4 v) {
+  return make_uint4(__float_as_uint(tf32_round(__uint_as_float(v.x))),
+                    __float_as_uint(tf32_round(__uint_as_float(v.y))),
+                    __float_as_uint(tf32_round(__uint_as_float(v.z))),
+                    __float_as_uint(tf32_round(__uint_as_float(v.w))));
+}
+
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);

@@ -778,6 +778,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               bits_to_f32(v3, h3);
 #pragma unroll
               for (int i = 0; i < 32; ++i) av[i] = fv[i] * sigmoid_f(fv[i]) * h3[i];
+              if constexpr (kTF32) {
+                // a feeds TF32 GEMMs only (FC2, FC2 wgrad): stored rounded to TF32
+#pragma unroll
+                for (int i = 0; i < 32; ++i) av[i] = tf32_round(av[i]);
+              }
               if (whole) {
                 staged_store<OutT, C::NBUF>(stage_buf + 0 * C::CH, fv, lane, &tmO, h0 + c, rbase,
                                             false);
@@ -814,6 +819,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                 const float da = fv[j];
                 d3[j] = da * h1[j] * sg;
                 fv[j] = da * h3[j] * sg * (1.0f + h1[j] * (1.0f - sg));
+                if constexpr (kTF32) {
+                  // dH13 feeds TF32 GEMMs only (FC1 dgrad, FC1 wgrad): rounded to TF32
+                  d3[j] = tf32_round(d3[j]);
+                  fv[j] = tf32_round(fv[j]);
+                }
               }
               if (whole) {
                 // each lane rewrites only the row it read, so no barrier is needed first

@@ -116,6 +116,8 @@ moe_status router_logits_tc(int T, int d, int E, const void* x, const void* Wr, 
 moe_status router_bwd_tc(int T, int d, int E, const void* x, const void* Wr, const void* dl16,
                          float* dx_extra, void* dWr, void* maps_ws, int* status, cudaStream_t s);
 cudaError_t launch_f32_to_bf16(int64_t n, const float* src, void* dst, cudaStream_t s);
+// dst[i] = src[i] rounded to TF32 (n a multiple of 4)
+cudaError_t launch_tf32_round(int64_t n, const float* src, float* dst, cudaStream_t s);
 
 // Shared expert (a dense SwiGLU FFN over all g.R = T rows, one segment): forward writes
 // H13s, as (act) and ys [T,d] (float); backward writes dH13s (act scratch), dxs [T,d]

@@ -46,6 +46,7 @@ struct WsLayout {
   size_t dl16;                                  // bf16 copy of d_logits (router, bf16)
   size_t sh_f32, sh_dH13, rc_sh_H13, rc_sh_a;   // shared expert: y / dx (float), dH13, recompute
   size_t mx_ints, mx_bytes[24];   // MXFP8 operands (codes and scale chunks), see MxWork
+  size_t w13_t, w2_t, x_t, dy_t;  // fp32: TF32-rounded weights (and shared expert's x, dy)
   size_t total;
 };
 
@@ -77,6 +78,14 @@ WsLayout ws_layout(const moe_desc& d) {
   w.rc_H13 = o; if (rc) o = up(o + R * 2 * (size_t)d.d_ff * es);
   w.rc_a = o; if (rc) o = up(o + R * (size_t)d.d_ff * es);
   w.rc_y_perm = o; if (rc) o = up(o + R * d.d * es);
+  w.w13_t = o; w.w2_t = o; w.x_t = o; w.dy_t = o;
+  if (d.dtype == MOE_FP32) {
+    const size_t nw = (size_t)d.E + (sh ? 1 : 0);
+    w.w13_t = o; o = up(o + nw * 2 * (size_t)d.d_ff * d.d * 4);
+    w.w2_t = o; o = up(o + nw * (size_t)d.d * d.d_ff * 4);
+    w.x_t = o; if (sh) o = up(o + T * d.d * 4);
+    w.dy_t = o; if (sh) o = up(o + T * d.d * 4);
+  }
   w.mx_ints = o;
   if (d.dtype == MOE_MXFP8) {
     const size_t E = d.E, f = d.d_ff, dm = d.d;
@@ -219,6 +228,37 @@ GemmShape gshape(const moe_desc& d, int rows = -1) {
   return g;
 }
 
+// fp32: the TF32 GEMMs read W13 / W2 rounded to TF32 (workspace copies made here; the
+// tensor core would otherwise truncate them); other dtypes read them as they are.
+struct Weights {
+  const void* W13;
+  const void* W2;
+};
+moe_status tf32_weights(const moe_desc& d, const void* W13, const void* W2, void* ws,
+                        cudaStream_t s, Weights* out) {
+  out->W13 = W13;
+  out->W2 = W2;
+  if (d.dtype != MOE_FP32) return MOE_OK;
+  const WsLayout w = ws_layout(d);
+  const int64_t nw = (int64_t)d.E + ((d.flags & MOE_FLAG_SHARED_EXPERT) ? 1 : 0);
+  float* w13 = at<float>(ws, w.w13_t);
+  float* w2 = at<float>(ws, w.w2_t);
+  MOE_TRY(cu(launch_tf32_round(nw * 2 * d.d_ff * d.d, static_cast<const float*>(W13), w13, s)));
+  MOE_TRY(cu(launch_tf32_round(nw * d.d * d.d_ff, static_cast<const float*>(W2), w2, s)));
+  out->W13 = w13;
+  out->W2 = w2;
+  return MOE_OK;
+}
+// fp32 with the shared expert: its GEMMs read x (and dy) directly, rounded here
+const void* tf32_tokens(const moe_desc& d, const void* src, size_t off, void* ws, cudaStream_t s,
+                        moe_status* st) {
+  *st = MOE_OK;
+  if (d.dtype != MOE_FP32 || d.T == 0) return src;
+  float* dst = at<float>(ws, off);
+  *st = cu(launch_tf32_round((int64_t)d.T * d.d, static_cast<const float*>(src), dst, s));
+  return dst;
+}
+
 // ---------------------------------------------------------------------------- bodies
 // Permutation steps with the layout's row bound; the padded layout first clears the
 // expert buffers its rows scatter into (padding rows must be zero for the weight
@@ -264,8 +304,10 @@ moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_p
     return cu(cudaMemsetAsync(dW2, 0, (size_t)d.E * d.d * d.d_ff * es, s));
   }
   MxWork mx = mx_work(d, ws);
-  return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, W13, W2, offsets, dH13, dx_perm, dW13, dW2,
-                  fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s, &mx);
+  Weights wt;
+  MOE_TRY(tf32_weights(d, W13, W2, ws, s, &wt));
+  return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, wt.W13, wt.W2, offsets, dH13, dx_perm, dW13,
+                  dW2, fp32_dw, acc, at<char>(ws, ws_layout(d).maps), status_ptr(ws), s, &mx);
 }
 
 // bf16 router GEMMs run on the tensor cores when E is a multiple of 64; fp32 (and other
@@ -406,7 +448,9 @@ moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const 
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   if (R_of(*desc) == 0) return MOE_OK;
   MxWork mx = mx_work(*desc, ws);
-  return gemm_fwd(gshape(*desc), x_perm, W13, W2, offsets, H13, a, y_perm, status_ptr(ws),
+  Weights wt;
+  MOE_TRY(tf32_weights(*desc, W13, W2, ws, S(stream), &wt));
+  return gemm_fwd(gshape(*desc), x_perm, wt.W13, wt.W2, offsets, H13, a, y_perm, status_ptr(ws),
                   S(stream), &mx);
 }
 
@@ -570,14 +614,19 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   const Acts A = acts(d, saved, L, ws);
   MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
   MxWork mx = mx_work(d, ws);
-  MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+  Weights wt;
+  MOE_TRY(tf32_weights(d, W13, W2, ws, s, &wt));
+  MOE_TRY(gemm_fwd(gshape(d), A.x_perm, wt.W13, wt.W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
   float* ys = nullptr;
   if (d.flags & MOE_FLAG_SHARED_EXPERT) {
     // the shared expert over every token, its output in fp32 for the combine to add
     const size_t es = act_bytes(d);
     ys = at<float>(ws, ws_layout(d).sh_f32);
-    MOE_TRY(shared_fwd(gshape(d, d.T), x, w13_slice(d, W13, es), w2_slice(d, W2, es), A.H13s, A.as,
-                       ys, st, s));
+    moe_status r;
+    const void* xs = tf32_tokens(d, x, ws_layout(d).x_t, ws, s, &r);
+    MOE_TRY(r);
+    MOE_TRY(shared_fwd(gshape(d, d.T), xs, w13_slice(d, wt.W13, es), w2_slice(d, wt.W2, es), A.H13s,
+                       A.as, ys, st, s));
   }
   return cu(launch_gather_sum(f32, d.T, d.d, d.k, (int)R_of(d), A.y_perm, gates, slot, ys, y, st,
                               s));
@@ -613,15 +662,28 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
   void* dH13 = at<char>(ws, w.dH13);
   void* dx_perm = at<char>(ws, w.dx_perm);
   const Acts A = acts(d, saved, L, ws);
+  // (the backward GEMMs round the weights themselves; the recomputed forward and the
+  // shared expert read this copy)
+  Weights wt{W13, W2};
+  if (recompute || shared) MOE_TRY(tf32_weights(d, W13, W2, ws, s, &wt));
+  const void* xs = x;                     // the shared expert's x and dy (fp32: TF32-rounded)
+  const void* dys = dy;
+  if (shared) {
+    moe_status r;
+    xs = tf32_tokens(d, x, w.x_t, ws, s, &r);
+    MOE_TRY(r);
+    dys = tf32_tokens(d, dy, w.dy_t, ws, s, &r);
+    MOE_TRY(r);
+  }
   if (recompute && d.T > 0) {
     // the forward's activations again, from x and the saved routing (same kernels,
     // same inputs: bit-identical to the ones the forward used)
     MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
     MxWork mx = mx_work(d, ws);
-    MOE_TRY(gemm_fwd(gshape(d), A.x_perm, W13, W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+    MOE_TRY(gemm_fwd(gshape(d), A.x_perm, wt.W13, wt.W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
     if (shared)
-      MOE_TRY(shared_fwd(gshape(d, d.T), x, w13_slice(d, W13, es), w2_slice(d, W2, es), A.H13s,
-                         A.as, at<float>(ws, w.sh_f32), st, s));
+      MOE_TRY(shared_fwd(gshape(d, d.T), xs, w13_slice(d, wt.W13, es), w2_slice(d, wt.W2, es),
+                         A.H13s, A.as, at<float>(ws, w.sh_f32), st, s));
   }
 
   MOE_TRY(combine_bwd_body(d, dy, A.y_perm, gates, idx, slot, dy_perm, d_logits, st, s));
@@ -632,8 +694,8 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
     // the shared expert's backward: dy is its (unpermuted, ungated) output gradient
     const size_t dw_es = (d.flags & MOE_FLAG_DW_FP32) ? 4 : es;
     dxs = at<float>(ws, w.sh_f32);
-    MOE_TRY(shared_bwd(gshape(d, d.T), dy, x, A.H13s, A.as, w13_slice(d, W13, es),
-                       w2_slice(d, W2, es), at<char>(ws, w.sh_dH13), dxs,
+    MOE_TRY(shared_bwd(gshape(d, d.T), dys, xs, A.H13s, A.as, w13_slice(d, wt.W13, es),
+                       w2_slice(d, wt.W2, es), at<char>(ws, w.sh_dH13), dxs,
                        const_cast<void*>(w13_slice(d, dW13, dw_es)),
                        const_cast<void*>(w2_slice(d, dW2, dw_es)), d.flags & MOE_FLAG_DW_FP32,
                        d.flags & MOE_FLAG_ACCUM_DW, at<char>(ws, w.maps), st, s));

@@ -55,6 +55,8 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(const T* __restri
     for (int u = 0; u < U; ++u) {
       const int v = base + u * 32 + lane;
       if (v < nvec) buf[u] = ld_stream16(src + (int64_t)v * V);
+      // fp32: x_perm feeds TF32 GEMMs only (FC1, FC1 wgrad): rounded to TF32 here
+      if constexpr (sizeof(T) == 4) buf[u] = tf32_round4(buf[u]);
     }
     for (int j = 0; j < k; ++j) {
       const int s = bcast(my, j);
@@ -184,6 +186,8 @@ __global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
         for (int i = 0; i < V; ++i) {
           dot[j] = fmaf(fdy[i], fy[i], dot[j]);
           o[i] = g[j] * fdy[i];
+          // fp32: dy_perm feeds TF32 GEMMs only (FC2 dgrad, FC2 wgrad): rounded to TF32
+          if constexpr (sizeof(T) == 4) o[i] = tf32_round(o[i]);
         }
         Vec16<T> pk;
         pk.from_float(o);
@@ -234,6 +238,25 @@ cudaError_t launch_add_f32(bool fp32, int64_t n, void* y, const float* extra, cu
   const int blocks = 4 * num_sms();
   if (fp32) add_f32_kernel<float><<<blocks, 256, 0, s>>>((float*)y, extra, n);
   else add_f32_kernel<__nv_bfloat16><<<blocks, 256, 0, s>>>((__nv_bfloat16*)y, extra, n);
+  return cudaGetLastError();
+}
+
+// dst = src rounded to TF32 (tf32_round), n a multiple of 4: the fp32 weights (and the
+// shared expert's x and dy) before the TF32 GEMMs read them.
+__global__ void tf32_round_kernel(const float* __restrict__ src, float* __restrict__ dst,
+                                  int64_t n) {
+  const int64_t nv = n / 4;
+  for (int64_t v = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; v < nv;
+       v += (int64_t)gridDim.x * blockDim.x)
+    reinterpret_cast<uint4*>(dst)[v] = tf32_round4(reinterpret_cast<const uint4*>(src)[v]);
+}
+
+cudaError_t launch_tf32_round(int64_t n, const float* src, float* dst, cudaStream_t s) {
+  if (n == 0) return cudaSuccess;
+  if (n % 4 != 0) return cudaErrorInvalidValue;
+  const int64_t nv = n / 4;
+  const int blocks = (int)std::min<int64_t>((nv + 255) / 256, (int64_t)num_sms() * 8);
+  tf32_round_kernel<<<blocks, 256, 0, s>>>(src, dst, n);
   return cudaGetLastError();
 }
 

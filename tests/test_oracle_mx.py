@@ -144,3 +144,35 @@ def test_mx_operand_of_layer_oracle_is_bf16_rounded():
     a = g.standard_normal((64, 128))
     assert np.array_equal(_mx(a, 1, True), mx.mx_quantize_dequantize(oracle.bf16_round(a), axis=1))
     assert _mx(a, 1, False) is a
+
+
+def test_tf32_round_hand_values():
+    # TF32 keeps 10 mantissa bits: the spacing at 1 is 2**-10, ties go away from zero
+    # subnormals keep 10 bits too: 2**-136 is the smallest TF32 step, 2**-137 a tie that
+    # goes to it, 2**-140 below half of it goes to 0
+    x = np.array([1 + 2.0 ** -11, 1 + 2.0 ** -12, 1 + 3 * 2.0 ** -11, -(1 + 2.0 ** -11),
+                  1 + 2.0 ** -10, 3.0, 2.0 ** -136, 2.0 ** -137, 2.0 ** -140, 0.0, -0.0],
+                 dtype=np.float32)
+    want = np.array([1 + 2.0 ** -10, 1.0, 1 + 2.0 ** -9, -(1 + 2.0 ** -10),
+                     1 + 2.0 ** -10, 3.0, 2.0 ** -136, 2.0 ** -136, 0.0, 0.0, -0.0],
+                    dtype=np.float32)
+    got = oracle.tf32_round(x)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+def test_tf32_round_properties():
+    rng = np.random.default_rng(3)
+    x = (rng.standard_normal(100000) * 10.0 ** rng.integers(-8, 8, 100000)).astype(np.float32)
+    r = oracle.tf32_round(x)
+    assert np.all((r.view(np.uint32) & 0x1FFF) == 0)            # 10 mantissa bits left
+    assert np.array_equal(oracle.tf32_round(r), r)               # idempotent
+    assert np.array_equal(np.signbit(r), np.signbit(x))
+    # nearest: within half a TF32 spacing (2**(e-10) in the binade of |x|)
+    _, e = np.frexp(x.astype(np.float64))
+    half = np.ldexp(1.0, e - 12)
+    assert np.all(np.abs(r.astype(np.float64) - x.astype(np.float64)) <= half)
+    # unbiased on random data, unlike dropping the 13 bits (which always shrinks |x|)
+    rel = (r.astype(np.float64) - x) / x
+    assert abs(rel.mean()) < 2e-6
+    trunc = (x.view(np.uint32) & np.uint32(0xFFFFE000)).view(np.float32)
+    assert ((trunc.astype(np.float64) - x) / x).mean() < -1e-4
