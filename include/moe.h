@@ -104,6 +104,15 @@ typedef enum moe_dtype {
 #define MOE_DEV_BAD_INDEX   1  /* an expert index or slot was out of range; the row was skipped */
 #define MOE_DEV_BAD_OFFSETS 2  /* offsets not an exclusive scan ending at R; GEMM skipped */
 #define MOE_DEV_TIMEOUT     4  /* a bounded device wait gave up; results are invalid */
+/* With the environment variable MOE_CHECKS set (to anything but "" or "0", read at each
+ * call): moe_route and moe_layer_fwd verify the routing they produce, and moe_dispatch
+ * the slots it is given, as a whole -- slot maps the T*k (token, expert) pairs to
+ * distinct rows in [0,R), inside each pair's expert range, with row_token[slot[t,j]]
+ * == t; offsets are a monotone scan of the counts ending at R (or the multiples of the
+ * capacity); moe_grouped_gemm_fwd checks the offsets -- and set this bit on a failure.
+ * The checks add device launches and a bitmap of R bits in the workspace; off by
+ * default. */
+#define MOE_DEV_CHECK_FAILED 8
 
 typedef struct moe_desc {
   int32_t T, d, d_ff, E, k;

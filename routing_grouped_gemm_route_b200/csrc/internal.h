@@ -36,6 +36,15 @@ cudaError_t launch_router_gemm(bool fp32_act, int M, int N, int K, const void* A
                                int64_t sbn, bool b_is_act, void* C, bool c_is_act,
                                bool accumulate, cudaStream_t s);
 
+// MOE_CHECKS: whole-layout verification of the routing (slot a permutation / injection
+// into the experts' ranges, offsets a monotone scan), setting MOE_DEV_CHECK_FAILED.
+bool checks_enabled();
+size_t check_scratch_bytes(int64_t R);   // the bitmap: one bit per routed row
+// null slot: offsets only; null topk_idx / offsets / counts / row_token: those parts skipped
+cudaError_t launch_checks(const int32_t* slot, const int32_t* topk_idx, const int32_t* offsets,
+                          const int32_t* counts, const int32_t* row_token, int T, int k, int E,
+                          int R, int capacity, uint32_t* bitmap, int* status, cudaStream_t s);
+
 // ----------------------------------------------------------------------------- permute
 // R: the number of routed rows (slots must be in [0, R)): T*k, or E*capacity padded.
 cudaError_t launch_dispatch(bool fp32, int T, int d, int k, int R, const void* x,

@@ -47,6 +47,7 @@ struct WsLayout {
   size_t sh_f32, sh_dH13, rc_sh_H13, rc_sh_a;   // shared expert: y / dx (float), dH13, recompute
   size_t mx_ints, mx_bytes[24];   // MXFP8 operands (codes and scale chunks), see MxWork
   size_t w13_t, w2_t, x_t, dy_t;  // fp32: TF32-rounded weights (and shared expert's x, dy)
+  size_t checks;                  // MOE_CHECKS bitmap
   size_t total;
 };
 
@@ -60,6 +61,7 @@ WsLayout ws_layout(const moe_desc& d) {
   w.hist = o; o = up(o + hrows * d.E * 4);
   w.cta_base = o; o = up(o + ctas * d.E * 4);
   w.maps = o; o = up(o + 2 * (size_t)d.E * kTensorMapBytes);
+  w.checks = o; o = up(o + check_scratch_bytes((int64_t)R));
   w.dy_perm = o; o = up(o + R * d.d * es);
   w.dH13 = o; o = up(o + R * 2 * (size_t)d.d_ff * es);
   w.dx_perm = o; o = up(o + R * d.d * es);
@@ -286,9 +288,13 @@ moe_status route_body(const moe_desc& d, const float* logits, int32_t* idx, floa
     MOE_TRY(cu(cudaMemsetAsync(counts, 0, sizeof(int32_t) * d.E, s)));
     return cu(cudaMemsetAsync(offsets, 0, sizeof(int32_t) * (d.E + 1), s));
   }
-  return cu(launch_route(d, logits, idx, gates, counts, offsets, slot, row_token, row_gate,
-                         at<int32_t>(ws, w.hist), at<int32_t>(ws, w.cta_base),
-                         at<unsigned int>(ws, kRouteCounterOffset), status_ptr(ws), s));
+  MOE_TRY(cu(launch_route(d, logits, idx, gates, counts, offsets, slot, row_token, row_gate,
+                          at<int32_t>(ws, w.hist), at<int32_t>(ws, w.cta_base),
+                          at<unsigned int>(ws, kRouteCounterOffset), status_ptr(ws), s)));
+  if (checks_enabled())
+    MOE_TRY(cu(launch_checks(slot, idx, offsets, counts, row_token, d.T, d.k, d.E, (int)R_of(d),
+                             d.capacity, at<uint32_t>(ws, w.checks), status_ptr(ws), s)));
+  return MOE_OK;
 }
 
 moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_perm,
@@ -435,6 +441,10 @@ moe_status moe_dispatch(const moe_desc* desc, const void* x, const int32_t* slot
   if (x_perm_sf) return MOE_EINVAL;
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   const moe_desc& d = *desc;
+  if (checks_enabled())
+    MOE_TRY(cu(launch_checks(slot, nullptr, nullptr, nullptr, nullptr, d.T, d.k, d.E, (int)R_of(d),
+                             d.capacity, at<uint32_t>(ws, ws_layout(d).checks), status_ptr(ws),
+                             S(stream))));
   return dispatch_body(d, x, slot, x_perm, status_ptr(ws), S(stream));
 }
 
@@ -447,6 +457,10 @@ moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const 
   if (x_perm_sf) return MOE_EINVAL;
   MOE_TRY(ws_ok(*desc, ws, ws_bytes));
   if (R_of(*desc) == 0) return MOE_OK;
+  if (checks_enabled())
+    MOE_TRY(cu(launch_checks(nullptr, nullptr, offsets, nullptr, nullptr, desc->T, desc->k,
+                             desc->E, (int)R_of(*desc), desc->capacity, nullptr, status_ptr(ws),
+                             S(stream))));
   MxWork mx = mx_work(*desc, ws);
   Weights wt;
   MOE_TRY(tf32_weights(*desc, W13, W2, ws, S(stream), &wt));

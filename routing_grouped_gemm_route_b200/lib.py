@@ -22,7 +22,7 @@ MOE_FP32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
 MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW, MOE_FLAG_RECOMPUTE = 1, 2, 4, 8
 MOE_FLAG_SHARED_EXPERT = 16
 MOE_FLAG_TEST_WAIT_TIMEOUT = 1 << 30      # test hook: the GEMMs' device waits run out
-MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT = 1, 2, 4
+MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT, MOE_DEV_CHECK_FAILED = 1, 2, 4, 8
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024
 
 DTYPES = {"fp32": MOE_FP32, "bf16": MOE_BF16, "mxfp8": MOE_MXFP8}

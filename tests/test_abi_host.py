@@ -220,3 +220,17 @@ def test_product_code_never_reaches_the_oracle():
             if "oracle" in fh.read():
                 bad.append(f"include/{name}")
     assert not bad, bad
+
+
+def test_binding_constants_match_the_header():
+    """Every MOE_FLAG_* / MOE_DEV_* / MOE_* status the header defines has the same value in
+    the binding (which only passes them through)."""
+    import re
+    hdr = open(os.path.join(ROOT, "include", "moe.h")).read()
+    found = 0
+    for name, expr in re.findall(r"#define (MOE_(?:FLAG|DEV)_[A-Z0-9_]+)\s+(\(?[0-9 <]+\)?)", hdr):
+        assert getattr(lib, name) == eval(expr), name
+        found += 1
+    assert found >= 9
+    for name, val in re.findall(r"(MOE_E[A-Z]+|MOE_OK)\s*=\s*(-?\d+)", hdr):
+        assert getattr(lib, name) == int(val), name
