@@ -192,8 +192,9 @@ __device__ __forceinline__ Tile decode_tile(int t, int n_tiles, int m_tiles, con
     tl.cnt = 0;
   } else {
     const int per = m_tiles * n_tiles;
-    tl.e = t / per;
-    const int r = t - tl.e * per;
+    const int slot = t / per;
+    tl.e = s_mt[slot];               // RAGGED_K: s_mt holds the experts, longest K first
+    const int r = t - slot * per;
     const int mt = r / n_tiles;
     tl.m0 = mt * TM;
     tl.n0 = (r - mt * n_tiles) * BN;
@@ -415,6 +416,26 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     }
   }
   __syncthreads();
+  if (MODE == RAGGED_K) {
+    // Tiles are dealt to the CTAs round-robin, expert by expert.  When the experts' row
+    // counts are skewed (the largest above twice the mean), ordering the experts by row
+    // count (longest K first, ties to the lower index) keeps the long tiles of hot experts
+    // from piling up on a few CTAs; otherwise the experts keep their own order (the
+    // layout order of their rows and weights).  (s_mt, the ragged-M tile prefix, is not
+    // used by the ragged-K tiles: it holds the order instead.)
+    for (int e = threadIdx.x; e < E; e += C::THREADS) {
+      const int c = s_off[e + 1] - s_off[e];
+      int rank = 0, mx = 0;
+      for (int o = 0; o < E; ++o) {
+        const int co = s_off[o + 1] - s_off[o];
+        rank += co > c || (co == c && o < e);
+        mx = co > mx ? co : mx;
+      }
+      const bool skewed = (int64_t)mx * E > 2 * (int64_t)(s_off[E] - s_off[0]);
+      s_mt[skewed ? rank : e] = e;
+    }
+    __syncthreads();
+  }
   const int total = s_total[0];
   if (unit >= total) return;   // uniform over the CTA (and over a CTA pair)
 
