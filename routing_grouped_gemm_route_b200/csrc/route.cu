@@ -5,17 +5,20 @@
 // path's host round trip for the expert-group sizes, so the CPU can queue work
 // without waiting for a copy back (deniz.in, "Ai2, Olmo-core 3'ü Apache 2.0 ile
 // yayınladı", section "Yeni stack nasıl çalışıyor"; unite.ai, "पैरालेलिज़्म, प्रिसीजन,
-// और मेमोरी तकनीकें").  Two launches (three above 256 experts), no host sync:
+// और मेमोरी तकनीकें").  Two launches (three above 256 experts, or above 32768 tokens
+// when the caller gives no counter), no host sync:
 //   1. topk:  one warp per token, logits in registers, k rounds of warp arg-max
 //             (ties to the lower expert index); gates = softmax over the kept
 //             logits; an expert histogram per 64 tokens (one CTA each, so even a
 //             few thousand tokens spread over every SM).
-//   2. scan:  the last top-k CTA to finish (a counter in global memory, the
-//             classic fence-then-count pattern: no CTA waits for another): per expert,
-//             an exclusive scan of the histogram rows (each expert's column split over
-//             several threads), giving the base of every 256-token slot CTA inside the
-//             expert, the counts, and offsets = exclusive scan of counts.  (Above 256
-//             experts, where top-k runs 8-warp CTAs, it is a separate one-CTA launch.)
+//   2. prefix: per expert, an exclusive scan of the histogram rows gives the base of
+//             every 256-token slot CTA inside the expert, the counts, and offsets =
+//             exclusive scan of the counts.  Up to 512 histogram rows (32768 tokens)
+//             and 256 experts, each slot CTA sums the rows it needs itself (step 3).
+//             Above that, the last top-k CTA to finish runs the scan (a counter in
+//             global memory, the classic fence-then-count pattern: no CTA waits for
+//             another), each expert's column split over several threads; above 256
+//             experts, where top-k runs 8-warp CTAs, it is a separate one-CTA launch.
 //   3. slots: per warp of 32 tokens, a bitmask per expert of the lanes that chose
 //             it; a token's rank inside the expert is the population count of the
 //             lower lanes' bits plus the bases of earlier warps and CTAs.  So the
