@@ -159,7 +159,9 @@ struct FusedScan {
 // every lane (its lowest index on ties), the warp's largest key by one reduction and the
 // lowest index holding it by a second: ties go to the lower expert index, as the
 // descending stable order of the logits has it.
-template <int NPL>   // logits per lane = ceil(E / 32)
+// FUSED: the CTA that finishes last runs the scan (compiled only where it is used: its
+// register arrays do not fit the 32 registers a thread of the scan-free CTAs has).
+template <int NPL, bool FUSED>   // logits per lane = ceil(E / 32)
 __global__ void __launch_bounds__(topk_warps<NPL>() * 32, topk_ctas_per_sm<NPL>())
 topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ topk_idx,
             float* __restrict__ gates, int32_t* __restrict__ hist, FusedScan fs) {
@@ -169,7 +171,22 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
   __syncthreads();
 
   const int t0 = blockIdx.x * kRouteTokensPerHistRow;
-  for (int i = warp; i < kRouteTokensPerHistRow; i += topk_warps<NPL>()) {
+  // a warp's tokens: their logits are all loaded before the first selection (NPL <= 4:
+  // two tokens a warp, 2 * NPL registers), so their memory latencies overlap
+  constexpr int kPre = NPL <= 4 ? kRouteTokensPerHistRow / topk_warps<NPL>() : 1;
+  float pre[kPre][NPL];
+  if constexpr (kPre > 1) {
+#pragma unroll
+    for (int u = 0; u < kPre; ++u) {
+      const int t = t0 + warp + u * topk_warps<NPL>();
+#pragma unroll
+      for (int c = 0; c < NPL; ++c) {
+        const int e = c * 32 + lane;
+        pre[u][c] = t < T && e < E ? logits[(int64_t)t * E + e] : 0.f;
+      }
+    }
+  }
+  for (int i = warp, u = 0; i < kRouteTokensPerHistRow; i += topk_warps<NPL>(), ++u) {
     const int t = t0 + i;
     if (t >= T) break;
     const float* row = logits + (int64_t)t * E;
@@ -177,7 +194,14 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
 #pragma unroll
     for (int c = 0; c < NPL; ++c) {
       const int e = c * 32 + lane;
-      float f = e < E ? row[e] : 0.f;
+      float f = 0.f;
+      if constexpr (kPre > 1) {
+#pragma unroll
+        for (int uu = 0; uu < kPre; ++uu)
+          if (uu == u) f = pre[uu][c];
+      } else {
+        f = e < E ? row[e] : 0.f;
+      }
       // a NaN logit ranks as -inf (it would lose every comparison, and a row of them
       // would select no expert at all)
       if (f != f) f = -INFINITY;
@@ -220,7 +244,11 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
   }
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
-  if constexpr (topk_warps<NPL>() * 32 == kScanThreads) {
+  // This CTA is done: the slot kernel (a programmatic dependent, which waits for this
+  // grid's completion itself) may be scheduled once every CTA got here.  Not earlier:
+  // CTAs scheduled while top-k holds the SMs would crowd onto the few with room.
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  if constexpr (FUSED && topk_warps<NPL>() * 32 == kScanThreads) {
     if (fs.done == nullptr) return;
     // the last CTA to finish scans every CTA's histogram row
     __shared__ int s_last;
@@ -255,19 +283,23 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
   int* wbase = reinterpret_cast<int*>(s_mem + kWarps * E);          // [kWarps][E]
   int* s_off = wbase + kWarps * E;                                  // [E] (NPL > 0)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // launched as a programmatic dependent of the top-k kernel: everything it wrote is
+  // visible from here on
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   int start = 0;                     // thread e: the CTA's first row in expert e
   if constexpr (NPL > 0) {
     // per-warp sums of the rows before this CTA and of all rows, into masks / wbase
+    // (eight rows of loads in flight per warp)
     const int r_cta = blockIdx.x * kHistRowsPerCta;
     int pre[NPL], tot[NPL];
 #pragma unroll
     for (int c = 0; c < NPL; ++c) pre[c] = tot[c] = 0;
-#pragma unroll 4
+#pragma unroll 8
     for (int r = warp; r < nrows; r += kWarps) {
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         const int e = c * 32 + lane;
-        const int v = e < E ? hist[(int64_t)r * E + e] : 0;
+        const int v = e < E ? __ldcg(hist + (int64_t)r * E + e) : 0;
         tot[c] += v;
         if (r < r_cta) pre[c] += v;
       }
@@ -367,9 +399,14 @@ cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, 
                         int32_t* hist, const FusedScan& fs, cudaStream_t s) {
   const int ctas = route_hist_rows(T);
   // the fused scan reuses the histogram's shared memory (kScanThreads ints)
-  const int words = fs.done != nullptr && E < kScanThreads ? kScanThreads : E;
-  topk_kernel<NPL><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(logits, T, E, k, idx,
-                                                                            gates, hist, fs);
+  const bool fused = fs.done != nullptr;
+  const int words = fused && E < kScanThreads ? kScanThreads : E;
+  if (fused)
+    topk_kernel<NPL, true><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(
+        logits, T, E, k, idx, gates, hist, fs);
+  else
+    topk_kernel<NPL, false><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(
+        logits, T, E, k, idx, gates, hist, fs);
   return cudaGetLastError();
 }
 
@@ -509,16 +546,30 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
     if ((err = cudaMemsetAsync(row_token, 0xff, rows * 4, s)) != cudaSuccess) return err;
     if ((err = cudaMemsetAsync(row_gate, 0, rows * 4, s)) != cudaSuccess) return err;
   }
-#define MOE_SLOT(NP)                                                                            \
-  slot_kernel<NP><<<ctas, kWarps * 32, smem, s>>>(topk_idx, gates, offsets, cta_base, hist, nrows, \
-                                                  counts, T, E, k, C, slot, row_token, row_gate,  \
-                                                  status)
-  if (!in_slot) MOE_SLOT(0);
-  else if (npl <= 1) MOE_SLOT(1);
-  else if (npl <= 2) MOE_SLOT(2);
-  else if (npl <= 4) MOE_SLOT(4);
-  else MOE_SLOT(8);
-#undef MOE_SLOT
+  // The slot kernel is a programmatic dependent of the kernel before it (top-k, or the
+  // scan): it may be scheduled while that one drains and waits for it in-kernel.  (The
+  // padded layout's memsets come between them: then it is an ordinary launch.)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(ctas, 1, 1);
+  cfg.blockDim = dim3(kWarps * 32, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = C > 0 ? 0 : 1;
+  auto go = [&](auto kern) {
+    return cudaLaunchKernelEx(&cfg, kern, (const int32_t*)topk_idx, (const float*)gates, offsets,
+                              (const int32_t*)cta_base, (const int32_t*)hist, nrows, counts, T, E,
+                              k, C, slot, row_token, row_gate, status);
+  };
+  if (!in_slot) err = go(slot_kernel<0>);
+  else if (npl <= 1) err = go(slot_kernel<1>);
+  else if (npl <= 2) err = go(slot_kernel<2>);
+  else if (npl <= 4) err = go(slot_kernel<4>);
+  else err = go(slot_kernel<8>);
+  if (err != cudaSuccess) return err;
   return cudaGetLastError();
 }
 
