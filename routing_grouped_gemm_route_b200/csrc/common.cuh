@@ -54,6 +54,18 @@ __device__ __forceinline__ void set_status(int* status, int bits) {
   if (status) atomicOr(status, bits);
 }
 
+// Programmatic dependent launch.  A kernel started with launch_pdl may be scheduled
+// while the kernel before it in the stream drains; pdl_wait(), before its first access
+// to global memory, waits for that kernel's completion and the visibility of all its
+// writes, so the data dependences are those of an ordinary launch.  pdl_trigger() lets
+// the next such kernel be scheduled once every CTA of this one has called it or exited
+// (placed at the end of the work: earlier, the next kernel's CTAs would take SM slots
+// while this one still has CTAs to place).  Both do nothing in an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint64_t globaltimer_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));

@@ -340,6 +340,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
   static_assert(MODE == RAGGED_M || (A_MN && B_MN && EPI == EPI_STORE), "wgrad layout");
 
+  // a programmatic dependent of the previous kernel: its writes are visible from here on
+  pdl_wait();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -916,6 +918,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
     __syncwarp();
   }
 
+  pdl_trigger();   // this CTA's tiles are done
   // A pair's leader reads the follower's shared memory and writes its TMEM until its
   // last MMA completes (the leader waited for that above): neither CTA leaves before.
   tc_fence_before();
@@ -935,6 +938,7 @@ __global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
                                    const __grid_constant__ CUtensorMap tmpl1,
                                    const int32_t* __restrict__ offsets, int E, int R,
                                    CUtensorMap* maps) {
+  pdl_wait();
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= 2 * E) return;
   const int e = i < E ? i : i - E;
@@ -945,6 +949,7 @@ __global__ void expert_maps_kernel(const __grid_constant__ CUtensorMap tmpl0,
   const int rows = offsets ? offsets[e + 1] : R;   // no offsets: one segment of R rows
   tmap_replace_row_dim(maps + i, static_cast<uint32_t>(rows > 0 ? rows : 1));
   fence_tmap_release();
+  pdl_trigger();
 }
 
 // =============================================================================== host side
@@ -1048,17 +1053,17 @@ static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ECUDA;
   cudaLaunchConfig_t cfg = {};
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  cfg.attrs = attr;
   int units = num_sms();
   if (PAIR) {
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
     cfg.numAttrs = 1;
     // how many CTA pairs fit at once (one CTA per SM: the shared memory takes it all)
     static int max_pairs[64] = {0};
@@ -1074,6 +1079,10 @@ static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUt
   }
   if (max_tiles < units) units = max_tiles;
   if (units < 1) return MOE_OK;
+  // a programmatic dependent of the previous kernel (the kernel waits for it itself)
+  attr[cfg.numAttrs].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[cfg.numAttrs].val.programmaticStreamSerializationAllowed = 1;
+  ++cfg.numAttrs;
   cfg.gridDim = dim3(PAIR ? 2 * units : units, 1, 1);
   if (cudaLaunchKernelEx(&cfg, kern, ta, tb, to, to2, ti, tsa, tsb, p) != cudaSuccess)
     return MOE_ECUDA;
@@ -1311,8 +1320,8 @@ static moe_status build_wgrad_maps(const GemmShape& g, const void* dy_perm, cons
       return MOE_ECUDA;
   }
   const int threads = 2 * g.E;
-  expert_maps_kernel<<<(threads + 127) / 128, 128, 0, s>>>(t0, t1, off, g.E, g.R, maps);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ECUDA;
+  return launch_pdl(expert_maps_kernel, (threads + 127) / 128, 128, 0, s, t0, t1, off, g.E, g.R,
+                    maps) == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 // ------------------------------------------------------------------------ MXFP8 GEMMs
@@ -1508,8 +1517,9 @@ static moe_status router_dwr_tc(int T, int d, int E, const void* x, const void* 
   using C = Cfg<bf16, bf16, 128, EPI_STORE>;
   CUtensorMap t0;
   if (!make_tmap_mn3(&t0, x, 2, d, T, C::KB, BM / C::MNB)) return MOE_ECUDA;
-  expert_maps_kernel<<<1, 128, 0, s>>>(t0, t0, nullptr, 1, T, maps);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ECUDA;
+  if (launch_pdl(expert_maps_kernel, 1, 128, 0, s, t0, t0, (const int32_t*)nullptr, 1, T, maps) !=
+      cudaSuccess)
+    return MOE_ECUDA;
   const int bn = bn_of(E);
   if (d % 256 == 0 && bn >= 128) {
     if (bn == 256) return run_k<bf16, bf16, 256, true>(g, x, d, dl16, E, dWr, false, nullptr, maps, st, s);

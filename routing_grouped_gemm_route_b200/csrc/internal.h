@@ -11,6 +11,24 @@ namespace moe {
 
 int num_sms();
 
+// Launch as a programmatic dependent of the previous kernel in the stream (the kernel
+// calls pdl_wait() before it touches global memory).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ----------------------------------------------------------------------------- routing
 // Top-k CTAs take 64 tokens each and write one row of the expert histogram; the slot
 // CTAs take 256 (8 warps x 32 tokens) and read the expert bases at their first token.

@@ -33,6 +33,7 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(const T* __restri
                                                                const int32_t* __restrict__ slot,
                                                                T* __restrict__ x_perm, int T_,
                                                                int d, int k, int R, int* status) {
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
   if (t >= T_) return;
@@ -69,6 +70,7 @@ __global__ void __launch_bounds__(kWarps * 32) dispatch_kernel(const T* __restri
       }
     }
   }
+  pdl_trigger();
 }
 
 // y[t] = sum_j w_tj * src[slot[t,j]] (+ extra[t]), w = gates or 1
@@ -77,6 +79,7 @@ __global__ void __launch_bounds__(kWarps * 32) gather_sum_kernel(
     const T* __restrict__ src, const float* __restrict__ gates, const int32_t* __restrict__ slot,
     const float* __restrict__ extra, const float* __restrict__ extra2, T* __restrict__ y, int T_,
     int d, int k, int R, int* status) {
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
   if (t >= T_) return;
@@ -136,6 +139,7 @@ __global__ void __launch_bounds__(kWarps * 32) gather_sum_kernel(
     o.from_float(acc);
     stg16(y + (int64_t)t * d + (int64_t)v * V, o.raw);
   }
+  pdl_trigger();
 }
 
 // dy_perm[slot] = g * dy[t]; dg = <dy[t], y_perm[slot]>; d_logits via the softmax Jacobian
@@ -144,6 +148,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
     const T* __restrict__ dy, const T* __restrict__ y_perm, const float* __restrict__ gates,
     const int32_t* __restrict__ topk_idx, const int32_t* __restrict__ slot, T* __restrict__ dy_perm,
     float* __restrict__ d_logits, int T_, int d, int k, int E, int R, int* status) {
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
   if (t >= T_) return;
@@ -209,6 +214,7 @@ __global__ void __launch_bounds__(kWarps * 32) combine_bwd_kernel(
   for (int e = lane; e < E; e += 32) row[e] = 0.f;
   __syncwarp();
   if (lane < k && my_e >= 0 && my_e < E) row[my_e] = my_dl;
+  pdl_trigger();
 }
 
 // y[i] += extra[i] (fp32 add, one rounding to T)
@@ -288,28 +294,27 @@ cudaError_t launch_dispatch(bool fp32, int T, int d, int k, int R, const void* x
   if (T == 0) return cudaSuccess;
   const int blocks = (T + kWarps - 1) / kWarps;
   if (fp32)
-    dispatch_kernel<float><<<blocks, kWarps * 32, 0, s>>>((const float*)x, slot, (float*)x_perm, T,
-                                                          d, k, R, status);
-  else
-    dispatch_kernel<__nv_bfloat16><<<blocks, kWarps * 32, 0, s>>>(
-        (const __nv_bfloat16*)x, slot, (__nv_bfloat16*)x_perm, T, d, k, R, status);
-  return cudaGetLastError();
+    return launch_pdl(dispatch_kernel<float>, blocks, kWarps * 32, 0, s, (const float*)x, slot,
+                      (float*)x_perm, T, d, k, R, status);
+  return launch_pdl(dispatch_kernel<__nv_bfloat16>, blocks, kWarps * 32, 0, s,
+                    (const __nv_bfloat16*)x, slot, (__nv_bfloat16*)x_perm, T, d, k, R, status);
 }
 
 template <typename T>
-static void gather_sum_t(int km, int blocks, cudaStream_t s, const void* src, const float* gates,
-                         const int32_t* slot, const float* extra, const float* extra2, void* y,
-                         int T_, int d, int k, int R, int* status) {
-#define MOE_GS(KM)                                                                            \
-  gather_sum_kernel<T, KM><<<blocks, kWarps * 32, 0, s>>>((const T*)src, gates, slot, extra, \
-                                                          extra2, (T*)y, T_, d, k, R, status)
+static cudaError_t gather_sum_t(int km, int blocks, cudaStream_t s, const void* src,
+                                const float* gates, const int32_t* slot, const float* extra,
+                                const float* extra2, void* y, int T_, int d, int k, int R,
+                                int* status) {
+#define MOE_GS(KM)                                                                             \
+  return launch_pdl(gather_sum_kernel<T, KM>, blocks, kWarps * 32, 0, s, (const T*)src, gates, \
+                    slot, extra, extra2, (T*)y, T_, d, k, R, status)
   switch (km) {
-    case 1: MOE_GS(1); break;
-    case 2: MOE_GS(2); break;
-    case 4: MOE_GS(4); break;
-    case 8: MOE_GS(8); break;
-    case 16: MOE_GS(16); break;
-    default: MOE_GS(32); break;
+    case 1: MOE_GS(1);
+    case 2: MOE_GS(2);
+    case 4: MOE_GS(4);
+    case 8: MOE_GS(8);
+    case 16: MOE_GS(16);
+    default: MOE_GS(32);
   }
 #undef MOE_GS
 }
@@ -321,29 +326,27 @@ cudaError_t launch_gather_sum(bool fp32, int T, int d, int k, int R, const void*
   const int blocks = (T + kWarps - 1) / kWarps;
   const int km = kmax_of(k);
   if (fp32)
-    gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, R, status);
-  else
-    gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, R,
-                                status);
-  return cudaGetLastError();
+    return gather_sum_t<float>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k, R,
+                               status);
+  return gather_sum_t<__nv_bfloat16>(km, blocks, s, src, gates, slot, extra, extra2, y, T, d, k,
+                                     R, status);
 }
 
 template <typename T>
-static void combine_bwd_t(int km, int blocks, cudaStream_t s, const void* dy, const void* y_perm,
-                          const float* gates, const int32_t* idx, const int32_t* slot,
-                          void* dy_perm, float* dl, int T_, int d, int k, int E, int R,
-                          int* status) {
-#define MOE_CB(KM)                                                                         \
-  combine_bwd_kernel<T, KM><<<blocks, kWarps * 32, 0, s>>>((const T*)dy, (const T*)y_perm, \
-                                                           gates, idx, slot, (T*)dy_perm, dl, \
-                                                           T_, d, k, E, R, status)
+static cudaError_t combine_bwd_t(int km, int blocks, cudaStream_t s, const void* dy,
+                                 const void* y_perm, const float* gates, const int32_t* idx,
+                                 const int32_t* slot, void* dy_perm, float* dl, int T_, int d,
+                                 int k, int E, int R, int* status) {
+#define MOE_CB(KM)                                                                              \
+  return launch_pdl(combine_bwd_kernel<T, KM>, blocks, kWarps * 32, 0, s, (const T*)dy,         \
+                    (const T*)y_perm, gates, idx, slot, (T*)dy_perm, dl, T_, d, k, E, R, status)
   switch (km) {
-    case 1: MOE_CB(1); break;
-    case 2: MOE_CB(2); break;
-    case 4: MOE_CB(4); break;
-    case 8: MOE_CB(8); break;
-    case 16: MOE_CB(16); break;
-    default: MOE_CB(32); break;
+    case 1: MOE_CB(1);
+    case 2: MOE_CB(2);
+    case 4: MOE_CB(4);
+    case 8: MOE_CB(8);
+    case 16: MOE_CB(16);
+    default: MOE_CB(32);
   }
 #undef MOE_CB
 }
@@ -356,12 +359,10 @@ cudaError_t launch_combine_bwd(bool fp32, int T, int d, int k, int E, int R, con
   const int blocks = (T + kWarps - 1) / kWarps;
   const int km = kmax_of(k);
   if (fp32)
-    combine_bwd_t<float>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm, d_logits, T, d,
-                         k, E, R, status);
-  else
-    combine_bwd_t<__nv_bfloat16>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm,
-                                 d_logits, T, d, k, E, R, status);
-  return cudaGetLastError();
+    return combine_bwd_t<float>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm,
+                                d_logits, T, d, k, E, R, status);
+  return combine_bwd_t<__nv_bfloat16>(km, blocks, s, dy, y_perm, gates, topk_idx, slot, dy_perm,
+                                      d_logits, T, d, k, E, R, status);
 }
 
 }  // namespace moe

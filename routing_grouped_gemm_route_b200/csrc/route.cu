@@ -166,6 +166,7 @@ __global__ void __launch_bounds__(topk_warps<NPL>() * 32, topk_ctas_per_sm<NPL>(
 topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __restrict__ topk_idx,
             float* __restrict__ gates, int32_t* __restrict__ hist, FusedScan fs) {
   extern __shared__ int s_hist[];          // [E] (fused: [max(E, kScanThreads)], then the scan's)
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
@@ -247,7 +248,7 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
   // This CTA is done: the slot kernel (a programmatic dependent, which waits for this
   // grid's completion itself) may be scheduled once every CTA got here.  Not earlier:
   // CTAs scheduled while top-k holds the SMs would crowd onto the few with room.
-  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  pdl_trigger();
   if constexpr (FUSED && topk_warps<NPL>() * 32 == kScanThreads) {
     if (fs.done == nullptr) return;
     // the last CTA to finish scans every CTA's histogram row
@@ -285,7 +286,7 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // launched as a programmatic dependent of the top-k kernel: everything it wrote is
   // visible from here on
-  asm volatile("griddepcontrol.wait;" ::: "memory");
+  pdl_wait();
   int start = 0;                     // thread e: the CTA's first row in expert e
   if constexpr (NPL > 0) {
     // per-warp sums of the rows before this CTA and of all rows, into masks / wbase
@@ -392,6 +393,7 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
       row_gate[s] = gates[(int64_t)t * k + j];
     }
   }
+  pdl_trigger();
 }
 
 template <int NPL>
@@ -402,12 +404,10 @@ cudaError_t launch_topk(const float* logits, int T, int E, int k, int32_t* idx, 
   const bool fused = fs.done != nullptr;
   const int words = fused && E < kScanThreads ? kScanThreads : E;
   if (fused)
-    topk_kernel<NPL, true><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(
-        logits, T, E, k, idx, gates, hist, fs);
-  else
-    topk_kernel<NPL, false><<<ctas, topk_warps<NPL>() * 32, words * sizeof(int), s>>>(
-        logits, T, E, k, idx, gates, hist, fs);
-  return cudaGetLastError();
+    return launch_pdl(topk_kernel<NPL, true>, ctas, topk_warps<NPL>() * 32, words * sizeof(int),
+                      s, logits, T, E, k, idx, gates, hist, fs);
+  return launch_pdl(topk_kernel<NPL, false>, ctas, topk_warps<NPL>() * 32, words * sizeof(int), s,
+                    logits, T, E, k, idx, gates, hist, fs);
 }
 
 // ----------------------------------------------------------------------------- router GEMM
