@@ -166,6 +166,61 @@ class ClockSampler:
                 "power_w_max": max(power) if power else None, "reasons": sorted(reasons)}
 
 
+class NvmlSampler:
+    """SM clock and board power read in-process every ~2 ms while the timed steps run.
+
+    nvidia-smi samples every 100 ms at best, so a timed region of a few tens of ms holds
+    one sample or none, and the idle clock before it dominates the record.  NVML is read
+    here from a thread, started right before the first timed launch and stopped right
+    after the synchronize that ends the region (the GPU runs the queued steps meanwhile).
+    The device is matched by PCI bus id (falls back to the index)."""
+
+    def __init__(self, dev_index: int):
+        self.h, self.samples, self.thread, self.stop_flag = None, [], None, False
+        try:
+            import pynvml
+            self.nv = pynvml
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(dev_index)
+            try:
+                bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id,
+                                            props.pci_device_id)
+                self.h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:  # noqa: BLE001
+                self.h = pynvml.nvmlDeviceGetHandleByIndex(dev_index)
+        except Exception:  # noqa: BLE001
+            self.h = None
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_flag:
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:  # noqa: BLE001
+                return
+            time.sleep(0.002)
+
+    def start(self):
+        if self.h is None:
+            return
+        import threading
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def stop(self) -> dict:
+        if self.thread is None:
+            return {}
+        self.stop_flag = True
+        self.thread.join(timeout=5)
+        if not self.samples:
+            return {}
+        sm = [c for c, _ in self.samples]
+        pw = [w for _, w in self.samples]
+        return {"sm_mhz": statistics.median(sm), "sm_mhz_min": min(sm), "samples": len(sm),
+                "power_w_median": round(statistics.median(pw), 1), "power_w_max": round(max(pw), 1)}
+
+
 def dist_setup():
     """One process per GPU under torchrun (NCCL); gloo when no GPU is visible (CPU runs of
     the multi-rank bookkeeping and of the reference arm)."""
@@ -539,6 +594,8 @@ def main():
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
+    nvml = NvmlSampler(local)
+    nvml.start()
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     start.record()
     for i in range(K):
@@ -550,7 +607,15 @@ def main():
     stop.record()
     torch.cuda.synchronize()
     barrier(world)
+    in_region = nvml.stop()
     clk = clocks.stop()
+    if in_region.get("samples", 0) >= 3:
+        # the in-region NVML record decides the clock; nvidia-smi gives the throttle reasons
+        clk = dict(clk, smi_sm_mhz=clk.get("sm_mhz"), smi_samples=clk.get("samples"),
+                   sm_mhz=in_region["sm_mhz"], sm_mhz_min=in_region["sm_mhz_min"],
+                   samples=in_region["samples"], power_w_median=in_region["power_w_median"],
+                   power_w_max=in_region["power_w_max"],
+                   source="NVML every ~2 ms during the timed region (reasons: nvidia-smi)")
     ms_local = start.elapsed_time(stop)
     ms_total = max_over_ranks(ms_local, world)
     if lib.moe_read_device_status(layer.ws if layer else ws) != 0:

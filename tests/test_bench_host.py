@@ -91,3 +91,17 @@ def test_tensor_peak_burst_only_at_full_clock():
     assert abs(fp8["peak"] - 1652.2 * 2) < 1e-9 and fp8["nominal"] == 4500.0
     tf32 = bench.tensor_peak(pk, "tf32", {"sm_mhz": 1300.0, "sm_max_mhz": 1965.0}, 0.06)
     assert abs(tf32["peak"] - 1379.2 * 1.1 / 2.25) < 1e-9
+
+
+def test_nvml_sampler_summary_and_absence(monkeypatch):
+    """The in-region sampler reports the median and minimum SM clock and the power of its
+    samples; without a usable device it reports nothing (the nvidia-smi record stands)."""
+    s = bench.NvmlSampler.__new__(bench.NvmlSampler)
+    s.h, s.thread, s.stop_flag = None, None, False
+    s.samples = []
+    assert s.stop() == {}
+    s.thread = type("T", (), {"join": lambda self, timeout=None: None})()
+    s.samples = [(1965, 400.0), (1400, 990.0), (1500, 1000.0), (1450, 995.0)]
+    r = s.stop()
+    assert r["sm_mhz"] == 1475 and r["sm_mhz_min"] == 1400 and r["samples"] == 4
+    assert r["power_w_max"] == 1000.0 and r["power_w_median"] == 992.5
