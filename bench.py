@@ -484,9 +484,12 @@ def main():
     lib.load()
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = make_inputs(w, device=dev, seed=w.seed + rank)
+    # MXFP8: the backward of a training step reuses the weight codes its forward made
+    # (the weights change only in the optimizer step after it)
     flags = (lib.MOE_FLAG_ROUTER if w.router else 0) | \
         (lib.MOE_FLAG_RECOMPUTE if args.recompute else 0) | \
-        (lib.MOE_FLAG_SHARED_EXPERT if w.shared else 0)
+        (lib.MOE_FLAG_SHARED_EXPERT if w.shared else 0) | \
+        (lib.MOE_FLAG_MX_KEEP_WEIGHT_CODES if w.dtype == "mxfp8" else 0)
     desc = lib.make_desc(w.T, w.d, w.d_ff, w.E, w.k, w.dtype, flags)
     capacity = 0
     if args.capacity is not None:

@@ -90,6 +90,20 @@ typedef enum moe_dtype {
  * It runs as the grouped GEMM with one segment of all T tokens; x is required in
  * moe_layer_bwd.  Not with MOE_MXFP8 (MOE_EUNSUPPORTED). */
 #define MOE_FLAG_SHARED_EXPERT 16
+/* MOE_MXFP8 only: keep the weights' column-wise codes from the forward for the backward.
+ * The MXFP8 GEMMs read W13 and W2 quantised along d (forward) and along their rows (the
+ * dgrads); without the flag each direction is a pass over the bf16 weights of its own.
+ * With it, a forward call (moe_layer_fwd, moe_grouped_gemm_fwd, the recompute inside
+ * moe_layer_bwd) quantises each weight both ways in one pass and records, for its
+ * workspace, the W13 / W2 pointers and the shape; a backward call on the same workspace
+ * with the same pointers and shape uses those codes instead of quantising the weights
+ * again (any other backward quantises them as usual).  The weights must not change
+ * between the two calls, as in a training step, where only the optimizer step that
+ * follows the backward changes them; the calls must be ordered on the device, like the
+ * forward's other outputs that the backward reads.  Results are bit-identical to the
+ * run without the flag.  moe_workspace_init and a forward without the flag forget the
+ * record.  MOE_EINVAL with another dtype. */
+#define MOE_FLAG_MX_KEEP_WEIGHT_CODES 32
 /* Test hook, off by default; the paper has no counterpart.  Every expert grouped-GEMM
  * launch (routed and shared experts) made under a descriptor with this flag issues no
  * operand loads and gives each of its

@@ -1385,8 +1385,10 @@ static moe_status mx_fwd(const GemmShape& g, const void* x_perm, const void* W13
   MOE_MX_TRY(cuq(launch_mx_prefix(off, E, w.act_pref, w.act_pref + (E + 1), s)));
   // FC1: x_perm and W13 rowwise along d; W13's scales in the gate/up tile order
   MOE_MX_TRY(cuq(launch_mx_quant(x_perm, g.R, d, act, 0, w.xr, w.xr_sf, nullptr, nullptr, st, s)));
+  // (with w_col_in_fwd also column-wise, for the backward's FC1 dgrad: one pass)
   MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), f, w.w13r,
-                                 w.w13r_sf, nullptr, nullptr, st, s)));
+                                 w.w13r_sf, w.w_col_in_fwd ? w.w13c : nullptr,
+                                 w.w_col_in_fwd ? w.w13c_sf : nullptr, st, s)));
   MxRefs m1;
   act_sf(m1.a, m1.a_chunks, g, w.xr_sf, d, true);
   weight_sf(m1.b, m1.b_chunks, g, w.w13r_sf, 2 * f, d, true);
@@ -1398,7 +1400,8 @@ static moe_status mx_fwd(const GemmShape& g, const void* x_perm, const void* W13
       g, w.xr, d, w.w13r, 2 * f, 2 * f, d, H13, 2 * f, a, nullptr, off, st, s, m1)));
   // FC2: W2 rowwise along d_ff (a's codes came from FC1)
   MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, w.w2r, w.w2r_sf,
-                                 nullptr, nullptr, st, s)));
+                                 w.w_col_in_fwd ? w.w2c : nullptr,
+                                 w.w_col_in_fwd ? w.w2c_sf : nullptr, st, s)));
   MxRefs m2;
   act_sf(m2.a, m2.a_chunks, g, w.ar_sf, f, true);
   weight_sf(m2.b, m2.b_chunks, g, w.w2r_sf, d, f, true);
@@ -1430,8 +1433,9 @@ static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_
   // dY both ways in one pass: rowwise along d (FC2 dgrad), colwise along tokens (FC2 wgrad);
   // W2 colwise along its d rows (FC2 dgrad)
   MOE_MX_TRY(cuq(launch_mx_quant(dy_perm, g.R, d, act, 0, w.dyr, w.dyr_sf, w.dyc, w.dyc_sf, st, s)));
-  MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, nullptr, nullptr,
-                                 w.w2c, w.w2c_sf, st, s)));
+  if (!w.w_col_ready)   // (else the forward's pass made them)
+    MOE_MX_TRY(cuq(launch_mx_quant(W2, (int64_t)E * d, f, weight_segs(E, d), 0, nullptr, nullptr,
+                                   w.w2c, w.w2c_sf, st, s)));
   MxRefs m1;
   act_sf(m1.a, m1.a_chunks, g, w.dyr_sf, d, true);
   weight_sf(m1.b, m1.b_chunks, g, w.w2c_sf, d, f, false);
@@ -1454,8 +1458,9 @@ static moe_status mx_bwd(const GemmShape& g, const void* dy_perm, const void* x_
   // colwise along tokens.  (Quantising dH13's rows in FC2 dgrad's epilogue instead was
   // slower: that epilogue holds the single accumulator, so its MMAs wait for it.)
   MOE_MX_TRY(cuq(launch_mx_quant(dH13, g.R, 2 * f, act, 0, w.dhr, w.dhr_sf, w.dhc, w.dhc_sf, st, s)));
-  MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), 0, nullptr,
-                                 nullptr, w.w13c, w.w13c_sf, st, s)));
+  if (!w.w_col_ready)
+    MOE_MX_TRY(cuq(launch_mx_quant(W13, (int64_t)E * 2 * f, d, weight_segs(E, 2 * f), 0, nullptr,
+                                   nullptr, w.w13c, w.w13c_sf, st, s)));
   MxRefs m3;
   act_sf(m3.a, m3.a_chunks, g, w.dhr_sf, 2 * f, true);
   weight_sf(m3.b, m3.b_chunks, g, w.w13c_sf, 2 * f, d, false);

@@ -113,6 +113,10 @@ struct MxWork {
   uint8_t *dhr, *dhr_sf, *dhc, *dhc_sf;   // dH13
   uint8_t *w13r, *w13r_sf, *w13c, *w13c_sf;
   uint8_t *w2r, *w2r_sf, *w2c, *w2c_sf;
+  // MOE_FLAG_MX_KEEP_WEIGHT_CODES: the forward's weight passes also write the column-wise
+  // codes (w13c, w2c); the backward finds them ready and skips its weight passes
+  bool w_col_in_fwd = false;
+  bool w_col_ready = false;
 };
 
 // ----------------------------------------------------------------------------- grouped GEMM

@@ -5,6 +5,9 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+#include <unordered_map>
+
 #include "internal.h"
 #include "moe.h"
 
@@ -146,8 +149,10 @@ moe_status check(const moe_desc* d) {
     return MOE_EINVAL;
   if (d->dtype != MOE_FP32 && d->dtype != MOE_BF16 && d->dtype != MOE_MXFP8) return MOE_EINVAL;
   if (d->flags & ~(MOE_FLAG_ROUTER | MOE_FLAG_DW_FP32 | MOE_FLAG_ACCUM_DW | MOE_FLAG_RECOMPUTE |
-                   MOE_FLAG_SHARED_EXPERT | MOE_FLAG_TEST_WAIT_TIMEOUT))
+                   MOE_FLAG_SHARED_EXPERT | MOE_FLAG_MX_KEEP_WEIGHT_CODES |
+                   MOE_FLAG_TEST_WAIT_TIMEOUT))
     return MOE_EINVAL;
+  if ((d->flags & MOE_FLAG_MX_KEEP_WEIGHT_CODES) && d->dtype != MOE_MXFP8) return MOE_EINVAL;
   if (d->capacity < 0 || (int64_t)d->E * d->capacity >= (int64_t(1) << 31)) return MOE_EINVAL;
   if (d->flags & MOE_FLAG_SHARED_EXPERT) {
     if (d->dtype == MOE_MXFP8) return MOE_EUNSUPPORTED;
@@ -297,6 +302,40 @@ moe_status route_body(const moe_desc& d, const float* logits, int32_t* idx, floa
   return MOE_OK;
 }
 
+// MOE_FLAG_MX_KEEP_WEIGHT_CODES: for each workspace, the weights (pointers and shape) whose
+// column-wise MX codes the last forward on it left in its w13c / w2c buffers.
+struct KeptCodes {
+  const void* W13;
+  const void* W2;
+  int E, d, f;
+  bool operator==(const KeptCodes& o) const {
+    return W13 == o.W13 && W2 == o.W2 && E == o.E && d == o.d && f == o.f;
+  }
+};
+std::mutex g_kept_mu;
+std::unordered_map<const void*, KeptCodes> g_kept;
+
+bool keep_codes(const moe_desc& d) {
+  return d.dtype == MOE_MXFP8 && (d.flags & MOE_FLAG_MX_KEEP_WEIGHT_CODES);
+}
+// After an MXFP8 forward enqueued its weight passes: remember (flag) or forget.
+void kept_after_fwd(const moe_desc& d, const void* ws, const void* W13, const void* W2) {
+  if (d.dtype != MOE_MXFP8) return;
+  std::lock_guard<std::mutex> lk(g_kept_mu);
+  if (keep_codes(d)) g_kept[ws] = KeptCodes{W13, W2, d.E, d.d, d.d_ff};
+  else g_kept.erase(ws);
+}
+bool kept_ready(const moe_desc& d, const void* ws, const void* W13, const void* W2) {
+  if (!keep_codes(d)) return false;
+  std::lock_guard<std::mutex> lk(g_kept_mu);
+  const auto it = g_kept.find(ws);
+  return it != g_kept.end() && it->second == KeptCodes{W13, W2, d.E, d.d, d.d_ff};
+}
+void kept_forget(const void* ws) {
+  std::lock_guard<std::mutex> lk(g_kept_mu);
+  g_kept.erase(ws);
+}
+
 moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_perm,
                          const void* H13, const void* a, const void* W13, const void* W2,
                          const int32_t* offsets, void* dH13, void* dx_perm, void* dW13, void* dW2,
@@ -310,6 +349,7 @@ moe_status gemm_bwd_body(const moe_desc& d, const void* dy_perm, const void* x_p
     return cu(cudaMemsetAsync(dW2, 0, (size_t)d.E * d.d * d.d_ff * es, s));
   }
   MxWork mx = mx_work(d, ws);
+  mx.w_col_ready = kept_ready(d, ws, W13, W2);
   Weights wt;
   MOE_TRY(tf32_weights(d, W13, W2, ws, s, &wt));
   return gemm_bwd(gshape(d), dy_perm, x_perm, H13, a, wt.W13, wt.W2, offsets, dH13, dx_perm, dW13,
@@ -402,6 +442,7 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
   if (!ws) return MOE_EINVAL;
   if (!aligned16(ws)) return MOE_EALIGN;
   if (ws_bytes < 256) return MOE_EWORKSPACE;
+  kept_forget(ws);
   return cu(cudaMemsetAsync(ws, 0, 256, S(stream)));
 }
 
@@ -462,10 +503,13 @@ moe_status moe_grouped_gemm_fwd(const moe_desc* desc, const void* x_perm, const 
                              desc->E, (int)R_of(*desc), desc->capacity, nullptr, status_ptr(ws),
                              S(stream))));
   MxWork mx = mx_work(*desc, ws);
+  mx.w_col_in_fwd = keep_codes(*desc);
   Weights wt;
   MOE_TRY(tf32_weights(*desc, W13, W2, ws, S(stream), &wt));
-  return gemm_fwd(gshape(*desc), x_perm, wt.W13, wt.W2, offsets, H13, a, y_perm, status_ptr(ws),
-                  S(stream), &mx);
+  MOE_TRY(gemm_fwd(gshape(*desc), x_perm, wt.W13, wt.W2, offsets, H13, a, y_perm,
+                   status_ptr(ws), S(stream), &mx));
+  kept_after_fwd(*desc, ws, W13, W2);
+  return MOE_OK;
 }
 
 moe_status moe_combine(const moe_desc* desc, const void* y_perm, const float* gates,
@@ -628,9 +672,11 @@ moe_status moe_layer_fwd(const moe_desc* desc, const void* x, const float* logit
   const Acts A = acts(d, saved, L, ws);
   MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
   MxWork mx = mx_work(d, ws);
+  mx.w_col_in_fwd = keep_codes(d);
   Weights wt;
   MOE_TRY(tf32_weights(d, W13, W2, ws, s, &wt));
   MOE_TRY(gemm_fwd(gshape(d), A.x_perm, wt.W13, wt.W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+  kept_after_fwd(d, ws, W13, W2);
   float* ys = nullptr;
   if (d.flags & MOE_FLAG_SHARED_EXPERT) {
     // the shared expert over every token, its output in fp32 for the combine to add
@@ -694,7 +740,9 @@ moe_status moe_layer_bwd(const moe_desc* desc, const void* dy, const void* x, co
     // same inputs: bit-identical to the ones the forward used)
     MOE_TRY(dispatch_body(d, x, slot, A.x_perm, st, s));
     MxWork mx = mx_work(d, ws);
+    mx.w_col_in_fwd = keep_codes(d);
     MOE_TRY(gemm_fwd(gshape(d), A.x_perm, wt.W13, wt.W2, offsets, A.H13, A.a, A.y_perm, st, s, &mx));
+    kept_after_fwd(d, ws, W13, W2);
     if (shared)
       MOE_TRY(shared_fwd(gshape(d, d.T), xs, w13_slice(d, wt.W13, es), w2_slice(d, wt.W2, es),
                          A.H13s, A.as, at<float>(ws, w.sh_f32), st, s));

@@ -21,6 +21,7 @@ MOE_OK, MOE_EINVAL, MOE_EALIGN, MOE_EWORKSPACE, MOE_EUNSUPPORTED, MOE_ECUDA, MOE
 MOE_FP32, MOE_BF16, MOE_MXFP8 = 0, 1, 2
 MOE_FLAG_ROUTER, MOE_FLAG_DW_FP32, MOE_FLAG_ACCUM_DW, MOE_FLAG_RECOMPUTE = 1, 2, 4, 8
 MOE_FLAG_SHARED_EXPERT = 16
+MOE_FLAG_MX_KEEP_WEIGHT_CODES = 32       # MXFP8: weight codes of the forward reused
 MOE_FLAG_TEST_WAIT_TIMEOUT = 1 << 30      # test hook: the GEMMs' device waits run out
 MOE_DEV_BAD_INDEX, MOE_DEV_BAD_OFFSETS, MOE_DEV_TIMEOUT, MOE_DEV_CHECK_FAILED = 1, 2, 4, 8
 MOE_ROUTE_NOALLOC_SCRATCH_BYTES = 4 * 1024 * 1024

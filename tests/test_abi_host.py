@@ -53,7 +53,12 @@ def test_descriptor_checks(L, args, code):
 
 
 def test_flag_checks(L):
-    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 32)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16", 64)) == lib.MOE_EINVAL
+    # the weight-code reuse is an MXFP8 option only
+    keep = lib.MOE_FLAG_MX_KEEP_WEIGHT_CODES
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 128, 4, 2, "bf16", keep)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 128, 4, 2, "fp32", keep)) == lib.MOE_EINVAL
+    assert lib.moe_check_desc(lib.make_desc(8, 128, 128, 4, 2, "mxfp8", keep)) == 0
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",
                                             lib.MOE_FLAG_RECOMPUTE)) == 0
     assert lib.moe_check_desc(lib.make_desc(8, 128, 64, 4, 2, "bf16",

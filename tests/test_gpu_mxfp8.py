@@ -185,3 +185,60 @@ def test_full_size_mxfp8_sampled(cuda_lib):
         _, _, dW13, dW2 = oracle.experts_bwd(dYe, Xe, H, A, off, W13e, W2e, mx=True)
         assert rel(g["dW2"][e], dW2[0]) < TOL_MX, e
         assert rel(g["dW13"][e], dW13[0]) < TOL_MX, e
+
+
+# --------------------------------------------------- weight codes kept from the forward
+KEEP = lib.MOE_FLAG_MX_KEEP_WEIGHT_CODES
+
+
+@pytest.mark.parametrize("extra", [0, lib.MOE_FLAG_RECOMPUTE])
+def test_kept_weight_codes_layer_is_bit_identical(cuda_lib, extra):
+    """MOE_FLAG_MX_KEEP_WEIGHT_CODES: the forward quantises the weights both ways in one
+    pass and the backward uses its column-wise codes; every output equals the run
+    without the flag bit for bit (the codes are the same bytes)."""
+    w = Workload("mx", 700, 256, 8, 4, 128, "mxfp8", router=False, skew=False, seed=5)
+    inp = make_inputs(w)
+    _, _, _, y0, g0, st0 = run_layer(w, inp, flags=extra)
+    _, _, _, y1, g1, st1 = run_layer(w, inp, flags=extra | KEEP)
+    assert st0 == 0 and st1 == 0
+    assert torch.equal(y0, y1)
+    for name in ("dx", "d_logits", "dW13", "dW2"):
+        assert torch.equal(g0[name], g1[name]), name
+
+
+def test_kept_weight_codes_follow_the_weights(cuda_lib):
+    """Grouped-GEMM calls with the flag: a backward given the forward's weights reuses
+    their codes; one given other weights (here W * 2 at other addresses) quantises its
+    own.  Both equal the flag-free backward on the same weights bit for bit (reusing the
+    first codes for the second would halve dx)."""
+    T, d, f, E, k = 600, 256, 128, 6, 2
+
+    def bwd(desc, ws, W13_, W2_):
+        R = T * k
+        dH13 = torch.empty(R, 2 * f, dtype=torch.bfloat16, device="cuda")
+        dxp = torch.empty(R, d, dtype=torch.bfloat16, device="cuda")
+        dW13 = torch.empty(E, 2 * f, d, dtype=torch.bfloat16, device="cuda")
+        dW2 = torch.empty(E, d, f, dtype=torch.bfloat16, device="cuda")
+        lib.moe_grouped_gemm_bwd(desc, dyp, xp, H13, a, W13_, W2_, r["offsets"], dH13, dxp, dW13,
+                                 dW2, ws)
+        torch.cuda.synchronize()
+        assert lib.moe_read_device_status(ws) == 0
+        return dH13, dxp, dW13, dW2
+
+    desc, r, W13, W2, ws, xp = make(T, d, f, E, k, None, seed=7)
+    dyp = normal_tensor((T * k, d), seed=23).cuda()
+    H13, a, _ = gpu_fwd(desc, r, W13, W2, ws, xp)
+    ref_same = bwd(desc, ws, W13, W2)
+    W13b, W2b = (W13 * 2).contiguous(), (W2 * 2).contiguous()
+    ref_other = bwd(desc, ws, W13b, W2b)
+
+    kdesc = lib.make_desc(T, d, f, E, k, "mxfp8", KEEP)
+    kws = lib.alloc_workspace(kdesc)
+    gpu_fwd(kdesc, r, W13, W2, kws, xp)
+    got_same = bwd(kdesc, kws, W13, W2)
+    gpu_fwd(kdesc, r, W13, W2, kws, xp)
+    got_other = bwd(kdesc, kws, W13b, W2b)
+    for ref, got in ((ref_same, got_same), (ref_other, got_other)):
+        for x_, y_ in zip(ref, got):
+            assert torch.equal(x_, y_)
+    assert not torch.equal(ref_same[1], ref_other[1])
