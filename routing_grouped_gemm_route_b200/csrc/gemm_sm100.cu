@@ -106,16 +106,23 @@ __device__ __forceinline__ int64_t sf_chunk(const Params::Sf& f, const int32_t* 
 // PAIR: a cluster of two CTAs on two SMs computes 256-row tiles with cta_group::2 MMAs;
 // each CTA loads its 128 rows of A and half of the BN rows of B, so each SM moves a
 // third fewer operand bytes per MMA flop than a lone CTA with a 128 x BN tile.
-template <typename T, typename OutT, int BN, int EPI, bool PAIR = false, int MODE = RAGGED_M>
+// KAT: 128-byte K atoms per stage.  Two for the 16-bit ragged-M pair GEMMs whose K allows
+// it: a stage then carries eight MMAs instead of four for the same per-stage cost (the
+// barrier round trip and the TMA issue of each stage weigh as much as its bytes).
+template <typename T, typename OutT, int BN, int EPI, bool PAIR = false, int MODE = RAGGED_M,
+          int KAT = 1>
 struct Cfg {
   static constexpr int ES = sizeof(T);
-  static constexpr int KB = 128 / ES;     // K elements per stage (one 128-byte swizzle row)
+  static constexpr int KA = 128 / ES;     // K elements of one 128-byte swizzle row (an atom)
+  static constexpr int KB = KA * KAT;     // K elements per stage
   static constexpr int MNB = 128 / ES;    // M/N elements per 128-byte block (M/N-major tiles)
   static constexpr int UK = 32 / ES;      // K of one MMA instruction
   static constexpr int TM = PAIR ? 2 * BM : BM;     // tile rows (M) of the whole cluster
   static constexpr int BNC = PAIR ? BN / 2 : BN;    // rows of B held by one CTA
-  static constexpr int A_BYTES = BM * 128;
-  static constexpr int B_BYTES = BNC * 128;
+  static constexpr int A_ATOM = BM * 128;           // one K atom of A (K-major)
+  static constexpr int B_ATOM = BNC * 128;          // one K atom of B (K-major)
+  static constexpr int A_BYTES = A_ATOM * KAT;
+  static constexpr int B_BYTES = B_ATOM * KAT;
   static constexpr int STAGE = A_BYTES + B_BYTES;
   // MXFP8: per stage, one 512-byte scale chunk for this CTA's 128 rows of A and one per
   // 128 rows of the whole BN of B (in a pair each CTA's MMA half reads all of B's scales
@@ -322,13 +329,14 @@ __device__ __forceinline__ void store_packed32(bf16* dst, const uint32_t* w) {
   for (int j = 0; j < 4; ++j) stg16(dst + 8 * j, make_uint4(w[4 * j], w[4 * j + 1], w[4 * j + 2], w[4 * j + 3]));
 }
 
-template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
-__global__ void __launch_bounds__(Cfg<T, OutT, BN, EPI, PAIR, MODE>::THREADS, 1)
+template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR,
+          int KAT>
+__global__ void __launch_bounds__(Cfg<T, OutT, BN, EPI, PAIR, MODE, KAT>::THREADS, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO, const __grid_constant__ CUtensorMap tmO2,
                     const __grid_constant__ CUtensorMap tmI, const __grid_constant__ CUtensorMap tmSA,
                     const __grid_constant__ CUtensorMap tmSB, const Params p) {
-  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
+  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE, KAT>;
   using ActT = typename std::conditional<sizeof(T) == 4, float, bf16>::type;  // epilogue inputs
   constexpr bool kTF32 = sizeof(T) == 4;
   constexpr bool kMX = C::MX;
@@ -339,6 +347,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
   static_assert(!B_MN || C::BNC % C::MNB == 0, "an M/N-major B half is whole 128-byte blocks");
   static_assert(BN == 64 || BN == 128 || BN == 256, "tile width");
   static_assert(MODE == RAGGED_M || (A_MN && B_MN && EPI == EPI_STORE), "wgrad layout");
+  static_assert(KAT == 1 || (MODE == RAGGED_M && PAIR && !A_MN && !kMX), "two-atom stages");
+  static_assert(KAT == 1 || C::STAGES >= 3, "two-atom stages need a ring of three");
 
   // a programmatic dependent of the previous kernel: its writes are visible from here on
   pdl_wait();
@@ -498,20 +508,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
                    static_cast<int>(sf_chunk(p.sfb, p.tile_pref, tl.e, tl.n0 + 128 * j, kb)));
           }
           if (MODE == RAGGED_M) {
-            load(sA, &tmA, k0, tl.row0 + arow);
+#pragma unroll
+            for (int at = 0; at < KAT; ++at)
+              load(sA + at * C::A_ATOM, &tmA, k0 + at * C::KA, tl.row0 + arow);
             const int brow = tl.e * p.b_rows_per_expert;
             if (!B_MN) {
-              if (EPI == EPI_SWIGLU_FWD) {
-                // B rows: the gate block W1[h0, h0+BN/2) then the up block W3[h0, ...)
-                const int h0 = tl.n0 / 2;
-                if (PAIR) {
-                  load(sB, &tmB, k0, brow + (rank ? p.f : 0) + h0);
+#pragma unroll
+              for (int at = 0; at < KAT; ++at) {
+                uint8_t* sBa = sB + at * C::B_ATOM;
+                const int ka = k0 + at * C::KA;
+                if (EPI == EPI_SWIGLU_FWD) {
+                  // B rows: the gate block W1[h0, h0+BN/2) then the up block W3[h0, ...)
+                  const int h0 = tl.n0 / 2;
+                  if (PAIR) {
+                    load(sBa, &tmB, ka, brow + (rank ? p.f : 0) + h0);
+                  } else {
+                    load(sBa, &tmB, ka, brow + h0);
+                    load(sBa + (BN / 2) * 128, &tmB, ka, brow + p.f + h0);
+                  }
                 } else {
-                  load(sB, &tmB, k0, brow + h0);
-                  load(sB + (BN / 2) * 128, &tmB, k0, brow + p.f + h0);
+                  load(sBa, &tmB, ka, brow + tl.n0 + bcol);
                 }
-              } else {
-                load(sB, &tmB, k0, brow + tl.n0 + bcol);
               }
             } else {
 #pragma unroll
@@ -597,10 +614,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_consta
               else tmem_cp_scales(tmem_base + col + 4 * j, sdesc(src + 512 * j, 128, 128, 0));
             }
           }
+          // K-major operands: MMA kk reads atom kk / KPA at K offset kk % KPA; M/N-major
+          // ones hold the stage's K rows contiguously in each 128-byte block
+          constexpr int KPA = C::KA / C::UK;
 #pragma unroll
           for (int kk = 0; kk < C::KB / C::UK; ++kk) {
-            const uint64_t ad = a_desc0 + so + kk * A_STEP;
-            const uint64_t bd = b_desc0 + so + kk * B_STEP;
+            const uint32_t a_off = A_MN ? kk * A_STEP
+                                        : (kk / KPA) * (C::A_ATOM >> 4) + (kk % KPA) * A_STEP;
+            const uint32_t b_off = B_MN ? kk * B_STEP
+                                        : (kk / KPA) * (C::B_ATOM >> 4) + (kk % KPA) * B_STEP;
+            const uint64_t ad = a_desc0 + so + a_off;
+            const uint64_t bd = b_desc0 + so + b_off;
             const uint32_t accum = (kb | kk) != 0 ? 1u : 0u;
             if constexpr (kMX) {
               if (PAIR) umma_mx_pair(d_tmem, ad, bd, IDESC | idesc_sf_ids(kk, kk), sfa_t, sfb_t, accum);
@@ -1042,12 +1066,13 @@ static bool make_tmap_mn3(CUtensorMap* m, const void* base, int es_, uint64_t co
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR>
+template <typename T, typename OutT, int BN, bool A_MN, bool B_MN, int MODE, int EPI, bool PAIR,
+          int KAT = 1>
 static moe_status launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& to,
                          const CUtensorMap& to2, const CUtensorMap& ti, const CUtensorMap& tsa,
                          const CUtensorMap& tsb, const Params& p, int max_tiles, cudaStream_t s) {
-  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE>;
-  auto kern = grouped_gemm_kernel<T, OutT, BN, A_MN, B_MN, MODE, EPI, PAIR>;
+  using C = Cfg<T, OutT, BN, EPI, PAIR, MODE, KAT>;
+  auto kern = grouped_gemm_kernel<T, OutT, BN, A_MN, B_MN, MODE, EPI, PAIR, KAT>;
   const size_t smem = C::smem_bytes(p.E);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
@@ -1122,19 +1147,20 @@ static bool sf_maps(const MxRefs& mx, bool is_mx, const CUtensorMap& dummy, CUte
   return make_sf_map(tsa, mx.a.base, mx.a_chunks) && make_sf_map(tsb, mx.b.base, mx.b_chunks);
 }
 
-template <typename T, bool B_MN, int EPI, int BN, bool PAIR, typename OutT = T>
+template <typename T, bool B_MN, int EPI, int BN, bool PAIR, typename OutT = T, int KAT = 1>
 static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B, int N,
                         int b_rows_per_expert, int b_cols, void* out, int out_cols, void* out_a,
                         const void* aux, const int32_t* offsets, int* status, cudaStream_t s,
                         const MxRefs& mx = MxRefs()) {
-  using C = Cfg<T, OutT, BN, EPI, PAIR>;
+  using C = Cfg<T, OutT, BN, EPI, PAIR, RAGGED_M, KAT>;
   constexpr int ES = sizeof(T);
   constexpr int OES = sizeof(OutT);
+  if (K % C::KB != 0) return MOE_EINVAL;
   CUtensorMap ta, tb, to, to2, ti;
-  if (!make_tmap(&ta, A, ES, K, g.R, C::KB, BM, Box::KMajor)) return MOE_ECUDA;
+  if (!make_tmap(&ta, A, ES, K, g.R, C::KA, BM, Box::KMajor)) return MOE_ECUDA;
   if (!B_MN) {
     const int box_rows = EPI == EPI_SWIGLU_FWD ? BN / 2 : C::BNC;
-    if (!make_tmap(&tb, B, ES, K, (uint64_t)g.E * b_rows_per_expert, C::KB, box_rows,
+    if (!make_tmap(&tb, B, ES, K, (uint64_t)g.E * b_rows_per_expert, C::KA, box_rows,
                    Box::KMajor))
       return MOE_ECUDA;
   } else {
@@ -1172,7 +1198,7 @@ static moe_status run_m(const GemmShape& g, const void* A, int K, const void* B,
   p.wait_ns = g.test_stall ? 10000000ull : kWaitLimitNs;
   CUtensorMap tsa, tsb;
   if (!sf_maps(mx, C::MX, ta, &tsa, &tsb)) return MOE_ECUDA;
-  return launch<T, OutT, BN, false, B_MN, RAGGED_M, EPI, PAIR>(
+  return launch<T, OutT, BN, false, B_MN, RAGGED_M, EPI, PAIR, KAT>(
       ta, tb, to, to2, ti, tsa, tsb, p, ragged_m_tiles(g, N / BN, C::TM), s);
 }
 
@@ -1227,11 +1253,18 @@ static moe_status run_k(const GemmShape& g, const void* G, int M, const void* X,
 // CTA pairs for the 16-bit kernels; the TF32 kernels run one CTA per tile.
 template <typename T>
 constexpr bool kPair = sizeof(T) == 2;
+// K atoms per stage of the 16-bit pair forward and FC1-dgrad GEMMs (Cfg)
+constexpr int kWideAtoms = 2;
 
 template <typename T>
 static moe_status fc1_fwd(const GemmShape& g, const void* x_perm, const void* W13,
                           const int32_t* off, void* H13, void* a, int* st, cudaStream_t s) {
   // accumulator grid: 2f columns, each tile = BN/2 gate columns + the matching BN/2 up columns
+  if constexpr (kPair<T>) {
+    if (g.f % 128 == 0 && g.d % 128 == 0)
+      return run_m<T, false, EPI_SWIGLU_FWD, 256, true, T, kWideAtoms>(
+          g, x_perm, g.d, W13, 2 * g.f, 2 * g.f, g.d, H13, 2 * g.f, a, nullptr, off, st, s);
+  }
   if (g.f % 128 == 0)
     return run_m<T, false, EPI_SWIGLU_FWD, 256, kPair<T>>(g, x_perm, g.d, W13, 2 * g.f, 2 * g.f,
                                                            g.d, H13, 2 * g.f, a, nullptr, off, st,
@@ -1243,6 +1276,11 @@ static moe_status fc1_fwd(const GemmShape& g, const void* x_perm, const void* W1
 template <typename T, typename OutT = T>
 static moe_status fc2_fwd(const GemmShape& g, const void* a, const void* W2, const int32_t* off,
                           void* y_perm, int* st, cudaStream_t s) {
+  if constexpr (kPair<T> && sizeof(OutT) == 2) {   // (fp32 staging leaves room for two stages)
+    if (g.d % 256 == 0 && g.f % 128 == 0)
+      return run_m<T, false, EPI_STORE, 256, true, OutT, kWideAtoms>(
+          g, a, g.f, W2, g.d, g.d, g.f, y_perm, g.d, nullptr, nullptr, off, st, s);
+  }
   if (g.d % 256 == 0)
     return run_m<T, false, EPI_STORE, 256, kPair<T>, OutT>(g, a, g.f, W2, g.d, g.d, g.f, y_perm,
                                                             g.d, nullptr, nullptr, off, st, s);
@@ -1271,6 +1309,11 @@ template <typename T, typename OutT = T>
 static moe_status fc1_dgrad(const GemmShape& g, const void* dH13, const void* W13,
                             const int32_t* off, void* dx_perm, int* st, cudaStream_t s) {
   // dX = dH13 . W13_e: K = 2f, N = d; B[n, k] = W13[e*2f + k, n] (M/N-major)
+  if constexpr (kPair<T> && sizeof(OutT) == 2) {
+    if (g.d % 256 == 0)   // K = 2f, a multiple of 128
+      return run_m<T, true, EPI_STORE, 256, true, OutT, kWideAtoms>(
+          g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d, dx_perm, g.d, nullptr, nullptr, off, st, s);
+  }
   if (g.d % 256 == 0)
     return run_m<T, true, EPI_STORE, 256, kPair<T>, OutT>(g, dH13, 2 * g.f, W13, g.d, 2 * g.f, g.d,
                                                            dx_perm, g.d, nullptr, nullptr, off, st,
