@@ -272,8 +272,13 @@ topk_kernel(const float* __restrict__ logits, int T, int E, int k, int32_t* __re
 // CTA waits for another and no separate scan runs: every CTA reads the histogram
 // (nrows x E int32, 128 KB at 16384 tokens and 128 experts) from L2.
 constexpr int kSlotScanRows = 512;
+// 1024 threads: all 32 warps sum the histogram rows (a few rows each, all loads in
+// flight at once), the first kWarps warps (one token a lane) place the CTA's tokens
+constexpr int kSlotWarps = 32;
+constexpr int kSlotThreads = kSlotWarps * 32;
+static_assert(kSlotWarps >= kWarps, "the token warps are the first warps");
 template <int NPL>
-__global__ void __launch_bounds__(kWarps * 32) slot_kernel(
+__global__ void __launch_bounds__(kSlotThreads) slot_kernel(
     const int32_t* __restrict__ topk_idx, const float* __restrict__ gates,
     int32_t* __restrict__ offsets, const int32_t* __restrict__ cta_base,
     const int32_t* __restrict__ hist, int nrows, int32_t* __restrict__ counts, int T, int E,
@@ -283,20 +288,21 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
   unsigned* masks = s_mem;                                          // [kWarps][E]
   int* wbase = reinterpret_cast<int*>(s_mem + kWarps * E);          // [kWarps][E]
   int* s_off = wbase + kWarps * E;                                  // [E] (NPL > 0)
+  int* s_pre = s_off + E;                                           // [kSlotWarps][E]
+  int* s_tot = s_pre + kSlotWarps * E;                              // [kSlotWarps][E]
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // launched as a programmatic dependent of the top-k kernel: everything it wrote is
   // visible from here on
   pdl_wait();
   int start = 0;                     // thread e: the CTA's first row in expert e
   if constexpr (NPL > 0) {
-    // per-warp sums of the rows before this CTA and of all rows, into masks / wbase
-    // (eight rows of loads in flight per warp)
+    // per-warp sums of the rows before this CTA and of all rows, into s_pre / s_tot
     const int r_cta = blockIdx.x * kHistRowsPerCta;
     int pre[NPL], tot[NPL];
 #pragma unroll
     for (int c = 0; c < NPL; ++c) pre[c] = tot[c] = 0;
-#pragma unroll 8
-    for (int r = warp; r < nrows; r += kWarps) {
+#pragma unroll 4
+    for (int r = warp; r < nrows; r += kSlotWarps) {
 #pragma unroll
       for (int c = 0; c < NPL; ++c) {
         const int e = c * 32 + lane;
@@ -309,19 +315,19 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
     for (int c = 0; c < NPL; ++c) {
       const int e = c * 32 + lane;
       if (e < E) {
-        reinterpret_cast<int*>(masks)[warp * E + e] = pre[c];
-        wbase[warp * E + e] = tot[c];
+        s_pre[warp * E + e] = pre[c];
+        s_tot[warp * E + e] = tot[c];
       }
     }
     __syncthreads();
     // thread e: base and count of expert e; offsets = exclusive scan of the counts
-    const int e = threadIdx.x;                 // E <= 256 = blockDim.x
+    const int e = threadIdx.x;                 // E <= 256 < blockDim.x
     int base = 0, cnt = 0;
     if (e < E) {
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) {
-        base += reinterpret_cast<int*>(masks)[w * E + e];
-        cnt += wbase[w * E + e];
+#pragma unroll 8
+      for (int w = 0; w < kSlotWarps; ++w) {
+        base += s_pre[w * E + e];
+        cnt += s_tot[w * E + e];
       }
     }
     int incl = cnt;                            // warp-inclusive scan, then across warps
@@ -330,13 +336,12 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
       const int v = __shfl_up_sync(0xffffffffu, incl, o);
       if (lane >= o) incl += v;
     }
-    __shared__ int s_warp[kWarps];
-    __syncthreads();                           // masks / wbase reads done
+    __shared__ int s_warp[kSlotWarps];
     if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
     int before = 0, total = 0;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
+#pragma unroll 8
+    for (int w = 0; w < kSlotWarps; ++w) {
       before += w < warp ? s_warp[w] : 0;
       total += s_warp[w];
     }
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(kWarps * 32) slot_kernel(
   for (int i = threadIdx.x; i < kWarps * E; i += blockDim.x) masks[i] = 0u;
   __syncthreads();
   const int t = blockIdx.x * kRouteTokensPerCta + threadIdx.x;
-  const bool live = t < T;
+  const bool live = threadIdx.x < kRouteTokensPerCta && t < T;   // warps 0 .. kWarps-1
   if (live) {
     for (int j = 0; j < k; ++j) {
       const int e = topk_idx[(int64_t)t * k + j];
@@ -534,12 +539,8 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
     scan_kernel<<<1, kScanThreads, 0, s>>>(hist, nrows, E, C, cta_base, counts, offsets);
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
   }
-  const size_t smem = (size_t(2) * kWarps * E + (in_slot ? E : 0)) * sizeof(int);
-  if (smem > 48 * 1024) {
-    err = cudaFuncSetAttribute(slot_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
-    if (err != cudaSuccess) return err;
-  }
+  const size_t smem =
+      (size_t(2) * kWarps * E + (in_slot ? E + size_t(2) * kSlotWarps * E : 0)) * sizeof(int);
   if (C > 0 && T > 0) {
     // padded layout: rows no token fills are marked (token -1, gate 0)
     const size_t rows = (size_t)E * C;
@@ -551,7 +552,7 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   // padded layout's memsets come between them: then it is an ordinary launch.)
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(ctas, 1, 1);
-  cfg.blockDim = dim3(kWarps * 32, 1, 1);
+  cfg.blockDim = dim3(kSlotThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
@@ -560,6 +561,11 @@ cudaError_t launch_route(const moe_desc& d, const float* logits, int32_t* topk_i
   cfg.attrs = attr;
   cfg.numAttrs = C > 0 ? 0 : 1;
   auto go = [&](auto kern) {
+    if (smem > 48 * 1024) {
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem));
+      if (e != cudaSuccess) return e;
+    }
     return cudaLaunchKernelEx(&cfg, kern, (const int32_t*)topk_idx, (const float*)gates, offsets,
                               (const int32_t*)cta_base, (const int32_t*)hist, nrows, counts, T, E,
                               k, C, slot, row_token, row_gate, status);
