@@ -114,6 +114,34 @@ def workload_desc(w):
                               ("Zipf-skewed " if w.skew else "") + "iid N(0,1) routing logits"))
 
 
+def stage_launches(w, keep_codes: bool) -> dict:
+    """This library's kernel launches per call of each bench stage (the line's
+    `gpu_launches` claim), following the library's own dispatch: routing is top-k + slots
+    (+ a scan launch above 256 experts); the fp32 GEMM calls first round both weights to
+    TF32 copies; MXFP8 adds the scale-prefix and quantiser launches (the backward's two
+    weight passes are skipped when the forward kept the weight codes); the wgrad calls
+    build their per-expert tensor maps with one launch."""
+    mx, f32 = w.dtype == "mxfp8", w.dtype == "fp32"
+    route = 3 if w.E > 256 else 2
+    if mx:    # prefix, x rowwise, W13, FC1 (+ a's codes), W2, FC2
+        fwd, bwd = 6, (10 if keep_codes else 12)
+    else:     # (2 TF32 weight copies) FC1, FC2 | (2 copies) maps, FC2 dgrad, FC2 wgrad, FC1 dgrad, FC1 wgrad
+        fwd, bwd = (4, 7) if f32 else (2, 5)
+    # router: one GEMM; its backward: fp32 two CUDA-core GEMMs; bf16 a bf16 copy of
+    # d_logits, two tensor-core GEMMs and their maps, and the add into dx (E % 64 == 0),
+    # else two CUDA-core GEMMs and the add
+    router_bwd = 2 if f32 else (5 if w.E % 64 == 0 else 3)
+    n = {"router": 1, "route": route, "dispatch": 1, "gemm_fwd": fwd, "combine": 1,
+         "combine_bwd": 1, "gemm_bwd": bwd, "dispatch_bwd": 1, "router_bwd": router_bwd}
+    n["re_dispatch"], n["re_gemm_fwd"] = n["dispatch"], n["gemm_fwd"]
+    # whole-layer calls (the shared-expert runs): routing, dispatch, 2 GEMMs, 2 shared-expert
+    # GEMMs, combine (+ router); combine backward, the backward GEMMs, 5 shared-expert
+    # launches, unpermute (+ router: bf16 copy, maps, 2 GEMMs)
+    n["layer_fwd"] = route + 1 + fwd + 2 + 1 + (1 if w.router else 0)
+    n["layer_bwd"] = 1 + bwd + 5 + 1 + (4 if w.router else 0)
+    return n
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons during the timed region."""
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -547,16 +575,7 @@ def main():
     if w.router:
         stages = ["router"] + stages + ["router_bwd"]
     mx = w.dtype == "mxfp8"
-    # GEMM stages: bf16/fp32 fwd = 2 GEMMs, bwd = tensor-map builder + 4 GEMMs; MXFP8 adds
-    # the quantisers (one segment prefix per stage, one launch per quantised operand)
-    launches = {"router": 1, "route": 3, "dispatch": 1, "gemm_fwd": 7 if mx else 2,
-                "combine": 1, "combine_bwd": 1, "gemm_bwd": 12 if mx else 5, "dispatch_bwd": 1,
-                "router_bwd": 3}
-    launches["re_dispatch"], launches["re_gemm_fwd"] = launches["dispatch"], launches["gemm_fwd"]
-    # whole-layer calls: route 3, dispatch 1, GEMMs 2, shared 2, combine 1 (+ router 1);
-    # combine-bwd 1, GEMMs 5, shared 5, unpermute 1 (+ router: bf16 copy, maps, 2 GEMMs)
-    launches["layer_fwd"] = 9 + (1 if w.router else 0)
-    launches["layer_bwd"] = 12 + (4 if w.router else 0)
+    launches = stage_launches(w, bool(flags & lib.MOE_FLAG_MX_KEEP_WEIGHT_CODES))
 
     def run_stage(name):
         if name == "router":

@@ -105,3 +105,20 @@ def test_nvml_sampler_summary_and_absence(monkeypatch):
     r = s.stop()
     assert r["sm_mhz"] == 1475 and r["sm_mhz_min"] == 1400 and r["samples"] == 4
     assert r["power_w_max"] == 1000.0 and r["power_w_median"] == 992.5
+
+
+def test_stage_launch_counts_match_the_launch_lists():
+    """The per-step launch counts of the bench's stages (the line's gpu_launches claim):
+    13 for the headline bf16 step and 22 for the MXFP8 step with the weight codes kept,
+    the totals the ncu launch lists of those commands show per step."""
+    from routing_grouped_gemm_route_b200.inputs import WORKLOADS
+    steps = ["route", "dispatch", "gemm_fwd", "combine", "combine_bwd", "gemm_bwd",
+             "dispatch_bwd"]
+    n = bench.stage_launches(WORKLOADS["e128_bf16"], False)
+    assert sum(n[s] for s in steps) == 13
+    n = bench.stage_launches(WORKLOADS["e128_mxfp8_large"], True)
+    assert sum(n[s] for s in steps) == 22
+    assert bench.stage_launches(WORKLOADS["e128_mxfp8_large"], False)["gemm_bwd"] == 12
+    # the tiny fp32 workload runs the router: + 1 forward, + 2 backward; TF32 weight copies
+    n = bench.stage_launches(WORKLOADS["tiny_fp32"], False)
+    assert sum(n[s] for s in ["router"] + steps + ["router_bwd"]) == 20
